@@ -1,0 +1,274 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each check is chosen so that a plausible slip in the oracle (a wrong causal bound, a
+dropped head, a window off by one, a reversed tie rule, a transposed weight, log2 instead
+of ln) fails at least one of them:
+
+* library routines in special cases: torch scaled_dot_product_attention (fp64, explicit
+  mask), torch.softmax, numpy matmul;
+* closed forms: all-zero keys, a two-key row, constant values;
+* invariants the selection rule fixes: forced window, uniqueness, causality, the count
+  min(t+1, window+topk), the probability mass sum_j score(t, j) = H;
+* brute force: the chosen older tokens maximise the summed score over all subsets of the
+  same size (tiny rows), with scores from an independent torch computation.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import f32_to_bf16_bits, bf16_bits_to_f32
+
+
+def _rand_bf16(rng, shape, std=1.0):
+    return f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * np.float32(std))
+
+
+def _t64(bits):
+    return torch.from_numpy(bf16_bits_to_f32(bits).astype(np.float64))
+
+
+def _causal_mask(Lq, Lk):
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    return j <= (Lk - Lq + i)
+
+
+def _torch_dense(q, k, v, scale):
+    """Reference by torch SDPA (fp64): q [B,Lq,H,d], k/v [B,Lk,d] -> out [B,Lq,H,d]."""
+    Q = _t64(q).permute(0, 2, 1, 3)                       # B,H,Lq,d
+    K = _t64(k)[:, None].expand(-1, q.shape[2], -1, -1)   # B,H,Lk,d
+    V = _t64(v)[:, None].expand(-1, q.shape[2], -1, -1)
+    m = _causal_mask(q.shape[1], k.shape[1])
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=m, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def _torch_probs(q, k, scale):
+    """torch.softmax probabilities [B,H,Lq,Lk] with the causal mask (fp64)."""
+    Q = _t64(q).permute(0, 2, 1, 3)
+    K = _t64(k)[:, None]
+    s = scale * (Q @ K.transpose(-1, -2))
+    s = s.masked_fill(~_causal_mask(q.shape[1], k.shape[1]), float("-inf"))
+    return torch.softmax(s, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("B,Lq,Lk,H,d", [(2, 37, 37, 3, 8), (1, 5, 41, 4, 16), (3, 1, 29, 2, 8)])
+def test_attention_matches_torch_sdpa(B, Lq, Lk, H, d):
+    rng = np.random.default_rng(1)
+    q, k, v = _rand_bf16(rng, (B, Lq, H, d)), _rand_bf16(rng, (B, Lk, d)), _rand_bf16(rng, (B, Lk, d))
+    scale = 1.0 / math.sqrt(d)
+    r = oracle.full_attn_select(q, k, v, scale, 4, 6)
+    ref = _torch_dense(q, k, v, scale).reshape(B * Lq, H, d)
+    np.testing.assert_allclose(r["out"], ref, rtol=0, atol=1e-12)
+
+
+def test_closed_form_zero_keys():
+    """K == 0: every logit is 0, so p = 1/(t+1), lse = ln(t+1), out = mean(v_0..v_t)."""
+    rng = np.random.default_rng(2)
+    B, L, H, d = 1, 20, 3, 8
+    q = _rand_bf16(rng, (B, L, H, d))
+    k = np.zeros((B, L, d), np.uint16)
+    v = _rand_bf16(rng, (B, L, d))
+    r = oracle.full_attn_select(q, k, v, 0.3, 4, 5, want_score=True)
+    vf = bf16_bits_to_f32(v).astype(np.float64)[0]
+    for t in range(L):
+        np.testing.assert_allclose(r["lse"][t], math.log(t + 1), atol=1e-13)
+        np.testing.assert_allclose(r["out"][t], np.broadcast_to(vf[: t + 1].mean(0), (H, d)), atol=1e-13)
+        np.testing.assert_allclose(r["score"][t, : t + 1], H / (t + 1), atol=1e-13)
+        # all scores tie -> lower indices win: the older picks are 0..min(k, n_old)-1
+        n_old = max(0, t - 4 + 1)
+        picks = sorted(set(r["idx"][t][r["idx"][t] >= 0]) - set(range(max(0, t - 3), t + 1)))
+        assert picks == list(range(min(5, n_old)))
+
+
+def test_closed_form_two_keys():
+    """One head, q = e0, keys a*e0 and b*e0: lse = ln(exp(s a) + exp(s b)) at t = 1."""
+    d = 8
+    a, b, c = 1.5, -0.75, 2.0
+    q = np.zeros((1, 2, 1, d), np.float32); q[0, :, 0, 0] = 1.0
+    k = np.zeros((1, 2, d), np.float32); k[0, 0, 0] = a; k[0, 1, 0] = b
+    v = np.zeros((1, 2, d), np.float32); v[0, 0, :] = 1.0; v[0, 1, :] = c
+    s = 0.5
+    r = oracle.full_attn_select(f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v), s, 1, 1)
+    lse1 = math.log(math.exp(s * a) + math.exp(s * b))
+    assert abs(r["lse"][1, 0] - lse1) < 1e-14
+    assert abs(r["lse"][0, 0] - s * a) < 1e-15
+    p0 = math.exp(s * a - lse1)
+    np.testing.assert_allclose(r["out"][1, 0], p0 * 1.0 + (1 - p0) * c, atol=1e-14)
+
+
+def test_constant_values_give_constant_output():
+    rng = np.random.default_rng(3)
+    B, L, H, d = 2, 33, 4, 8
+    q, k = _rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d))
+    v = f32_to_bf16_bits(np.full((B, L, d), 0.625, np.float32))
+    r = oracle.full_attn_select(q, k, v, 0.35, 4, 4)
+    np.testing.assert_allclose(r["out"], 0.625, atol=1e-13)
+
+
+def test_score_mass_and_softmax_probabilities():
+    """score(t, j) equals torch's softmax summed over heads; its row mass is H."""
+    rng = np.random.default_rng(4)
+    B, L, H, d = 2, 24, 5, 16
+    q, k, v = _rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d)), _rand_bf16(rng, (B, L, d))
+    r = oracle.full_attn_select(q, k, v, 0.25, 4, 6, want_score=True)
+    p = _torch_probs(q, k, 0.25)                  # B,H,L,L
+    ref = p.sum(1).reshape(B * L, L)
+    np.testing.assert_allclose(r["score"], ref, atol=1e-13)
+    np.testing.assert_allclose(r["score"].sum(1), H, atol=1e-12)
+
+
+def test_single_head_ranking_equals_logit_ranking():
+    """H = 1: softmax is monotone, so the older picks are the top logits (numpy argsort)."""
+    rng = np.random.default_rng(5)
+    L, d, W, K = 60, 16, 8, 10
+    q, k, v = _rand_bf16(rng, (1, L, 1, d)), _rand_bf16(rng, (1, L, d)), _rand_bf16(rng, (1, L, d))
+    r = oracle.full_attn_select(q, k, v, 0.2, W, K)
+    qf = bf16_bits_to_f32(q)[0, :, 0].astype(np.float64)
+    kf = bf16_bits_to_f32(k)[0].astype(np.float64)
+    for t in range(L):
+        n_old = t - W + 1
+        sel = set(r["idx"][t][r["idx"][t] >= 0].tolist())
+        if n_old <= 0:
+            assert sel == set(range(t + 1))
+            continue
+        logit = kf[:n_old] @ qf[t]
+        order = np.lexsort((np.arange(n_old), -logit))[: min(K, n_old)]
+        assert sel == set(order.tolist()) | set(range(t - W + 1, t + 1))
+
+
+def test_planted_direction_ranking():
+    """H = 1, q = u and k_j = alpha_j u: the picks are the tokens with the largest alpha."""
+    d, L, W, K = 8, 30, 4, 5
+    alpha = np.array([((j * 7) % 30) / 8.0 - 1.5 for j in range(L)], np.float32)  # distinct, bf16-exact
+    u = np.zeros(d, np.float32); u[3] = 1.0
+    q = np.broadcast_to(u, (1, L, 1, d)).copy()
+    k = (alpha[:, None] * u[None, :])[None]
+    v = np.zeros((1, L, d), np.float32)
+    r = oracle.full_attn_select(f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v), 1.0, W, K)
+    t = L - 1
+    n_old = t - W + 1
+    expect = set(np.argsort(-alpha[:n_old], kind="stable")[:K].tolist()) | set(range(t - W + 1, t + 1))
+    assert set(r["idx"][t][r["idx"][t] >= 0].tolist()) == expect
+
+
+@pytest.mark.parametrize("W,K", [(4, 1), (4, 3), (4, 8), (1, 2), (0, 3)])
+def test_selection_brute_force_subsets(W, K):
+    """Tiny rows: the older picks maximise the summed (torch) score over all same-size subsets."""
+    rng = np.random.default_rng(10 + W * 10 + K)
+    B, L, H, d = 1, 12, 3, 8
+    q, k, v = _rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d)), _rand_bf16(rng, (B, L, d))
+    r = oracle.full_attn_select(q, k, v, 0.4, W, K)
+    sc = _torch_probs(q, k, 0.4).sum(1)[0]        # [L, L]
+    for t in range(L):
+        n_old = t - W + 1
+        sel = set(r["idx"][t][r["idx"][t] >= 0].tolist())
+        window = set(range(max(0, t - W + 1), t + 1))
+        assert window <= sel
+        older = sorted(sel - window)
+        m = min(K, max(0, n_old))
+        assert len(older) == m
+        if m == 0:
+            continue
+        best = max(itertools.combinations(range(n_old), m), key=lambda s: sum(sc[t, j] for j in s))
+        assert older == sorted(best)
+
+
+def test_selection_invariants_on_planted_workload():
+    wl = synth.small("tiny_prefill", Lq=300, Lk=300)
+    g = synth.SyntheticInputs(wl)
+    W, K = 32, 64
+    r = oracle.full_attn_select(g.q, g.k, g.v, wl.scale, W, K, want_score=True)
+    S = W + K
+    assert r["idx"].shape == (300, S)
+    for t in range(300):
+        row = r["idx"][t]
+        valid = row[row >= 0]
+        assert len(valid) == min(t + 1, S)
+        assert (row[len(valid):] == -1).all()
+        assert (np.diff(valid) > 0).all()                       # ascending, unique
+        assert valid.max() <= t and valid.min() >= 0            # causal
+        assert set(range(max(0, t - W + 1), t + 1)) <= set(valid.tolist())
+        # every older pick scores at least as high as every older non-pick
+        older = [j for j in valid if j <= t - W]
+        rest = sorted(set(range(max(0, t - W + 1))) - set(older))
+        if older and rest:
+            assert r["score"][t, older].min() >= r["score"][t, rest].max()
+    np.testing.assert_allclose(r["score"].sum(1), wl.H, atol=1e-11)
+
+
+def test_sparse_equals_dense_when_everything_fits():
+    """With window + topk >= t + 1 the selection is the whole causal row, so sparse == dense."""
+    rng = np.random.default_rng(6)
+    B, L, H, d = 2, 20, 3, 8
+    q, k, v = _rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d)), _rand_bf16(rng, (B, L, d))
+    q2 = _rand_bf16(rng, (B, L, H, d))
+    full = oracle.full_attn_select(q, k, v, 0.3, 8, 12)
+    idx = full["idx"].reshape(B, L, 20)
+    sp = oracle.sparse_attn(q2, k, v, idx, 0.3)
+    np.testing.assert_allclose(sp["out"], _torch_dense(q2, k, v, 0.3).reshape(B * L, H, d), atol=1e-12)
+
+
+def test_sparse_matches_sdpa_with_index_mask():
+    rng = np.random.default_rng(7)
+    B, Lq, Lk, H, d, S = 2, 6, 50, 4, 16, 9
+    q, k, v = _rand_bf16(rng, (B, Lq, H, d)), _rand_bf16(rng, (B, Lk, d)), _rand_bf16(rng, (B, Lk, d))
+    idx = np.full((B, Lq, S), -1, np.int32)
+    for b in range(B):
+        for i in range(Lq):
+            n = rng.integers(1, S + 1)
+            idx[b, i, :n] = rng.choice(Lk, size=n, replace=False)
+            rng.shuffle(idx[b, i])
+    sp = oracle.sparse_attn(q, k, v, idx, 0.25)
+    mask = torch.zeros(B, 1, Lq, Lk, dtype=torch.bool)
+    for b in range(B):
+        for i in range(Lq):
+            for j in idx[b, i]:
+                if j >= 0:
+                    mask[b, 0, i, j] = True
+    Q = _t64(q).permute(0, 2, 1, 3)
+    K = _t64(k)[:, None].expand(-1, H, -1, -1)
+    V = _t64(v)[:, None].expand(-1, H, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=0.25)
+    np.testing.assert_allclose(sp["out"], ref.permute(0, 2, 1, 3).reshape(B * Lq, H, d).numpy(), atol=1e-12)
+
+
+def test_sparse_rejects_bad_indices():
+    rng = np.random.default_rng(8)
+    q, k, v = _rand_bf16(rng, (1, 2, 2, 8)), _rand_bf16(rng, (1, 10, 8)), _rand_bf16(rng, (1, 10, 8))
+    idx = np.full((1, 2, 4), -1, np.int32)
+    idx[0, 0, 0] = 3
+    with pytest.raises(RuntimeError):
+        oracle.sparse_attn(q, k, v, idx, 0.3)          # row 1 has no valid index
+    idx[0, 1, 0] = 10
+    with pytest.raises(RuntimeError):
+        oracle.sparse_attn(q, k, v, idx, 0.3)          # out of range
+
+
+@pytest.mark.parametrize("T,hidden,n,d", [(7, 24, 2, 8), (33, 64, 4, 16), (5, 2048, 1, 128)])
+def test_bridge_matches_numpy_matmul(T, hidden, n, d):
+    rng = np.random.default_rng(9)
+    h = _rand_bf16(rng, (T, hidden))
+    w = _rand_bf16(rng, (n, 2, hidden, d), 0.02)
+    kv = oracle.bridge_kv_proj(h, w)
+    hf = bf16_bits_to_f32(h).astype(np.float64)
+    wf = bf16_bits_to_f32(w).astype(np.float64)
+    for layer in range(n):
+        for kvi in range(2):
+            np.testing.assert_allclose(kv[layer, kvi], hf @ wf[layer, kvi], rtol=1e-13, atol=1e-13)
+    rows = [T - 1, 0]
+    np.testing.assert_array_equal(oracle.bridge_kv_proj(h, w, rows=rows), kv[:, :, rows])
+
+
+def test_row_sampling_matches_full_run():
+    wl = synth.small("decode_32k", B=3, Lk=500, H=4, d=16)
+    g = synth.SyntheticInputs(wl)
+    full = oracle.full_attn_select(g.q, g.k, g.v, wl.scale, 16, 32, want_score=True)
+    part = oracle.full_attn_select(g.q, g.k, g.v, wl.scale, 16, 32, rows=[2, 0], want_score=True)
+    for key in ("out", "lse", "idx", "score"):
+        np.testing.assert_array_equal(part[key], full[key][[2, 0]])
