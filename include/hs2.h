@@ -1,0 +1,155 @@
+/*
+ * hs2.h -- C ABI of the B200 (sm_100a) HySparse2 hot path.
+ *
+ * Operations, as the pages about "HySparse2: Hybrid Sparse Attention with Two-Level KV
+ * Sharing" state the problem:
+ *
+ *  hs2_full_attn_select  A causal multi-query full-attention layer (64 query heads share
+ *                        one K/V head: arex-research.com article "小米 MiMo 负责人罗福利公开
+ *                        MiMo-V3 核心架构 HySparse2", section "三套 80B-A3B 对照模型里算出的数字")
+ *                        that also acts as the indexer: from its exact attention scores it
+ *                        selects, for every query position t, the `window` most recent tokens
+ *                        t-window+1..t plus the `topk` highest-scoring older tokens 0..t-window
+ *                        (same article, section "外层 KV Bridging，内层 KV Reuse"; toolnavs.com
+ *                        HySparse2 article, section "Was HySparse2 tut"; zgeo.com.cn article,
+ *                        section "核心技术原理解析": 128 + 1,024 tokens).
+ *                        The pages leave open how the heads' scores are combined. This library
+ *                        scores token j for query t as the sum over heads of the post-softmax
+ *                        probability (softmax over the whole causal row 0..t); equal scores go
+ *                        to the lower index.
+ *  hs2_sparse_attn       A sparse layer of the same hybrid block: reuses the full layer's K/V
+ *                        cache and selection indices unchanged, with its own Q, and attends
+ *                        only to the selected tokens (arex-research.com, section "外层 KV
+ *                        Bridging，内层 KV Reuse"; toolnavs.com, section "Was HySparse2 tut").
+ *  hs2_bridge_kv_proj    KV Bridging: one self-decoder hidden state H is projected by several
+ *                        cross-decoder layers' own W_k / W_v (arex-research.com, section
+ *                        "外层 KV Bridging，内层 KV Reuse"; toolnavs.com, section "Was HySparse2
+ *                        tut"), computed as one batched GEMM.
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc / torch memory), row-major,
+ *    contiguous, 16-byte aligned, owned by the caller. bf16 values are passed as
+ *    hs2_bf16 (the 16-bit pattern). Inputs are read only; outputs must not alias inputs.
+ *  - `workspace` is caller-owned device scratch of at least the size the matching
+ *    *_workspace_bytes query returns. Its first 16 bytes hold the device status word. The
+ *    library never allocates, frees or synchronises inside the compute calls.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *    Arguments are validated on the host before anything is launched; a non-zero return
+ *    means nothing was launched (HS2_ERR_CUDA: a launch failed).
+ *  - Device-side problems (a bounded wait that gave up, an index out of range) never trap:
+ *    the kernel records them in the status word and returns. Read them with
+ *    hs2_read_device_status.
+ *  - There is no CPU fallback: a device that is not sm_100 returns
+ *    HS2_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HS2_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define HS2_API __attribute__((visibility("default")))
+#else
+#define HS2_API
+#endif
+
+typedef uint16_t hs2_bf16; /* bf16 bit pattern */
+typedef void* hs2_stream;  /* cudaStream_t */
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1,       /* null / misaligned pointer, negative or inconsistent size */
+  HS2_ERR_UNSUPPORTED_SHAPE = 2, /* (H, d) not supported, or the device is not sm_100 */
+  HS2_ERR_WORKSPACE = 3,         /* workspace missing or smaller than required */
+  HS2_ERR_CUDA = 4,              /* a CUDA runtime call or kernel launch failed */
+  HS2_ERR_DEVICE_TIMEOUT = 5,    /* a kernel's bounded wait gave up (status word) */
+  HS2_ERR_DEVICE_BOUNDS = 6      /* a kernel saw an index outside [0, Lk) (status word) */
+} hs2_status;
+
+/* ABI version of the loaded library (HS2_ABI_VERSION at build time). */
+HS2_API int hs2_abi_version(void);
+
+/* Static, human-readable text of a status code. */
+HS2_API const char* hs2_status_string(hs2_status s);
+
+/* ---------------------------------------------------------------------------------
+ * Full attention + token selection
+ * ---------------------------------------------------------------------------------
+ * Q    [B, Lq, H, d] bf16  queries; query i sits at position t = Lk - Lq + i
+ *                           (Lq == Lk: prefill over the whole sequence; Lq == 1: one decode
+ *                           step whose own K/V row is already the last cache row)
+ * K, V [B, Lk, d]    bf16  the single K/V head
+ * scale                     softmax scale applied to q.k (e.g. 1/sqrt(d))
+ * window, topk              forced recent tokens and number of older tokens chosen by score
+ *                           (the pages: 128 and 1,024); window >= 1, topk >= 0
+ * out  [B, Lq, H, d] bf16  softmax(scale q K^T) V over the causal row
+ * lse  [B, Lq, H]    fp32  natural-log logsumexp of the scaled logits of the causal row
+ * idx  [B, Lq, window+topk] int32  selected token indices of each query, ascending;
+ *                           exactly min(t+1, window+topk) valid entries, then -1 padding
+ * Supported: (H, d) in {(64, 128), (16, 64)}; Lq == 1 or Lq == Lk (bf16, fp32 accumulate).
+ * Decode (Lq == 1) supports (H, d) = (64, 128).
+ */
+HS2_API size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk);
+HS2_API hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,
+                                int H, int d, float scale, int window, int topk, hs2_bf16* out, float* lse,
+                                int32_t* idx, void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
+ * Sparse attention over selected tokens (one sparse layer)
+ * ---------------------------------------------------------------------------------
+ * Q    [B, Lq, H, d] bf16  this layer's own queries
+ * K, V [B, Lk, d]    bf16  the full layer's K/V cache, reused unchanged
+ * idx  [B, Lq, S]    int32 the full layer's selection, reused unchanged; -1 slots are skipped,
+ *                           any other value must lie in [0, Lk) (else the status word records
+ *                           HS2_ERR_DEVICE_BOUNDS and the row's output is unspecified).
+ *                           Every row needs at least one valid entry.
+ * out  [B, Lq, H, d] bf16  softmax over the selected tokens of scale q.k, times V
+ * lse  [B, Lq, H]    fp32  natural-log logsumexp over the selected tokens, or NULL
+ * Supported: (H, d) in {(64, 128), (16, 64)}, 1 <= S <= 4096.
+ */
+HS2_API size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int d, int S);
+HS2_API hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
+                           int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
+                           void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
+ * KV Bridging projection
+ * ---------------------------------------------------------------------------------
+ * Hs   [T, hidden]                bf16  shared hidden state
+ * W    [n_layers, 2, hidden, d]   bf16  per layer: W_k (index 0) then W_v (index 1)
+ * KV   [n_layers, 2, T, d]        bf16  K_l = Hs W[l,0], V_l = Hs W[l,1] (fp32 accumulate)
+ * Supported: hidden % 64 == 0, d in {64, 128}.
+ */
+HS2_API size_t hs2_bridge_kv_proj_workspace_bytes(int T, int hidden, int n_layers, int d);
+HS2_API hs2_status hs2_bridge_kv_proj(const hs2_bf16* Hs, int T, int hidden, const hs2_bf16* W, int n_layers, int d,
+                              hs2_bf16* KV, void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
+ * Device status
+ * ---------------------------------------------------------------------------------
+ * hs2_read_device_status: waits for `stream`, reads the status word of `workspace` and
+ * returns HS2_OK, HS2_ERR_DEVICE_TIMEOUT or HS2_ERR_DEVICE_BOUNDS (HS2_ERR_CUDA if the
+ * read failed). hs2_clear_device_status: resets the word (asynchronously, on `stream`).
+ * hs2_set_wait_limit_ns: wall-time bound of every device-side wait of later launches
+ * (default 2 s, or the environment variable HS2_WAIT_LIMIT_MS at first use).
+ * hs2_selftest_wait_timeout: launches one kernel whose bounded wait is on a barrier that
+ * nothing completes; it gives up after `limit_ns`, records HS2_ERR_DEVICE_TIMEOUT in the
+ * status word and returns, leaving the context usable (a failure-detection test hook).
+ */
+HS2_API hs2_status hs2_read_device_status(const void* workspace, hs2_stream stream);
+HS2_API hs2_status hs2_clear_device_status(void* workspace, hs2_stream stream);
+HS2_API void hs2_set_wait_limit_ns(long long limit_ns);
+HS2_API hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_ns, hs2_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H_ */

@@ -1,0 +1,228 @@
+"""hs2 -- B200-native (sm_100a) hot path of HySparse2 token-level hybrid sparse attention.
+
+Thin Python binding of the C-ABI library ``libhs2.so`` (declared in ``include/hs2.h``):
+argument marshalling only, every step of the computation runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. There is no CPU fallback: importing
+this package fails loudly if the library cannot be loaded.
+
+    out, lse, idx = full_attn_select(q, k, v)            # full layer + indexer
+    out2 = sparse_attn(q2, k, v, idx)                     # a sparse layer (KV Reuse)
+    kv = bridge_kv_proj(h, w)                             # KV Bridging projection
+
+Tensors: q [B, Lq, H, d] bf16, k/v [B, Lk, d] bf16 (one K/V head), idx [B, Lq, S] int32,
+h [T, hidden] bf16, w [n_layers, 2, hidden, d] bf16 -> kv [n_layers, 2, T, d] bf16.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+WINDOW = 128
+TOPK = 1024
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libhs2.so")
+
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported shape or device", 3: "workspace missing or too small",
+    4: "CUDA error", 5: "device-side wait timed out", 6: "device-side index out of range",
+}
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BOUNDS = range(7)
+
+
+class HS2Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+def _load_library() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        from . import _build
+        _build.build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, i32, f32, sz, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
+    lib.hs2_abi_version.restype = i32
+    lib.hs2_status_string.argtypes = [i32]
+    lib.hs2_status_string.restype = ctypes.c_char_p
+    lib.hs2_full_attn_select_workspace_bytes.argtypes = [i32] * 7
+    lib.hs2_full_attn_select_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select.argtypes = [P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select.restype = i32
+    lib.hs2_sparse_attn_workspace_bytes.argtypes = [i32] * 6
+    lib.hs2_sparse_attn_workspace_bytes.restype = sz
+    lib.hs2_sparse_attn.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, sz, P]
+    lib.hs2_sparse_attn.restype = i32
+    lib.hs2_bridge_kv_proj_workspace_bytes.argtypes = [i32] * 4
+    lib.hs2_bridge_kv_proj_workspace_bytes.restype = sz
+    lib.hs2_bridge_kv_proj.argtypes = [P, i32, i32, P, i32, i32, P, P, sz, P]
+    lib.hs2_bridge_kv_proj.restype = i32
+    lib.hs2_read_device_status.argtypes = [P, P]
+    lib.hs2_read_device_status.restype = i32
+    lib.hs2_clear_device_status.argtypes = [P, P]
+    lib.hs2_clear_device_status.restype = i32
+    lib.hs2_set_wait_limit_ns.argtypes = [ll]
+    lib.hs2_set_wait_limit_ns.restype = None
+    lib.hs2_selftest_wait_timeout.argtypes = [P, sz, ll, P]
+    lib.hs2_selftest_wait_timeout.restype = i32
+    return lib
+
+
+lib = _load_library()
+LIBRARY_PATH = _LIB_PATH
+ABI_VERSION = lib.hs2_abi_version()
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def _workspace(nbytes: int, device: torch.device, key: str) -> torch.Tensor:
+    """Cached per-(device, op) workspace; pass your own for concurrent streams."""
+    with _ws_lock:
+        k = (device, key)
+        ws = _ws_cache.get(k)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            _ws_cache[k] = ws
+        return ws
+
+
+def _stream_ptr(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise HS2Error(code, what)
+
+
+def _need(t: torch.Tensor, name: str, dtype, dim: int):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window=WINDOW, topk=TOPK) -> int:
+    return int(lib.hs2_full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window, topk))
+
+
+def sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S) -> int:
+    return int(lib.hs2_sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S))
+
+
+def bridge_kv_proj_workspace_bytes(T, hidden, n_layers, d) -> int:
+    return int(lib.hs2_bridge_kv_proj_workspace_bytes(T, hidden, n_layers, d))
+
+
+def full_attn_select(q, k, v, *, scale=None, window=WINDOW, topk=TOPK, out=None, lse=None, idx=None,
+                     workspace=None, stream=None):
+    """Causal MQA attention that also selects tokens (hs2_full_attn_select).
+
+    Returns (out [B,Lq,H,d] bf16, lse [B,Lq,H] fp32 natural log, idx [B,Lq,window+topk] int32).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    if tuple(k.shape) != (B, Lk, d) or tuple(v.shape) != (B, Lk, d):
+        raise ValueError("k and v must be [B, Lk, d] matching q")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = window + topk
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, Lq, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    nbytes = full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window, topk)
+    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    code = lib.hs2_full_attn_select(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Lq, Lk, H, d, scale, window, topk,
+                                    out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                    ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select")
+    return out, lse, idx
+
+
+def sparse_attn(q, k, v, idx, *, scale=None, out=None, lse=None, want_lse=False, workspace=None, stream=None):
+    """Sparse attention of one sparse layer over the reused K/V and indices (hs2_sparse_attn).
+
+    Returns out [B,Lq,H,d] bf16, or (out, lse) when want_lse or lse is given.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(idx, "idx", torch.int32, 3)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    S = idx.shape[2]
+    if tuple(idx.shape[:2]) != (B, Lq):
+        raise ValueError("idx must be [B, Lq, S]")
+    if tuple(k.shape) != (B, Lk, d) or tuple(v.shape) != (B, Lk, d):
+        raise ValueError("k and v must be [B, Lk, d] matching q")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", torch.bfloat16, 4)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    nbytes = sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S)
+    ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
+    code = lib.hs2_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), B, Lq, Lk, H, d, S, scale,
+                               out.data_ptr(), lse.data_ptr() if lse is not None else None, ws.data_ptr(),
+                               ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_sparse_attn")
+    return (out, lse) if lse is not None else out
+
+
+def bridge_kv_proj(h, w, *, out=None, workspace=None, stream=None):
+    """KV Bridging: kv[l, 0] = h @ w[l, 0], kv[l, 1] = h @ w[l, 1] (hs2_bridge_kv_proj)."""
+    _need(h, "h", torch.bfloat16, 2)
+    _need(w, "w", torch.bfloat16, 4)
+    T, hidden = h.shape
+    n, two, hw, d = w.shape
+    if two != 2 or hw != hidden:
+        raise ValueError("w must be [n_layers, 2, hidden, d]")
+    out = torch.empty((n, 2, T, d), dtype=torch.bfloat16, device=h.device) if out is None else out
+    _need(out, "out", torch.bfloat16, 4)
+    nbytes = bridge_kv_proj_workspace_bytes(T, hidden, n, d)
+    ws = _workspace(nbytes, h.device, "bridge") if workspace is None else workspace
+    code = lib.hs2_bridge_kv_proj(h.data_ptr(), T, hidden, w.data_ptr(), n, d, out.data_ptr(), ws.data_ptr(),
+                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_bridge_kv_proj")
+    return out
+
+
+def read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Waits for the stream and returns the status word of `workspace` (0 = ok)."""
+    return int(lib.hs2_read_device_status(workspace.data_ptr(), _stream_ptr(stream)))
+
+
+def clear_device_status(workspace: torch.Tensor, stream=None) -> None:
+    _check(lib.hs2_clear_device_status(workspace.data_ptr(), _stream_ptr(stream)), "hs2_clear_device_status")
+
+
+def cached_workspace(key: str, device=None):
+    """The workspace the convenience calls used for `key` ("full", "sparse", "bridge")."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return _ws_cache.get((device, key))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib.hs2_set_wait_limit_ns(int(ns))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int, stream=None) -> None:
+    _check(lib.hs2_selftest_wait_timeout(workspace.data_ptr(), workspace.numel(), int(limit_ns), _stream_ptr(stream)),
+           "hs2_selftest_wait_timeout")

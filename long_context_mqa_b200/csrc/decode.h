@@ -1,0 +1,72 @@
+// Internal interfaces between the hs2 C-ABI layer (hs2_api.cu) and the kernel files.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hs2 {
+
+struct DevStatus;
+
+namespace dec {
+// Parameters of the decode (one query per sequence) full-attention + selection kernels.
+struct DecParams {
+  int B, N, W, K;          // sequences, cache length, window, top-k
+  int tps;                 // 128-key tiles per sequence
+  long long total_tiles;   // B * tps
+  int G;                   // CTAs of the two scan passes
+  int segmax;              // partial records per CTA
+  float c;                 // scale * log2(e)
+  long long wait_ns;       // bound of every device-side wait
+  float* ml;               // [G*segmax][2][H] pass-1 partial (max, sum), log2 domain
+  float* lse2;             // [B][H] row logsumexp, log2 domain
+  float* lse_out;          // [B][H] natural log (caller's lse)
+  float* opart;            // [G*segmax][H][D] pass-2 partial outputs
+  float* sc;               // [B][N-W] head-summed scores of the older tokens
+  unsigned* hist;          // [B][2048] histogram of score bits 30..20
+  DevStatus* st;
+};
+size_t pass1_smem_bytes(int H, int D);
+size_t pass2_smem_bytes(int H, int D);
+cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                               const DecParams& p, __nv_bfloat16* out, cudaStream_t stream);
+}  // namespace dec
+
+namespace sel {
+constexpr int NBINS = 2048;
+constexpr int META = 8;  // ints per sequence: beta, above, need, cnt_above, cnt_bnd
+// Top-k selection over a materialised score vector per sequence (decode path).
+struct SelParams {
+  int B, N, W, K, S;
+  int ncand;                     // max(N - W, 0) older tokens per sequence
+  const float* sc;               // [B][ncand]
+  const unsigned* hist;          // [B][NBINS]
+  int* meta;                     // [B][META]
+  int* above;                    // [B][K]
+  unsigned long long* bnd;       // [B][ncand] boundary-bin candidates (score bits << 32 | ~index)
+  int32_t* idx;                  // [B][S] output
+  DevStatus* st;
+};
+cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
+}  // namespace sel
+
+namespace sparse {
+struct SpParams {
+  const __nv_bfloat16 *Q, *K, *V;
+  const int32_t* idx;
+  int B, Lq, Lk, S;
+  int nsplit, split_slots;    // slots of idx handled per CTA (multiple of 128)
+  float c;                    // scale * log2(e)
+  __nv_bfloat16* out;
+  float* lse;                 // may be null
+  float* opart;               // [B*Lq*nsplit][H][D] (nsplit > 1)
+  float* mlpart;              // [B*Lq*nsplit][2][H]
+  long long wait_ns;
+  DevStatus* st;
+};
+size_t sparse_smem_bytes(int H, int D);
+cudaError_t launch_sparse(const SpParams& p, int H, int D, cudaStream_t stream);
+}  // namespace sparse
+
+}  // namespace hs2

@@ -1,0 +1,333 @@
+// C ABI of the hs2 library (declared in include/hs2.h): argument validation, workspace
+// layout, TMA descriptor set-up and dispatch to the kernel files. No allocation, no
+// synchronisation and no host fallback on the compute paths.
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "decode.h"
+#include "host_util.h"
+#include "prefill.h"
+#include "tc.cuh"
+
+namespace hs2 {
+
+// ------------------------------------------------------------------------------------------
+// host utilities
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                  uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner, uint32_t box_rows,
+                  bool swizzle128) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {row_stride_el * 2, batch_stride_el * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_el,
+                  uint32_t box_inner, uint32_t box_rows) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_el * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static long long g_wait_ns = -1;
+long long wait_limit_ns() {
+  if (g_wait_ns < 0) {
+    const char* e = getenv("HS2_WAIT_LIMIT_MS");
+    long long ms = e ? atoll(e) : 0;
+    g_wait_ns = (ms > 0 ? ms : 2000) * 1000000LL;
+  }
+  return g_wait_ns;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0;
+}
+
+// ------------------------------------------------------------------------------------------
+// workspace carving
+// ------------------------------------------------------------------------------------------
+constexpr size_t kStatusBytes = 256;
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Carve {
+  uint8_t* base;
+  size_t off;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align256(off + count * sizeof(T));
+    return p;
+  }
+};
+
+// decode (Lq == 1) layout
+struct DecodeWs {
+  dec::DecParams p;
+  int* meta;
+  int* above;
+  unsigned long long* bnd;
+  size_t bytes;
+};
+
+static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K, int sms) {
+  DecodeWs w{};
+  dec::DecParams& p = w.p;
+  p.B = B; p.N = N; p.W = W; p.K = K;
+  p.tps = (N + 127) / 128;
+  p.total_tiles = (long long)B * p.tps;
+  p.G = (int)(p.total_tiles < sms ? p.total_tiles : sms);
+  int segmax = 1;
+  for (int cta = 0; cta < p.G; ++cta) {
+    const long long t0 = p.total_tiles * cta / p.G, t1 = p.total_tiles * (cta + 1) / p.G;
+    if (t1 > t0) {
+      const int segs = (int)((t1 - 1) / p.tps - t0 / p.tps + 1);
+      if (segs > segmax) segmax = segs;
+    }
+  }
+  p.segmax = segmax;
+  const int ncand = N - W > 0 ? N - W : 0;
+  Carve c{(uint8_t*)ws, 0};
+  p.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
+  p.ml = c.take<float>((size_t)p.G * segmax * 2 * H);
+  p.lse2 = c.take<float>((size_t)B * H);
+  p.opart = c.take<float>((size_t)p.G * segmax * H * D);
+  p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
+  p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
+  w.meta = c.take<int>((size_t)B * sel::META);
+  w.above = c.take<int>((size_t)B * (K > 0 ? K : 1));
+  w.bnd = c.take<unsigned long long>((size_t)B * (ncand > 0 ? ncand : 1));
+  w.bytes = c.off;
+  return w;
+}
+
+// sparse layout
+static size_t carve_sparse(void* ws, int B, int Lq, int H, int D, int S, int sms, sparse::SpParams* p) {
+  const long long rows = (long long)B * Lq;
+  const int tiles = (S + 127) / 128;
+  int nsplit = 1;
+  if (rows < sms && tiles > 1) nsplit = tiles;  // few rows: one 128-slot tile per CTA
+  Carve c{(uint8_t*)ws, 0};
+  DevStatus* st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
+  float* opart = nullptr;
+  float* mlpart = nullptr;
+  if (nsplit > 1) {
+    opart = c.take<float>((size_t)rows * nsplit * H * D);
+    mlpart = c.take<float>((size_t)rows * nsplit * 2 * H);
+  }
+  if (p) {
+    p->st = st;
+    p->opart = opart;
+    p->mlpart = mlpart;
+    p->nsplit = nsplit;
+    p->split_slots = nsplit > 1 ? 128 : tiles * 128;
+  }
+  return c.off;
+}
+
+static bool shape_ok(int H, int d) { return (H == 64 && d == 128) || (H == 16 && d == 64); }
+
+// ------------------------------------------------------------------------------------------
+// device-side helpers of the C ABI
+// ------------------------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(DevStatus* st, long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the bounded wait must give up and report
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns)) report_status(st, kStatusTimeout, 900);
+}
+
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+int hs2_abi_version(void) { return HS2_ABI_VERSION; }
+
+const char* hs2_status_string(hs2_status s) {
+  switch (s) {
+    case HS2_OK: return "ok";
+    case HS2_ERR_INVALID_ARG: return "invalid argument";
+    case HS2_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or device";
+    case HS2_ERR_WORKSPACE: return "workspace missing or too small";
+    case HS2_ERR_CUDA: return "CUDA error";
+    case HS2_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case HS2_ERR_DEVICE_BOUNDS: return "device-side index out of range";
+  }
+  return "unknown status";
+}
+
+void hs2_set_wait_limit_ns(long long limit_ns) { g_wait_ns = limit_ns > 0 ? limit_ns : -1; }
+
+size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || d <= 0 || window < 1 || topk < 0) return 0;
+  const int sms = num_sms() > 0 ? num_sms() : 148;
+  if (Lq == 1) return carve_decode(nullptr, B, Lk, H, d, window, topk, sms).bytes;
+  return prefill::workspace_bytes(B, Lq, Lk, H, d, window, topk, sms, kStatusBytes);
+}
+
+hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,
+                                int H, int d, float scale, int window, int topk, hs2_bf16* out, float* lse,
+                                int32_t* idx, void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K || !V || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(lse) || !aligned16(idx))
+    return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || window < 1 || topk < 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (window + topk > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!shape_ok(H, d)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  const int sms = num_sms();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float c = scale * 1.4426950408889634f;
+  if (Lq == 1) {
+    if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
+    DecodeWs w = carve_decode(workspace, B, Lk, H, d, window, topk, sms);
+    if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
+    w.p.c = c;
+    w.p.wait_ns = wait_limit_ns();
+    w.p.lse_out = lse;
+    CUtensorMap tmK, tmV, tmQ;
+    if (!make_tmap_3d(&tmK, K, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+        !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+        !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
+      return HS2_ERR_CUDA;
+    if (cudaMemsetAsync(w.p.hist, 0, (size_t)B * sel::NBINS * sizeof(unsigned), st) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, reinterpret_cast<__nv_bfloat16*>(out), st) != cudaSuccess)
+      return HS2_ERR_CUDA;
+    sel::SelParams sp;
+    sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
+    sp.ncand = Lk - window > 0 ? Lk - window : 0;
+    sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.above = w.above; sp.bnd = w.bnd;
+    sp.idx = idx; sp.st = w.p.st;
+    if (sel::launch_select(sp, st) != cudaSuccess) return HS2_ERR_CUDA;
+    return HS2_OK;
+  }
+  if (Lq != Lk) return HS2_ERR_UNSUPPORTED_SHAPE;
+  return prefill::run(Q, K, V, B, Lq, Lk, H, d, c, window, topk, out, lse, idx, workspace, workspace_bytes, sms,
+                      kStatusBytes, st);
+}
+
+size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int d, int S) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || d <= 0 || S <= 0) return 0;
+  const int sms = num_sms() > 0 ? num_sms() : 148;
+  return carve_sparse(nullptr, B, Lq, H, d, S, sms, nullptr);
+}
+
+hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
+                           int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
+                           void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K || !V || !idx || !out) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (lse && !aligned16(lse)))
+    return HS2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) != 0) return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || S <= 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (S > 4096) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!shape_ok(H, d)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * Lq > 2147483647LL / 16) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  const int sms = num_sms();
+  sparse::SpParams p{};
+  const size_t need = carve_sparse(workspace, B, Lq, H, d, S, sms, &p);
+  if (workspace_bytes < need) return HS2_ERR_WORKSPACE;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.idx = idx;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.S = S;
+  p.c = scale * 1.4426950408889634f;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.wait_ns = wait_limit_ns();
+  if (sparse::launch_sparse(p, H, d, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+size_t hs2_bridge_kv_proj_workspace_bytes(int T, int hidden, int n_layers, int d) {
+  if (T <= 0 || hidden <= 0 || n_layers <= 0 || d <= 0) return 0;
+  return kStatusBytes;
+}
+
+hs2_status hs2_bridge_kv_proj(const hs2_bf16* Hs, int T, int hidden, const hs2_bf16* W, int n_layers, int d,
+                              hs2_bf16* KV, void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (!Hs || !W || !KV) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Hs) || !aligned16(W) || !aligned16(KV)) return HS2_ERR_INVALID_ARG;
+  if (T <= 0 || hidden <= 0 || n_layers <= 0 || d <= 0) return HS2_ERR_INVALID_ARG;
+  if (hidden % 64 != 0 || (d != 64 && d != 128)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes) return HS2_ERR_WORKSPACE;
+  return prefill::run_bridge(Hs, T, hidden, W, n_layers, d, KV, reinterpret_cast<DevStatus*>(workspace),
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+hs2_status hs2_read_device_status(const void* workspace, hs2_stream stream) {
+  if (!workspace) return HS2_ERR_WORKSPACE;
+  DevStatus h{};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return HS2_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HS2_ERR_CUDA;
+  if (h.flags & kStatusTimeout) return HS2_ERR_DEVICE_TIMEOUT;
+  if (h.flags & kStatusBounds) return HS2_ERR_DEVICE_BOUNDS;
+  return HS2_OK;
+}
+
+hs2_status hs2_clear_device_status(void* workspace, hs2_stream stream) {
+  if (!workspace) return HS2_ERR_WORKSPACE;
+  if (cudaMemsetAsync(workspace, 0, sizeof(DevStatus), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_ns, hs2_stream stream) {
+  if (!workspace || workspace_bytes < kStatusBytes) return HS2_ERR_WORKSPACE;
+  if (limit_ns <= 0 || limit_ns > 10000000000LL) return HS2_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(reinterpret_cast<DevStatus*>(workspace),
+                                                                               limit_ns);
+  return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+}  // extern "C"

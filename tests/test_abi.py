@@ -1,0 +1,61 @@
+"""The C-ABI library loads and exports every symbol include/hs2.h declares (CPU only).
+
+Only host-side paths are exercised here: version, status strings and argument validation
+that rejects calls before anything touches a device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    return re.findall(r"HS2_API\s+[\w\s\*]+?\b(hs2_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for n in ("hs2_full_attn_select", "hs2_sparse_attn", "hs2_bridge_kv_proj", "hs2_full_attn_select_workspace_bytes",
+              "hs2_sparse_attn_workspace_bytes", "hs2_bridge_kv_proj_workspace_bytes", "hs2_read_device_status",
+              "hs2_status_string", "hs2_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import long_context_mqa_b200 as hs2
+    lib = ctypes.CDLL(hs2.LIBRARY_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings():
+    import long_context_mqa_b200 as hs2
+    assert hs2.ABI_VERSION == 1
+    for code, text in hs2.STATUS.items():
+        assert hs2.lib.hs2_status_string(code).decode() == text
+
+
+def test_null_arguments_are_rejected_before_any_launch():
+    import long_context_mqa_b200 as hs2
+    L = hs2.lib
+    assert L.hs2_full_attn_select(None, None, None, 1, 1, 8, 64, 128, 0.1, 128, 1024, None, None, None, None, 0,
+                                  None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_sparse_attn(None, None, None, None, 1, 1, 8, 64, 128, 8, 0.1, None, None, None, 0,
+                             None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_bridge_kv_proj(None, 8, 64, None, 1, 128, None, None, 0, None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_read_device_status(None, None) == hs2.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("B,Lk", [(8, 262144), (2, 1048576), (32, 32768), (1, 100)])
+def test_workspace_queries_are_sane(B, Lk):
+    import long_context_mqa_b200 as hs2
+    n = hs2.full_attn_select_workspace_bytes(B, 1, Lk, 64, 128)
+    assert n >= 256
+    # scores (4 B) + boundary keys (8 B) per older token dominate
+    assert n >= B * max(Lk - 128, 0) * 12
+    assert hs2.full_attn_select_workspace_bytes(0, 1, Lk, 64, 128) == 0
+    assert hs2.sparse_attn_workspace_bytes(B, 1, Lk, 64, 128, 1152) >= 256

@@ -1,0 +1,90 @@
+"""GPU parity of the decode path (one query token per sequence) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import assert_out_close, bf16_to_f64, check_selection, to_torch_bf16
+
+pytestmark = pytest.mark.gpu
+
+W, K = synth.WINDOW, synth.TOPK
+
+
+@pytest.fixture(scope="module")
+def hs2():
+    import long_context_mqa_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def _run_full(hs2, g):
+    wl = g.wl
+    q, k, v = to_torch_bf16(g.q), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    out, lse, idx = hs2.full_attn_select(q, k, v, scale=wl.scale, window=wl.window, topk=wl.topk)
+    torch.cuda.synchronize()
+    ws = hs2.cached_workspace("full")
+    assert hs2.read_device_status(ws) == 0
+    return q, k, v, out, lse, idx
+
+
+def _check_full(g, out, lse, idx, rows=None):
+    wl = g.wl
+    ora = oracle.full_attn_select(g.q, g.k, g.v, wl.scale, wl.window, wl.topk, rows=rows, want_score=True)
+    sel_rows = np.arange(wl.B * wl.Lq) if rows is None else np.asarray(rows)
+    gout = bf16_to_f64(out).reshape(wl.B * wl.Lq, wl.H, wl.d)[sel_rows]
+    assert_out_close(gout, ora["out"], "full-attention output")
+    glse = lse.double().cpu().numpy().reshape(wl.B * wl.Lq, wl.H)[sel_rows]
+    assert np.abs(glse - ora["lse"]).max() < 2e-3
+    gidx = idx.cpu().numpy().reshape(wl.B * wl.Lq, -1)[sel_rows]
+    t_pos = wl.Lk - wl.Lq + (sel_rows % wl.Lq)
+    st = check_selection(gidx, ora["idx"], ora["score"], t_pos, wl.window, wl.topk)
+    assert st.ok(), st.failures
+    return ora, st
+
+
+@pytest.mark.parametrize("B,N", [(3, 100), (2, 1000), (2, 1152), (1, 1153), (3, 3000), (2, 20000), (1, 40000)])
+def test_decode_small(hs2, B, N):
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=N))
+    q, k, v, out, lse, idx = _run_full(hs2, g)
+    _check_full(g, out, lse, idx)
+
+
+def test_decode_all_ties_prefer_lower_index(hs2):
+    """K == 0 makes every score equal: the older picks must be tokens 0..topk-1."""
+    B, N = 2, 3000
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=N))
+    q = to_torch_bf16(g.q)
+    k = torch.zeros((B, N, 128), dtype=torch.bfloat16, device="cuda")
+    v = to_torch_bf16(g.v)
+    out, lse, idx = hs2.full_attn_select(q, k, v)
+    torch.cuda.synchronize()
+    expect = np.concatenate([np.arange(K), np.arange(N - W, N)])
+    for b in range(B):
+        np.testing.assert_array_equal(idx[b, 0].cpu().numpy(), expect)
+    np.testing.assert_allclose(lse.cpu().numpy(), np.log(N), rtol=0, atol=1e-4)
+
+
+def test_decode_repeatable(hs2):
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=2, Lk=9000))
+    _, _, _, out1, lse1, idx1 = _run_full(hs2, g)
+    out1, lse1, idx1 = out1.clone(), lse1.clone(), idx1.clone()
+    _, _, _, out2, lse2, idx2 = _run_full(hs2, g)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2) and torch.equal(idx1, idx2)
+
+
+@pytest.mark.parametrize("name", ["decode_32k", "decode_256k", "decode_1m"])
+def test_decode_full_size(hs2, name):
+    """Full configuration sizes, the launch the benchmark times; every sequence checked."""
+    g = synth.SyntheticInputs(synth.WORKLOADS[name])
+    q, k, v, out, lse, idx = _run_full(hs2, g)
+    ora, st = _check_full(g, out, lse, idx)
+    print(f"{name}: swaps {st.swaps} (max rel {st.max_swap_rel:.2e})")
+    # sparse layers of the same step reuse K, V and the GPU indices
+    for layer in range(g.wl.n_sparse):
+        qs = g.q_sparse(layer)
+        o2 = hs2.sparse_attn(to_torch_bf16(qs), k, v, idx, scale=g.wl.scale)
+        torch.cuda.synchronize()
+        ref = oracle.sparse_attn(qs, g.k, g.v, idx.cpu().numpy(), g.wl.scale)
+        assert_out_close(bf16_to_f64(o2).reshape(ref["out"].shape), ref["out"], f"sparse layer {layer}")
