@@ -148,6 +148,22 @@ HS2_API hs2_status hs2_clear_device_status(void* workspace, hs2_stream stream);
 HS2_API void hs2_set_wait_limit_ns(long long limit_ns);
 HS2_API hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_ns, hs2_stream stream);
 
+/* ---------------------------------------------------------------------------------
+ * Diagnostics (never needed on the compute path)
+ * ---------------------------------------------------------------------------------
+ * hs2_kernel_launches: number of CUDA kernels this library has launched since it was
+ * loaded (all devices, all streams).
+ * hs2_profile_enable: NULL turns per-kernel timing off; "*" times every kernel; any other
+ * string times only the kernel of that name (e.g. "dec_pass2", "sparse_attn"). While on,
+ * the library records a pair of CUDA events around each matching launch on its stream.
+ * hs2_profile_read: waits for the recorded events of `kernel`, returns their summed
+ * duration in milliseconds and the number of launches, and forgets them. Returns 0, or -1
+ * if an event could not be read.
+ */
+HS2_API unsigned long long hs2_kernel_launches(void);
+HS2_API void hs2_profile_enable(const char* kernel);
+HS2_API int hs2_profile_read(const char* kernel, double* total_ms, long long* launches);
+
 #ifdef __cplusplus
 }
 #endif

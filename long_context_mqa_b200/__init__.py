@@ -69,6 +69,11 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_set_wait_limit_ns.restype = None
     lib.hs2_selftest_wait_timeout.argtypes = [P, sz, ll, P]
     lib.hs2_selftest_wait_timeout.restype = i32
+    lib.hs2_kernel_launches.restype = ctypes.c_ulonglong
+    lib.hs2_profile_enable.argtypes = [ctypes.c_char_p]
+    lib.hs2_profile_enable.restype = None
+    lib.hs2_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    lib.hs2_profile_read.restype = i32
     return lib
 
 
@@ -226,3 +231,22 @@ def set_wait_limit_ns(ns: int) -> None:
 def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int, stream=None) -> None:
     _check(lib.hs2_selftest_wait_timeout(workspace.data_ptr(), workspace.numel(), int(limit_ns), _stream_ptr(stream)),
            "hs2_selftest_wait_timeout")
+
+
+def kernel_launches() -> int:
+    """CUDA kernels this library launched since it was loaded."""
+    return int(lib.hs2_kernel_launches())
+
+
+def profile_enable(kernel: str | None) -> None:
+    """None: off; "*": time every kernel; otherwise time only the named kernel."""
+    lib.hs2_profile_enable(kernel.encode() if kernel is not None else None)
+
+
+def profile_read(kernel: str) -> tuple[float, int]:
+    """(summed milliseconds, launches) of the recorded launches of `kernel`; forgets them."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_longlong(0)
+    if lib.hs2_profile_read(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)) != 0:
+        raise HS2Error(ERR_CUDA, "hs2_profile_read")
+    return ms.value, n.value

@@ -23,6 +23,7 @@
 // owner), warps 2..5 = the 128 softmax threads (warp w reads TMEM lanes 32*(w%4)..+31).
 // Every wait is bounded; on timeout the kernel records it in the status word and unwinds.
 #include "decode.h"
+#include "host_util.h"
 #include "tc.cuh"
 
 namespace hs2 {
@@ -540,10 +541,22 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
                          (int)pass2_smem_bytes(H, D));
     configured = true;
   }
-  dec_pass1_kernel<H, D><<<p.G, NTHREADS, pass1_smem_bytes(H, D), stream>>>(tmK, tmQ, p);
-  dec_lse_combine_kernel<H><<<p.B, H, 0, stream>>>(p);
-  dec_pass2_kernel<H, D><<<p.G, NTHREADS, pass2_smem_bytes(H, D), stream>>>(tmK, tmV, tmQ, p);
-  dec_out_combine_kernel<H, D><<<dim3(p.B, H), D, 0, stream>>>(p, out);
+  {
+    LaunchScope ls("dec_pass1", stream);
+    dec_pass1_kernel<H, D><<<p.G, NTHREADS, pass1_smem_bytes(H, D), stream>>>(tmK, tmQ, p);
+  }
+  {
+    LaunchScope ls("dec_lse_combine", stream);
+    dec_lse_combine_kernel<H><<<p.B, H, 0, stream>>>(p);
+  }
+  {
+    LaunchScope ls("dec_pass2", stream);
+    dec_pass2_kernel<H, D><<<p.G, NTHREADS, pass2_smem_bytes(H, D), stream>>>(tmK, tmV, tmQ, p);
+  }
+  {
+    LaunchScope ls("dec_out_combine", stream);
+    dec_out_combine_kernel<H, D><<<dim3(p.B, H), D, 0, stream>>>(p, out);
+  }
   return cudaGetLastError();
 }
 

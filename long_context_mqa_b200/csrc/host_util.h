@@ -27,4 +27,17 @@ bool device_is_sm100();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch accounting: every kernel launch site wraps its launch in a LaunchScope, which counts
+// the launch and, when per-kernel timing is on for `name`, records CUDA events around it.
+class LaunchScope {
+ public:
+  LaunchScope(const char* name, cudaStream_t stream);
+  ~LaunchScope();
+
+ private:
+  int slot_;
+  cudaStream_t stream_;
+  const char* name_;
+};
+
 }  // namespace hs2

@@ -1,9 +1,13 @@
 // C ABI of the hs2 library (declared in include/hs2.h): argument validation, workspace
 // layout, TMA descriptor set-up and dispatch to the kernel files. No allocation, no
 // synchronisation and no host fallback on the compute paths.
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "decode.h"
 #include "host_util.h"
@@ -78,6 +82,50 @@ bool device_is_sm100() {
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
   return major == 10 && minor == 0;
+}
+
+// ------------------------------------------------------------------------------------------
+// launch accounting / optional per-kernel timing
+// ------------------------------------------------------------------------------------------
+static std::atomic<unsigned long long> g_launches{0};
+static std::atomic<bool> g_prof_on{false};
+static std::mutex g_prof_mu;
+static std::string g_prof_filter;
+static std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> g_prof;
+static std::vector<cudaEvent_t> g_event_pool;
+static thread_local cudaEvent_t t_pending_start = nullptr;
+
+static cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : slot_(-1), stream_(stream), name_(name) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (g_prof_filter != "*" && g_prof_filter != name) return;
+  cudaEvent_t a = take_event();
+  if (!a) return;
+  cudaEventRecord(a, stream);
+  t_pending_start = a;
+  slot_ = 0;
+}
+
+LaunchScope::~LaunchScope() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t b = take_event();
+  if (!b) return;
+  cudaEventRecord(b, stream_);
+  g_prof[name_].push_back({t_pending_start, b});
+  t_pending_start = nullptr;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -325,9 +373,56 @@ hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, lo
   if (!workspace || workspace_bytes < kStatusBytes) return HS2_ERR_WORKSPACE;
   if (limit_ns <= 0 || limit_ns > 10000000000LL) return HS2_ERR_INVALID_ARG;
   if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
-  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(reinterpret_cast<DevStatus*>(workspace),
-                                                                               limit_ns);
+  {
+    LaunchScope ls("selftest_wait", reinterpret_cast<cudaStream_t>(stream));
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<DevStatus*>(workspace), limit_ns);
+  }
   return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+unsigned long long hs2_kernel_launches(void) { return g_launches.load(); }
+
+void hs2_profile_enable(const char* kernel) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (kernel) {
+    g_prof_filter = kernel;
+    g_prof_on = true;
+  } else {
+    g_prof_filter.clear();
+    g_prof_on = false;
+  }
+}
+
+int hs2_profile_read(const char* kernel, double* total_ms, long long* launches) {
+  if (!kernel) return -1;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    auto it = g_prof.find(kernel);
+    if (it != g_prof.end()) {
+      recs.swap(it->second);
+      g_prof.erase(it);
+    }
+  }
+  double sum = 0.0;
+  int rc = 0;
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.second) != cudaSuccess || cudaEventElapsedTime(&ms, r.first, r.second) != cudaSuccess)
+      rc = -1;
+    sum += ms;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : recs) {
+      g_event_pool.push_back(r.first);
+      g_event_pool.push_back(r.second);
+    }
+  }
+  if (total_ms) *total_ms = sum;
+  if (launches) *launches = (long long)recs.size();
+  return rc;
 }
 
 }  // extern "C"

@@ -9,6 +9,7 @@
 //  3. final     : MSB-first 8-bit radix select of the `need` largest boundary keys, then the
 //                 forced window is appended and the <= 2048 indices are sorted ascending.
 #include "decode.h"
+#include "host_util.h"
 #include "tc.cuh"
 
 namespace hs2 {
@@ -201,13 +202,20 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
 }
 
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream) {
-  sel_threshold_kernel<<<p.B, NT, 0, stream>>>(p);
+  {
+    LaunchScope ls("sel_threshold", stream);
+    sel_threshold_kernel<<<p.B, NT, 0, stream>>>(p);
+  }
   if (p.ncand > 0) {
     int blocks = (p.ncand + NT - 1) / NT;
     if (blocks > 64) blocks = 64;
+    LaunchScope ls("sel_collect", stream);
     sel_collect_kernel<<<dim3(blocks, p.B), NT, 0, stream>>>(p);
   }
-  sel_final_kernel<<<p.B, NT, 0, stream>>>(p);
+  {
+    LaunchScope ls("sel_final", stream);
+    sel_final_kernel<<<p.B, NT, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@
 // 128 threads; thread r owns key row r of the tile (TMEM lane r) and, for O^T, output
 // column d = r (d = 128) or the M=64 lane layout (d = 64).
 #include "decode.h"
+#include "host_util.h"
 #include "tc.cuh"
 
 namespace hs2 {
@@ -344,8 +345,14 @@ static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
     configured = true;
   }
   const int rows = p.B * p.Lq;
-  sparse_attn_kernel<H, D><<<dim3(rows, p.nsplit), NT, SpLayout<H, D>::BYTES, stream>>>(p);
-  if (p.nsplit > 1) sparse_combine_kernel<H, D><<<dim3(rows, H), D, 0, stream>>>(p);
+  {
+    LaunchScope ls("sparse_attn", stream);
+    sparse_attn_kernel<H, D><<<dim3(rows, p.nsplit), NT, SpLayout<H, D>::BYTES, stream>>>(p);
+  }
+  if (p.nsplit > 1) {
+    LaunchScope ls("sparse_combine", stream);
+    sparse_combine_kernel<H, D><<<dim3(rows, H), D, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 
