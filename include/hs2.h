@@ -120,6 +120,25 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const h
                            void* workspace, size_t workspace_bytes, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
+ * Sparse attention without a caller workspace
+ * ---------------------------------------------------------------------------------
+ * No counterpart in the paper: a library convenience for callers that cannot allocate
+ * device memory -- e.g. a plugin's enqueue hook inside an inference runtime that forbids
+ * allocation on that path and offers no scratch buffer, or a process whose device-memory
+ * budget is fixed up front. Same arguments and results as hs2_sparse_attn, minus the
+ * workspace: the scratch is a 16 MiB array inside the library, held by every GPU that loads
+ * it until process exit. Returns HS2_ERR_WORKSPACE (nothing launched) when the shape needs
+ * more scratch than that (hs2_sparse_attn_workspace_bytes(...) > 16 MiB). The first call on
+ * each device performs a one-time set-up (it looks up the array's device address) and should
+ * come before any stream capture. All calls share the array: calls whose GPU work overlaps
+ * (e.g. on different streams) race. The device status word of these calls is internal.
+ * No cudaMalloc / cudaFree is ever called.
+ */
+HS2_API hs2_status hs2_sparse_attn_noalloc(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
+                                           const int32_t* idx, int B, int Lq, int Lk, int H, int d, int S,
+                                           float scale, hs2_bf16* out, float* lse, hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
  * KV Bridging projection
  * ---------------------------------------------------------------------------------
  * Hs   [T, hidden]                bf16  shared hidden state
