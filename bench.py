@@ -237,12 +237,28 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (small profiling cases)")
     ap.add_argument("--cache", type=int, default=0, help="override cache length (small profiling cases)")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the prefill full-attention + selection")
+    ap.add_argument("--prefill-len", type=int, default=0, help="override the prefill length (profiling cases)")
+    ap.add_argument("--sparse-layers", type=int, default=-1, help="prefill-only: sparse layers to time after it")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill_only:
+        return run_prefill_only(args)
     return run_gpu(args)
+
+
+def run_prefill_only(args):
+    """Prefill full attention + selection (and optionally its sparse layers) alone; one JSON line."""
+    import torch
+    world, rank, local = _dist_init()
+    dev = torch.device("cuda", local)
+    res = bench_prefill(args, world, dev, _peaks(), reps=max(1, args.steps), warmup=args.warmup)
+    if rank == 0:
+        print(json.dumps({"prefill": res}), flush=True)
+    return 0
 
 
 def _bf16(bits, device):
@@ -391,11 +407,13 @@ def run_gpu(args):
     return 0
 
 
-def bench_prefill(args, world, dev, peaks):
+def bench_prefill(args, world, dev, peaks, reps=5, warmup=2):
     """Full-attention + top-k prefill on the 32k workload: tok/s and tensor roofline."""
     import torch
     import long_context_mqa_b200 as hs2
     wl = synth.WORKLOADS[PREFILL_WORKLOAD]
+    if args.prefill_len:   # reduced case for profiler captures
+        wl = wl.with_(name=f"{PREFILL_WORKLOAD}_L{args.prefill_len}", Lq=args.prefill_len, Lk=args.prefill_len)
     g = synth.SyntheticInputs(wl, seed=args.seed)
     try:
         q, k, v = _bf16(g.q, dev), _bf16(g.k, dev), _bf16(g.v, dev)
@@ -405,10 +423,15 @@ def bench_prefill(args, world, dev, peaks):
         hs2.full_attn_select(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx)
     except Exception as e:  # the prefill path reports its own absence
         return {"status": f"unavailable: {e}"}
-    reps = 5
-    for _ in range(2):
+    n_sparse = wl.n_sparse if args.sparse_layers < 0 else args.sparse_layers
+    qs = [_bf16(g.q_sparse(i), dev) for i in range(n_sparse)]
+    outs = torch.empty_like(q)
+    for _ in range(warmup):
         hs2.full_attn_select(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx)
+        for i in range(n_sparse):
+            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs)
     _barrier(world)
+    hs2.profile_enable("*")
     s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s)
@@ -416,13 +439,30 @@ def bench_prefill(args, world, dev, peaks):
         hs2.full_attn_select(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx)
     e1.record(s)
     e1.synchronize()
+    hs2.profile_enable(None)
+    kern = {}
+    for name in ("fa_fwd", "score_select"):
+        kms, kn = hs2.profile_read(name)
+        kern[name] = kms / max(kn, 1)
+    if n_sparse:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(s)
+        for _ in range(reps):
+            for i in range(n_sparse):
+                hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs)
+        t1.record(s)
+        t1.synchronize()
+        kern["sparse_attn_per_layer"] = t0.elapsed_time(t1) / (reps * n_sparse)
+    for name in ("sparse_attn", "sparse_combine"):
+        hs2.profile_read(name)
     ms = _max_over_ranks(e0.elapsed_time(e1), world) / reps
     P = wl.Lq * (wl.Lq + 1) / 2
     exec_flops = 6 * wl.H * wl.d * P
     alg_flops = 4 * wl.H * wl.d * P
     tf = exec_flops / (ms / 1e3) / 1e12
-    return {"workload": f"{PREFILL_WORKLOAD}: L={wl.Lq}, H={wl.H}, d={wl.d}", "tok_per_s": world * wl.Lq / (ms / 1e3),
-            "ms": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops_sustained"],
+    return {"workload": f"{wl.name}: L={wl.Lq}, H={wl.H}, d={wl.d}", "tok_per_s": world * wl.Lq / (ms / 1e3),
+            "ms": ms, "kernel_ms": kern, "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops_sustained"],
                                    "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops_sustained"],
                                    "flops": "executed 6*H*d*L(L+1)/2 (QK^T twice, PV once)",
                                    "algorithmic_tflops": alg_flops / (ms / 1e3) / 1e12}}

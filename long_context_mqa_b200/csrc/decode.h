@@ -30,7 +30,7 @@ struct DecParams {
 size_t pass1_smem_bytes(int H, int D);
 size_t pass2_smem_bytes(int H, int D);
 cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                               const DecParams& p, __nv_bfloat16* out, cudaStream_t stream);
+                               const DecParams& p, cudaStream_t stream);
 }  // namespace dec
 
 namespace sel {
@@ -47,6 +47,11 @@ struct SelParams {
   unsigned long long* bnd;       // [B][ncand] boundary-bin candidates (score bits << 32 | ~index)
   int32_t* idx;                  // [B][S] output
   DevStatus* st;
+  // output partials of the decode passes, summed into out by the threshold kernel
+  const float* opart;            // [G*segmax][H][D]
+  __nv_bfloat16* out;            // [B][H][D]
+  int H, D, G, segmax, tps;
+  long long total_tiles;
 };
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
 }  // namespace sel

@@ -281,11 +281,12 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
         !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
         !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
       return HS2_ERR_CUDA;
-    if (cudaMemsetAsync(w.p.hist, 0, (size_t)B * sel::NBINS * sizeof(unsigned), st) != cudaSuccess)
-      return HS2_ERR_CUDA;
-    if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, reinterpret_cast<__nv_bfloat16*>(out), st) != cudaSuccess)
-      return HS2_ERR_CUDA;
+    if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, st) != cudaSuccess) return HS2_ERR_CUDA;
     sel::SelParams sp;
+    sp.opart = w.p.opart;
+    sp.out = reinterpret_cast<__nv_bfloat16*>(out);
+    sp.H = H; sp.D = d; sp.G = w.p.G; sp.segmax = w.p.segmax; sp.tps = w.p.tps;
+    sp.total_tiles = w.p.total_tiles;
     sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
     sp.ncand = Lk - window > 0 ? Lk - window : 0;
     sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.above = w.above; sp.bnd = w.bnd;

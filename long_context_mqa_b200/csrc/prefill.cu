@@ -540,7 +540,9 @@ __global__ void __launch_bounds__(NT, 1)
     const unsigned lt_mask = (1u << lane) - 1u;
     uint32_t kt = 0;
     bool ok = true;
-    for (int item = p.n_items - 1 - blockIdx.x; item >= 0 && ok; item -= gridDim.x) {
+    // after a failed wait every later wait returns at once: the loop and named-barrier
+    // structure stays identical across the warpgroup, only the tile work is skipped
+    for (int item = p.n_items - 1 - blockIdx.x; item >= 0; item -= gridDim.x) {
       const ScItem si = sc_item(p, item, C::NQ);
       // per-query state of this warpgroup's queries
       for (int q = wt; q < C::QW; q += 128) {
@@ -556,7 +558,8 @@ __global__ void __launch_bounds__(NT, 1)
       wg_bar(wg);
       for (int j = si.n_tiles - 1; j >= 0; --j, ++kt) {
         const int buf = kt & 1;
-        if (!warp_wait(&s_full[buf], (kt >> 1) & 1, limit, &abort_flag, p.st, 721)) { ok = false; break; }
+        if (ok && !warp_wait(&s_full[buf], (kt >> 1) & 1, limit, &abort_flag, p.st, 721)) ok = false;
+        if (ok) {
         tc_fence_after();
         const int key = j * 128 + row;
 #pragma unroll 1
@@ -588,6 +591,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[buf]);
+        }
         wg_bar(wg);
         for (int qq = 0; qq < C::QW; ++qq) {
           const int q = wg * C::QW + qq;
@@ -599,7 +603,6 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
-      if (!ok) break;
       // final: top-k of each query, plus the forced window, sorted ascending
       for (int qq = 0; qq < C::QW; ++qq) {
         const int q = wg * C::QW + qq;

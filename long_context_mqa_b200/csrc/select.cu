@@ -1,5 +1,7 @@
 // Exact top-k over a per-sequence score vector (decode path), ties to the lower index.
 //
+//  0. (same kernel as 1) the decode output: per sequence, the sum of the per-segment output
+//                 partials of the CTAs whose tile ranges cover it, rounded to bf16.
 //  1. threshold : from the 2048-bin histogram of score bits 30..20 (filled by decode pass 2),
 //                 find the bin beta that holds the k-th largest score; `above` = number of
 //                 scores in higher bins, `need` = k - above.
@@ -47,6 +49,22 @@ __global__ void __launch_bounds__(NT) sel_threshold_kernel(SelParams p) {
   __shared__ unsigned h[NBINS];
   __shared__ unsigned wt[32];
   int* meta = p.meta + b * META;
+  {
+    // decode output: CTAs c_lo..c_hi cover this sequence's tiles (contiguous split of the
+    // flattened tile space); slot = c * segmax + (b - first sequence of c)
+    const long long x_lo = (long long)b * p.tps, x_hi = (long long)(b + 1) * p.tps - 1;
+    const int c_lo = (int)(((x_lo + 1) * p.G - 1) / p.total_tiles);
+    const int c_hi = (int)(((x_hi + 1) * p.G - 1) / p.total_tiles);
+    for (int e = tid; e < p.H * p.D; e += NT) {
+      float acc = 0.f;
+      for (int c = c_lo; c <= c_hi; ++c) {
+        const long long ct0 = p.total_tiles * c / p.G;
+        const int slot = c * p.segmax + (b - (int)(ct0 / p.tps));
+        acc += p.opart[(size_t)slot * p.H * p.D + e];
+      }
+      p.out[(size_t)b * p.H * p.D + e] = __float2bfloat16_rn(acc);
+    }
+  }
   if (tid == 0) { meta[3] = 0; meta[4] = 0; }
   if (p.K == 0) {  // nothing is chosen by score
     if (tid == 0) { meta[0] = NBINS; meta[1] = 0; meta[2] = 0; }
