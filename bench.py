@@ -288,14 +288,24 @@ def run_gpu(args):
     outs = [torch.empty_like(q) for _ in range(wl.n_sparse)]
     ws_full = torch.zeros(hs2.full_attn_select_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d), dtype=torch.uint8,
                           device=dev)
-    ws_sp = torch.zeros(hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S), dtype=torch.uint8,
-                        device=dev)
+    ws_sp_bytes = hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S)
+    ws_sp = [torch.zeros(ws_sp_bytes, dtype=torch.uint8, device=dev) for _ in range(wl.n_sparse)]
     stream = torch.cuda.current_stream()
+    # the sparse layers of a hybrid block only depend on the full layer's indices: each runs on
+    # its own stream (and workspace) and the main stream joins them before the next step
+    side = [torch.cuda.Stream(device=dev) for _ in range(wl.n_sparse)]
+    ev_idx = torch.cuda.Event()
+    ev_done = [torch.cuda.Event() for _ in range(wl.n_sparse)]
 
     def step():
         hs2.full_attn_select(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws_full)
+        ev_idx.record(stream)
         for i in range(wl.n_sparse):
-            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp)
+            side[i].wait_event(ev_idx)
+            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i], stream=side[i])
+            ev_done[i].record(side[i])
+        for i in range(wl.n_sparse):
+            stream.wait_event(ev_done[i])
 
     # ---------------- device-resident throughput
     with ClockSampler(local) as clocks:
@@ -315,8 +325,20 @@ def run_gpu(args):
         _barrier(world)
     ms_total = _max_over_ranks(e0.elapsed_time(e1), world)
     pass2_ms, pass2_n = hs2.profile_read("dec_pass2")
+    # per-kernel breakdown (separate short run with every launch timed by CUDA events)
+    hs2.profile_enable("*")
+    n_brk = min(args.steps, 50)
+    for _ in range(n_brk):
+        step()
+    torch.cuda.synchronize()
+    hs2.profile_enable(None)
+    breakdown = {}
+    for name in ("dec_pass1", "dec_pass2", "sel_collect", "sel_final", "sparse_attn"):
+        kms, kn = hs2.profile_read(name)
+        if kn:
+            breakdown[name] = kms / n_brk
     status = hs2.read_device_status(ws_full)
-    status_sp = hs2.read_device_status(ws_sp)
+    status_sp = max(hs2.read_device_status(w) for w in ws_sp)
     ms_per_step = ms_total / args.steps
     value = world * args.steps / (ms_total / 1e3)
 
@@ -394,7 +416,7 @@ def run_gpu(args):
                                    f"{wl.n_sparse} sparse layers per step",
                        "global_batch": wl.B * world, "seq_len": wl.Lk, "parallelism": f"dp{world} (replicas)",
                        "l2": "inputs larger than L2 (1.07 GB K+V per GPU), no flush"},
-            "roofline": roofline, "step_roofline": step_roof,
+            "roofline": roofline, "step_roofline": step_roof, "kernel_ms_per_step": breakdown,
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "note": "public Python API, pinned host inputs, result read every step"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
@@ -454,8 +476,7 @@ def bench_prefill(args, world, dev, peaks, reps=5, warmup=2):
         t1.record(s)
         t1.synchronize()
         kern["sparse_attn_per_layer"] = t0.elapsed_time(t1) / (reps * n_sparse)
-    for name in ("sparse_attn", "sparse_combine"):
-        hs2.profile_read(name)
+    hs2.profile_read("sparse_attn")
     ms = _max_over_ranks(e0.elapsed_time(e1), world) / reps
     P = wl.Lq * (wl.Lq + 1) / 2
     exec_flops = 6 * wl.H * wl.d * P

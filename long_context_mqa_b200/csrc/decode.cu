@@ -18,8 +18,9 @@
 //           MN-major operand and O^T += V^T P^T accumulates in TMEM. Two softmax warpgroups take
 //           alternate tiles. Scores of older tokens go to a global buffer and a 2048-bin
 //           histogram of their top bits (warp-aggregated shared atomics).
-//   finish  per sequence (select.cu): sum of the output partials -> bf16 out, the histogram
-//           threshold of the top-k, then collect / final selection.
+//           The last CTA to finish a sequence scans that sequence's histogram for the bin of
+//           its k-th largest score.
+//   finish  (select.cu) sum of the output partials -> bf16 out; collect / final selection.
 //
 // Work split: the flattened (sequence, 128-key tile) space is cut into G contiguous ranges,
 // one per CTA (G = number of SMs); a range may cross a sequence boundary, so a CTA handles
@@ -104,8 +105,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tile_range(p, cta, t0, t1);
   const long long limit = p.wait_ns;
 
-  if (cta == 0)  // pass 2 accumulates into the selection histogram
+  if (cta == 0) {  // pass 2 accumulates into the selection histogram and per-sequence counters
     for (int i = threadIdx.x; i < p.B * 2048; i += NTHREADS) p.hist[i] = 0u;
+    for (int i = threadIdx.x; i < p.B; i += NTHREADS) p.seq_done[i] = 0;
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
@@ -120,6 +123,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  griddep_launch_dependents();  // pass 2 may start streaming K/V into freed SMs
 
   if (warp == 0) {
     if (lane == 0) {
@@ -307,6 +311,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ __align__(16) float slse[H];
+  __shared__ int s_last;
+  __shared__ unsigned s_wtot[8];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -333,6 +339,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  griddep_launch_dependents();
+  // Launched early (programmatic dependent launch): the producers and the tensor core only read
+  // K, V and Q, so they start at once; the softmax warps wait for pass 1 to complete before they
+  // read its partials or touch the histogram / counters it cleared.
 
   // segments are walked from the end of the range backwards, tiles likewise
   if (warp == 0) {
@@ -439,6 +449,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int all_tid = wg * 128 + wg_tid;  // 0..255 over both warpgroups
     const float c = p.c;
     const int ncand = p.N - p.W > 0 ? p.N - p.W : 0;
+    griddep_wait();
     uint32_t j = 0;
     int seg = 0;
     bool ok = true;
@@ -545,6 +556,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t cnt = shist[i];
         if (cnt) { atomicAdd(&p.hist[(size_t)b * NBINS + i], cnt); shist[i] = 0; }
       }
+      __threadfence();
+      named_bar(3, 256);
+      // the last CTA to finish this sequence finds the bin of its k-th largest score
+      if (all_tid == 0) {
+        const int c_lo = cta_of_tile(p, (long long)b * p.tps), c_hi = cta_of_tile(p, (long long)(b + 1) * p.tps - 1);
+        s_last = atomicAdd(&p.seq_done[b], 1) == c_hi - c_lo;
+      }
+      named_bar(3, 256);
+      if (s_last) {
+        __threadfence();
+        int* meta = p.meta + b * 8;
+        const int K = p.K_sel;
+        if (ncand <= K || K == 0) {
+          if (all_tid == 0) {
+            meta[0] = K == 0 ? NBINS : -1;  // -1: every older token; NBINS: none
+            meta[1] = K == 0 ? 0 : ncand;
+            meta[2] = 0; meta[3] = 0; meta[4] = 0;
+          }
+        } else {
+          // thread i owns bins hi..hi-7 (descending); block-inclusive scan of their counts
+          const int hi = NBINS - 1 - 8 * all_tid;
+          unsigned cnt8[8], local = 0;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) { cnt8[x] = __ldcg(&p.hist[(size_t)b * NBINS + hi - x]); local += cnt8[x]; }
+          unsigned incl = local;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned nb = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nb;
+          }
+          const int wv = all_tid >> 5;
+          if (lane == 31) s_wtot[wv] = incl;
+          named_bar(3, 256);
+          unsigned add = 0;
+          for (int x = 0; x < wv; ++x) add += s_wtot[x];
+          incl += add;
+          const unsigned excl = incl - local;
+          if (excl < (unsigned)K && incl >= (unsigned)K) {
+            unsigned run = excl;
+            for (int x = 0; x < 8; ++x) {
+              if (run + cnt8[x] >= (unsigned)K) {
+                meta[0] = hi - x; meta[1] = (int)run; meta[2] = (int)(K - run); meta[3] = 0; meta[4] = 0;
+                break;
+              }
+              run += cnt8[x];
+            }
+          }
+        }
+      }
       named_bar(3, 256);
     }
   }
@@ -576,10 +636,13 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
     LaunchScope ls("dec_pass1", stream);
     dec_pass1_kernel<H, D><<<p.G, NTHREADS, pass1_smem_bytes(H, D), stream>>>(tmK, tmQ, p);
   }
+  cudaError_t e;
   {
     LaunchScope ls("dec_pass2", stream);
-    dec_pass2_kernel<H, D><<<p.G, NTHREADS, pass2_smem_bytes(H, D), stream>>>(tmK, tmV, tmQ, p);
+    e = launch_k(dec_pass2_kernel<H, D>, dim3(p.G), dim3(NTHREADS), pass2_smem_bytes(H, D), stream, true, tmK, tmV,
+                 tmQ, p);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

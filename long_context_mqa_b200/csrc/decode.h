@@ -25,6 +25,9 @@ struct DecParams {
   float* opart;            // [G*segmax][H][D] pass-2 partial outputs
   float* sc;               // [B][N-W] head-summed scores of the older tokens
   unsigned* hist;          // [B][2048] histogram of score bits 30..20
+  int* seq_done;           // [B] pass-2 CTAs done with each sequence's histogram
+  int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
+  int K_sel;               // top-k of the selection (== K)
   DevStatus* st;
 };
 size_t pass1_smem_bytes(int H, int D);
@@ -67,6 +70,7 @@ struct SpParams {
   float* lse;                 // may be null
   float* opart;               // [B*Lq*nsplit][H][D] (nsplit > 1)
   float* mlpart;              // [B*Lq*nsplit][2][H]
+  int* counters;              // [B*Lq] split arrivals (zeroed before every launch)
   long long wait_ns;
   DevStatus* st;
 };

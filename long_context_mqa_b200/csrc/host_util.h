@@ -7,6 +7,8 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hs2.h"
 
 namespace hs2 {
@@ -26,6 +28,25 @@ int num_sms();
 bool device_is_sm100();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launches `kernel` on `stream`; with pdl = true the launch may begin while the previous
+// kernel on the stream is still running (the kernel must call griddep_wait() before it reads
+// anything that kernel wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launch accounting: every kernel launch site wraps its launch in a LaunchScope, which counts
 // the launch and, when per-kernel timing is on for `name`, records CUDA events around it.

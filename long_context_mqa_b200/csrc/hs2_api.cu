@@ -160,6 +160,7 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   p.B = B; p.N = N; p.W = W; p.K = K;
   p.tps = (N + 127) / 128;
   p.total_tiles = (long long)B * p.tps;
+  if (sms > 256) sms = 256;  // the output combine keeps one table entry per covering CTA
   p.G = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   int segmax = 1;
   for (int cta = 0; cta < p.G; ++cta) {
@@ -178,7 +179,10 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   p.opart = c.take<float>((size_t)p.G * segmax * H * D);
   p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
+  p.seq_done = c.take<int>((size_t)B);
   w.meta = c.take<int>((size_t)B * sel::META);
+  p.meta = w.meta;
+  p.K_sel = K;
   w.above = c.take<int>((size_t)B * (K > 0 ? K : 1));
   w.bnd = c.take<unsigned long long>((size_t)B * (ncand > 0 ? ncand : 1));
   w.bytes = c.off;
@@ -195,14 +199,17 @@ static size_t carve_sparse(void* ws, int B, int Lq, int H, int D, int S, int sms
   DevStatus* st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
   float* opart = nullptr;
   float* mlpart = nullptr;
+  int* counters = nullptr;
   if (nsplit > 1) {
     opart = c.take<float>((size_t)rows * nsplit * H * D);
     mlpart = c.take<float>((size_t)rows * nsplit * 2 * H);
+    counters = c.take<int>((size_t)rows);
   }
   if (p) {
     p->st = st;
     p->opart = opart;
     p->mlpart = mlpart;
+    p->counters = counters;
     p->nsplit = nsplit;
     p->split_slots = nsplit > 1 ? 128 : tiles * 128;
   }

@@ -8,8 +8,10 @@
 //                             max is only raised when a tile exceeds it by more than 2^8,
 //                             so O^T is rarely rescaled)
 //   O^T += V_sel^T P^T       tcgen05, M = d, N = 64 (heads padded to 64), P^T MN-major bf16
-// Gathers of tile t+1 overlap the math of tile t. With one split the CTA writes the final
-// bf16 output (and lse); with several, unnormalised partials that a combine kernel merges.
+// With several tiles per CTA, the gathers of tile t+1 overlap the math of tile t (2 stages);
+// with one tile per CTA (few query rows: decode) a single stage keeps two CTAs per SM. With one
+// split the CTA writes the final bf16 output (and lse); with several, every split writes an
+// unnormalised partial, and the split that arrives last on the row's counter merges them.
 // 128 threads; thread r owns key row r of the tile (TMEM lane r) and, for O^T, output
 // column d = r (d = 128) or the M=64 lane layout (d = 64).
 #include "decode.h"
@@ -23,33 +25,41 @@ constexpr int TILE = 128;
 constexpr int NT = 128;
 constexpr float RESCALE_SLACK = 8.f;  // log2 units
 
-template <int H, int D>
+template <int H, int D, int STAGES>
 struct SpLayout {
   static constexpr int HP = 64;                       // heads padded for the PV MMA
   static constexpr int Q_BYTES = H * D * 2;           // K-major B operand, H rows
   static constexpr int KT_BYTES = TILE * D * 2;
-  static constexpr int X_STRIDE = H + 1;              // floats per row of the transpose buffer
-  static constexpr int X_BYTES = TILE * X_STRIDE * 4;
+  static constexpr int X_BYTES = TILE * H * 4;          // transpose buffer, XOR-swizzled columns
   static constexpr int P_BYTES = TILE * HP * 2;
-  static constexpr int XP_BYTES = X_BYTES > P_BYTES ? X_BYTES : P_BYTES;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = ((Q_BYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_V = OFF_K + 2 * KT_BYTES;
-  static constexpr int OFF_XP = OFF_V + 2 * KT_BYTES;
-  static constexpr int BYTES = OFF_XP + ((XP_BYTES + 1023) / 1024) * 1024 + 1024;
+  static constexpr int OFF_V = OFF_K + STAGES * KT_BYTES;
+  static constexpr int OFF_P = OFF_V + STAGES * KT_BYTES;
+  // one stage: the K tile is dead once S^T is in TMEM, so the transpose buffer reuses it;
+  // two stages: it shares the P^T buffer (P^T is written after the transpose is read)
+  static constexpr int XP_BYTES = STAGES == 1 ? P_BYTES : (X_BYTES > P_BYTES ? X_BYTES : P_BYTES);
+  static constexpr int OFF_X = STAGES == 1 ? OFF_K : OFF_P;
+  static_assert(STAGES == 2 || X_BYTES <= KT_BYTES, "transpose buffer must fit the K tile");
+  static constexpr int BYTES = OFF_P + ((XP_BYTES + 1023) / 1024) * 1024 + 1024;
 };
+// element (row, h) of the transpose buffer; the XOR keeps both access patterns conflict-free
+template <int H>
+__device__ __forceinline__ int xidx(int row, int h) {
+  return row * H + (h ^ (row & ((H < 32 ? H : 32) - 1)));
+}
 
-template <int H, int D>
+template <int H, int D, int STAGES>
 __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
-  using Lay = SpLayout<H, D>;
+  using Lay = SpLayout<H, D, STAGES>;
   constexpr int HP = Lay::HP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem + Lay::OFF_Q;
   uint8_t* sK = smem + Lay::OFF_K;
   uint8_t* sV = smem + Lay::OFF_V;
-  float* sX = (float*)(smem + Lay::OFF_XP);
-  uint8_t* sP = smem + Lay::OFF_XP;
+  float* sX = (float*)(smem + Lay::OFF_X);
+  uint8_t* sP = smem + Lay::OFF_P;
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ float sM[H], sAlpha[H], sL[H];
@@ -68,14 +78,12 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
   const __nv_bfloat16* Vb = p.V + (size_t)b * p.Lk * D;
   const uint32_t tS = 0, tO = 64;
 
-  // ---- query -> shared (K-major, 128B swizzle), barrier + TMEM set-up
+  // ---- query -> shared (K-major, 128B swizzle) by cp.async, in flight with tile 0's gather
   {
     const __nv_bfloat16* q = p.Q + (size_t)r * H * D;
     for (int c = tid; c < H * D / 8; c += NT) {
       const int row = c / (D / 8), ch = c % (D / 8);
-      const uint4 val = *reinterpret_cast<const uint4*>(q + row * D + ch * 8);
-      const uint32_t dst = smem_u32(sQ) + (ch / 8) * (H * 128) + sw128_off(row, ch % 8);
-      st_shared_v4(dst, val.x, val.y, val.z, val.w);
+      cp_async_16(smem_u32(sQ) + (ch / 8) * (H * 128) + sw128_off(row, ch % 8), q + row * D + ch * 8, true);
     }
   }
   if (tid < H) { sM[tid] = -INFINITY; sAlpha[tid] = 1.f; }
@@ -118,9 +126,9 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
   const int quarter = warp & 3;
 
   for (int t = 0; t < ntiles && ok; ++t) {
-    const int buf = t & 1;
+    const int buf = STAGES == 2 ? (t & 1) : 0;
     bool valid_next = false;
-    if (t + 1 < ntiles) {
+    if (STAGES == 2 && t + 1 < ntiles) {
       valid_next = gather(t + 1, buf ^ 1);
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
 #pragma unroll
     for (int h = 0; h < H; ++h) {
       x[h] = valid_cur ? x[h] * c : -INFINITY;
-      sX[row * Lay::X_STRIDE + h] = x[h];
+      sX[xidx<H>(row, h)] = x[h];
     }
     __syncthreads();
     // ---- per-head tile max: TPH threads per head
@@ -172,7 +180,7 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
       constexpr int ROWS = TILE / TPH;
       const int h = tid / TPH, part = tid % TPH;
       float mx = -INFINITY;
-      for (int q2 = 0; q2 < ROWS; ++q2) mx = fmaxf(mx, sX[(part * ROWS + q2) * Lay::X_STRIDE + h]);
+      for (int q2 = 0; q2 < ROWS; ++q2) mx = fmaxf(mx, sX[xidx<H>(part * ROWS + q2, h)]);
 #pragma unroll
       for (int o = 1; o < TPH; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (part == 0) {
@@ -222,7 +230,7 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
         tmem_st_wait();
       }
     }
-    // sX reads are complete (barrier above) -> P^T may overwrite the shared buffer
+    // sX reads are complete (barrier above) -> P^T may overwrite it (two stages share it)
     {
       const uint32_t prow = smem_u32(sP);
 #pragma unroll
@@ -252,16 +260,20 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
     }
     phase ^= 1;
     tc_fence_after();
+    if (STAGES == 1 && t + 1 < ntiles && ok) {  // the only stage is free again
+      valid_next = gather(t + 1, 0);
+      fence_async_smem();
+    }
     valid_cur = valid_next;
   }
   cp_async_wait_all();
   // ---- row sums across the 128 key lanes
 #pragma unroll
-  for (int h = 0; h < H; ++h) sX[tid * Lay::X_STRIDE + h] = lsum[h];
+  for (int h = 0; h < H; ++h) sX[xidx<H>(tid, h)] = lsum[h];
   __syncthreads();
   if (tid < H) {
     float s = 0.f;
-    for (int q2 = 0; q2 < TILE; ++q2) s += sX[q2 * Lay::X_STRIDE + tid];
+    for (int q2 = 0; q2 < TILE; ++q2) s += sX[xidx<H>(q2, tid)];
     sL[tid] = s;
   }
   __syncthreads();
@@ -307,58 +319,76 @@ __global__ void __launch_bounds__(NT, 1) sparse_attn_kernel(SpParams p) {
   tc_fence_before();
   __syncthreads();
   if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 128); }
-}
-
-template <int H, int D>
-__global__ void sparse_combine_kernel(SpParams p) {
-  const int r = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
-  float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float* ml = p.mlpart + ((size_t)r * p.nsplit + s) * 2 * H;
-    if (ml[H + h] > 0.f) M = fmaxf(M, ml[h]);
+  if (p.nsplit > 1) {
+    // the split that arrives last on this row's counter merges the row's partials
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.counters[r], 1) == p.nsplit - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      float* wgt = sX;  // [nsplit][H] merge weights, then [H] 1 / L
+      const float* mlr = p.mlpart + (size_t)r * p.nsplit * 2 * H;
+      if (tid < H) {
+        float M = -INFINITY, L = 0.f;
+        for (int s2 = 0; s2 < p.nsplit; ++s2)
+          if (mlr[s2 * 2 * H + H + tid] > 0.f) M = fmaxf(M, mlr[s2 * 2 * H + tid]);
+        for (int s2 = 0; s2 < p.nsplit; ++s2) {
+          const float l = mlr[s2 * 2 * H + H + tid];
+          const float w = l > 0.f ? exp2f(mlr[s2 * 2 * H + tid] - M) : 0.f;
+          wgt[s2 * H + tid] = w;
+          L += l * w;
+        }
+        wgt[p.nsplit * H + tid] = L > 0.f ? 1.f / L : 0.f;
+        if (p.lse) p.lse[(size_t)r * H + tid] = (M + log2f(L)) * 0.69314718055994531f;
+      }
+      __syncthreads();
+      const float4* op = reinterpret_cast<const float4*>(p.opart + (size_t)r * p.nsplit * H * D);
+      for (int e = tid; e < H * D / 4; e += NT) {
+        const int h = e / (D / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s2 = 0; s2 < p.nsplit; ++s2) {
+          const float w = wgt[s2 * H + h];
+          const float4 v4 = op[(size_t)s2 * (H * D / 4) + e];
+          acc.x += w * v4.x; acc.y += w * v4.y; acc.z += w * v4.z; acc.w += w * v4.w;
+        }
+        const float inv = wgt[p.nsplit * H + h];
+        uint2 o2;
+        o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        reinterpret_cast<uint2*>(p.out + (size_t)r * H * D)[e] = o2;
+      }
+    }
   }
-  float acc = 0.f, L = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float* ml = p.mlpart + ((size_t)r * p.nsplit + s) * 2 * H;
-    const float l = ml[H + h];
-    if (!(l > 0.f)) continue;
-    const float w = exp2f(ml[h] - M);
-    L += l * w;
-    acc += w * p.opart[(((size_t)r * p.nsplit + s) * H + h) * D + d];
-  }
-  p.out[((size_t)r * H + h) * D + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-  if (d == 0 && p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
 size_t sparse_smem_bytes(int H, int D) {
-  if (H == 64 && D == 128) return SpLayout<64, 128>::BYTES;
-  if (H == 16 && D == 64) return SpLayout<16, 64>::BYTES;
+  if (H == 64 && D == 128) return SpLayout<64, 128, 2>::BYTES;
+  if (H == 16 && D == 64) return SpLayout<16, 64, 2>::BYTES;
   return 0;
 }
 
-template <int H, int D>
+template <int H, int D, int STAGES>
 static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         SpLayout<H, D>::BYTES);
+    cudaFuncSetAttribute(sparse_attn_kernel<H, D, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         SpLayout<H, D, STAGES>::BYTES);
     configured = true;
   }
   const int rows = p.B * p.Lq;
-  {
-    LaunchScope ls("sparse_attn", stream);
-    sparse_attn_kernel<H, D><<<dim3(rows, p.nsplit), NT, SpLayout<H, D>::BYTES, stream>>>(p);
-  }
-  if (p.nsplit > 1) {
-    LaunchScope ls("sparse_combine", stream);
-    sparse_combine_kernel<H, D><<<dim3(rows, H), D, 0, stream>>>(p);
-  }
+  if (p.nsplit > 1 && cudaMemsetAsync(p.counters, 0, (size_t)rows * sizeof(int), stream) != cudaSuccess)
+    return cudaErrorUnknown;
+  LaunchScope ls("sparse_attn", stream);
+  sparse_attn_kernel<H, D, STAGES><<<dim3(rows, p.nsplit), NT, SpLayout<H, D, STAGES>::BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse(const SpParams& p, int H, int D, cudaStream_t stream) {
-  if (H == 64 && D == 128) return launch_t<64, 128>(p, stream);
-  if (H == 16 && D == 64) return launch_t<16, 64>(p, stream);
+  const bool one_tile = p.split_slots <= 128;  // one tile per CTA: a single stage suffices
+  if (H == 64 && D == 128) return one_tile ? launch_t<64, 128, 1>(p, stream) : launch_t<64, 128, 2>(p, stream);
+  if (H == 16 && D == 64) return one_tile ? launch_t<16, 64, 1>(p, stream) : launch_t<16, 64, 2>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -241,6 +241,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------------------------
+// programmatic dependent launch
+// ------------------------------------------------------------------------------------
+// Blocks until the grids this one depends on (launched before it on the stream with the
+// programmatic-serialization attribute) have completed and their memory is visible.
+// A no-op when the kernel was launched without that attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next grid on the stream start launching (its CTAs still wait in griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------
 // small math helpers
 // ------------------------------------------------------------------------------------
 __device__ __forceinline__ float fast_exp2(float x) {
