@@ -94,7 +94,7 @@ HS2_API const char* hs2_status_string(hs2_status s);
  * idx  [B, Lq, window+topk] int32  selected token indices of each query, ascending;
  *                           exactly min(t+1, window+topk) valid entries, then -1 padding
  * Supported: (H, d) in {(64, 128), (16, 64)}; Lq == 1 or Lq == Lk (bf16, fp32 accumulate).
- * Decode (Lq == 1) supports (H, d) = (64, 128).
+ * Decode (Lq == 1) supports (H, d) = (64, 128); prefill (Lq == Lk) supports topk <= 1024.
  */
 HS2_API size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk);
 HS2_API hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,

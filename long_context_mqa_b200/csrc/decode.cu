@@ -109,6 +109,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = threadIdx.x; i < p.B * 2048; i += NTHREADS) p.hist[i] = 0u;
     for (int i = threadIdx.x; i < p.B; i += NTHREADS) p.seq_done[i] = 0;
   }
+  {  // the selection bitmap, cleared by all CTAs (the collect kernel sets bits)
+    const long long total = (long long)p.B * p.words;
+    const long long per = (total + p.G - 1) / p.G;
+    const long long w0 = per * cta, w1 = w0 + per < total ? w0 + per : total;
+    for (long long i = w0 + threadIdx.x; i < w1; i += NTHREADS) p.bitmap[i] = 0u;
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {

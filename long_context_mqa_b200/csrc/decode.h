@@ -26,6 +26,8 @@ struct DecParams {
   float* sc;               // [B][N-W] head-summed scores of the older tokens
   unsigned* hist;          // [B][2048] histogram of score bits 30..20
   int* seq_done;           // [B] pass-2 CTAs done with each sequence's histogram
+  unsigned* bitmap;        // [B][words] selection bitmap of the older tokens (cleared by pass 1)
+  int words;               // ceil((N - W) / 32)
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
   DevStatus* st;
@@ -38,7 +40,7 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
 
 namespace sel {
 constexpr int NBINS = 2048;
-constexpr int META = 8;  // ints per sequence: beta, above, need, cnt_above, cnt_bnd
+constexpr int META = 8;  // ints per sequence: beta, above, need, (unused), cnt_bnd
 // Top-k selection over a materialised score vector per sequence (decode path).
 struct SelParams {
   int B, N, W, K, S;
@@ -46,7 +48,8 @@ struct SelParams {
   const float* sc;               // [B][ncand]
   const unsigned* hist;          // [B][NBINS]
   int* meta;                     // [B][META]
-  int* above;                    // [B][K]
+  unsigned* bitmap;              // [B][words] chosen older tokens, one bit each
+  int words;
   unsigned long long* bnd;       // [B][ncand] boundary-bin candidates (score bits << 32 | ~index)
   int32_t* idx;                  // [B][S] output
   DevStatus* st;

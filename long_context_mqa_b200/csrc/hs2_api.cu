@@ -149,7 +149,6 @@ struct Carve {
 struct DecodeWs {
   dec::DecParams p;
   int* meta;
-  int* above;
   unsigned long long* bnd;
   size_t bytes;
 };
@@ -183,7 +182,8 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   w.meta = c.take<int>((size_t)B * sel::META);
   p.meta = w.meta;
   p.K_sel = K;
-  w.above = c.take<int>((size_t)B * (K > 0 ? K : 1));
+  p.words = (ncand + 31) / 32;
+  p.bitmap = c.take<unsigned>((size_t)B * (p.words > 0 ? p.words : 1));
   w.bnd = c.take<unsigned long long>((size_t)B * (ncand > 0 ? ncand : 1));
   w.bytes = c.off;
   return w;
@@ -296,7 +296,8 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
     sp.total_tiles = w.p.total_tiles;
     sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
     sp.ncand = Lk - window > 0 ? Lk - window : 0;
-    sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.above = w.above; sp.bnd = w.bnd;
+    sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.bnd = w.bnd;
+    sp.bitmap = w.p.bitmap; sp.words = w.p.words;
     sp.idx = idx; sp.st = w.p.st;
     if (sel::launch_select(sp, st) != cudaSuccess) return HS2_ERR_CUDA;
     return HS2_OK;

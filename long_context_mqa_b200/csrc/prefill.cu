@@ -250,19 +250,23 @@ __global__ void __launch_bounds__(NT, 1)
         if (!warp_wait(&s_full[w], n_s & 1, limit, &abort_flag, p.st, 621)) { ok = false; break; }
         n_s++;
         tc_fence_after();
-        // pass over S: row max of the visible keys
-        float mx = -INFINITY;
+        // causal masking only where the tile reaches past some row's query (warp-uniform)
+        const bool masked = __any_sync(0xffffffffu, j * 128 + 127 > t);
+        const int kvis = t - j * 128;  // keys 0..kvis of this tile are visible to this row
+        // pass over S: max of the raw logits (c > 0, so scaling commutes with the max)
+        float rmax = -INFINITY;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           float v[32];
           tmem_ld32(sS + cc * 32, v);
           tmem_ld_wait();
+          if (masked) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int key = j * 128 + cc * 32 + x;
-            if (key <= t) mx = fmaxf(mx, v[x] * c);
+            for (int x = 0; x < 32; ++x) v[x] = cc * 32 + x <= kvis ? v[x] : -INFINITY;
           }
+          rmax = fmaxf(rmax, max32(v));
         }
+        const float mx = rmax * c;
         const bool raise = mx > -INFINITY && (m_used == -INFINITY || mx > m_used + 8.f);
         const float m_new = raise ? mx : m_used;
         const float alpha = raise ? (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new)) : 1.f;
@@ -286,7 +290,9 @@ __global__ void __launch_bounds__(NT, 1)
         }
         l *= alpha;
         m_used = m_new;
+        const float negm = -m_used;
         // probabilities -> P (K-major: row = this thread's (query, head), K = the 128 keys)
+        float la = 0.f, lb = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           float v[32];
@@ -295,10 +301,14 @@ __global__ void __launch_bounds__(NT, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            const int key = j * 128 + cc * 32 + x;
-            const float p0 = key <= t ? fast_exp2(fmaf(v[x], c, -m_used)) : 0.f;
-            const float p1 = key + 1 <= t ? fast_exp2(fmaf(v[x + 1], c, -m_used)) : 0.f;
-            l += p0 + p1;
+            float e0, e1;
+            ffma2(e0, e1, v[x], v[x + 1], c, c, negm, negm);
+            float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
+            if (masked) {
+              p0 = cc * 32 + x <= kvis ? p0 : 0.f;
+              p1 = cc * 32 + x + 1 <= kvis ? p1 : 0.f;
+            }
+            fadd2(la, lb, la, lb, p0, p1);
             pk[x / 2] = pack_bf16x2(p0, p1);
           }
           const uint32_t blk = pbase + (cc / 2) * (128 * 128);
@@ -306,6 +316,7 @@ __global__ void __launch_bounds__(NT, 1)
           for (int q = 0; q < 4; ++q)
             st_shared_v4(blk + sw128_off(row, (cc % 2) * 4 + q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
+        l += la + lb;
         tc_fence_before();
         fence_async_smem();
         __syncwarp();
@@ -377,10 +388,30 @@ __device__ __forceinline__ ScItem sc_item(const PfParams& p, int item, int nq) {
 template <int CAP>
 __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int keep, int wg, int wt, unsigned* hist,
                                          unsigned long long* s_prefix, int* s_need, int* s_cnt) {
-  if (wt == 0) { *s_prefix = 0ull; *s_need = keep; *s_cnt = 0; }
-  unsigned long long mask = 0ull;
+  // bits on which all n keys agree need no radix pass: find the highest differing bit first
+  __shared__ unsigned long long s_and[2], s_or[2];
+  __shared__ int s_exact[2];
+  if (wt == 0) { s_and[wg] = ~0ull; s_or[wg] = 0ull; *s_need = keep; *s_cnt = 0; s_exact[wg] = 0; }
   wg_bar(wg);
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  {
+    unsigned long long a = ~0ull, o = 0ull;
+    for (int i = wt; i < n; i += 128) { const unsigned long long key = buf[i]; a &= key; o |= key; }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      a &= __shfl_xor_sync(0xffffffffu, a, off);
+      o |= __shfl_xor_sync(0xffffffffu, o, off);
+    }
+    if ((wt & 31) == 0) { atomicAnd(&s_and[wg], a); atomicOr(&s_or[wg], o); }
+  }
+  wg_bar(wg);
+  const unsigned long long diff = s_and[wg] ^ s_or[wg];
+  const int top = diff ? 63 - __clzll((long long)diff) : 0;
+  unsigned long long mask = top >= 63 ? 0ull : ~((2ull << top) - 1ull);
+  if (wt == 0) *s_prefix = s_and[wg] & mask;
+  wg_bar(wg);
+  // 8-bit digit windows from the highest differing bit down; the last is clamped at bit 0
+  for (int sh_raw = top - 7;; sh_raw -= 8) {
+    const int shift = sh_raw < 0 ? 0 : sh_raw;
     for (int i = wt; i < 256; i += 128) hist[i] = 0u;
     wg_bar(wg);
     const unsigned long long prefix = *s_prefix;
@@ -408,6 +439,7 @@ __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int kee
           if (run + cnt[x] >= k) {
             *s_need = (int)(k - run);
             *s_prefix = prefix | ((unsigned long long)(255u - 8u * ln - x) << shift);
+            s_exact[wg] = run + cnt[x] == k;  // the whole bucket is kept: no further digit needed
             break;
           }
           run += cnt[x];
@@ -416,7 +448,9 @@ __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int kee
     }
     mask |= 255ull << shift;
     wg_bar(wg);
+    if (shift == 0 || s_exact[wg]) break;
   }
+  // keys whose masked prefix is >= the chosen prefix are exactly the `keep` largest
   const unsigned long long thr = *s_prefix;
   constexpr int PER = CAP / 128;
   unsigned long long mine[PER];
@@ -427,7 +461,7 @@ __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int kee
     mine[m] = 0ull;
     if (i < n) {
       const unsigned long long key = buf[i];
-      if (key >= thr) { mine[m] = key; nm++; }
+      if ((key & mask) >= thr) { mine[m] = key; nm++; }
     }
   }
   wg_bar(wg);
@@ -449,7 +483,7 @@ __global__ void __launch_bounds__(NT, 1)
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[C::KST], k_empty[C::KST], s_full[2], s_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
-  __shared__ float slse2[256];
+  __shared__ __align__(16) float slse2[256];
   __shared__ int cnt[C::NQ];
   __shared__ unsigned long long theta[C::NQ];
   __shared__ unsigned hist[2][256];
@@ -553,7 +587,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int q = wg * C::QW + x / H, h = x % H;
         const int t = si.tq0 + q;
         const float l = t < p.L ? p.lse[((size_t)si.b * p.L + t) * H + h] : 0.f;
-        slse2[q * H + h] = l * LOG2E;
+        slse2[q * H + h] = -l * LOG2E;  // stored negated: one FFMA gives s*c - lse2
       }
       wg_bar(wg);
       for (int j = si.n_tiles - 1; j >= 0; --j, ++kt) {
@@ -567,15 +601,24 @@ __global__ void __launch_bounds__(NT, 1)
           const int q = wg * C::QW + qq;
           const int t = si.tq0 + q;
           const bool cand = t < p.L && key <= t - p.W;
-          float score = 0.f;
+          if (!__any_sync(0xffffffffu, cand)) continue;  // warp-uniform: no lane has a candidate here
+          float sa = 0.f, sb = 0.f;
 #pragma unroll
           for (int hc = 0; hc < H; hc += 16) {
             float v[16];
             tmem_ld16(tmem + lane_base + buf * 256 + q * H + hc, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int x = 0; x < 16; ++x) score += fast_exp2(fmaf(v[x], c, -slse2[q * H + hc + x]));
+            for (int x = 0; x < 16; x += 4) {
+              const float4 nl = *reinterpret_cast<const float4*>(&slse2[q * H + hc + x]);  // -lse2
+              float e0, e1, e2, e3;
+              ffma2(e0, e1, v[x], v[x + 1], c, c, nl.x, nl.y);
+              ffma2(e2, e3, v[x + 2], v[x + 3], c, c, nl.z, nl.w);
+              fadd2(sa, sb, sa, sb, fast_exp2(e0), fast_exp2(e1));
+              fadd2(sa, sb, sa, sb, fast_exp2(e2), fast_exp2(e3));
+            }
           }
+          const float score = sa + sb;
           const unsigned long long k64 =
               ((unsigned long long)__float_as_uint(score) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)key);
           const bool take = cand && k64 > theta[q];
@@ -624,18 +667,16 @@ __global__ void __launch_bounds__(NT, 1)
         int* ib32 = reinterpret_cast<int*>(qb);
         const int wlo = t - p.W + 1 > 0 ? t - p.W + 1 : 0;
         const int wlen = t - wlo + 1;
+        // the picks (<= topk <= 1024) are sorted; the window t-W+1..t follows them, all larger
 #pragma unroll
-        for (int m2 = 0; m2 < 2048 / 128; ++m2) {
+        for (int m2 = 0; m2 < 1024 / 128; ++m2) {
           const int i = wt + 128 * m2;
-          int v = 0x7FFFFFFF;
-          if (i < keep) v = m2 < PER ? mine[m2 < PER ? m2 : 0] : 0x7FFFFFFF;
-          else if (i < keep + wlen) v = wlo + (i - keep);
-          ib32[i] = v;
+          ib32[i] = (i < keep && m2 < PER) ? mine[m2 < PER ? m2 : 0] : 0x7FFFFFFF;
         }
         wg_bar(wg);
-        for (int k2 = 2; k2 <= 2048; k2 <<= 1) {
+        for (int k2 = 2; k2 <= 1024; k2 <<= 1) {
           for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-            for (int pr = wt; pr < 1024; pr += 128) {
+            for (int pr = wt; pr < 512; pr += 128) {
               const int i = 2 * pr - (pr & (j2 - 1));
               const int l2 = i + j2;
               const int a = ib32[i], cv = ib32[l2];
@@ -647,7 +688,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         const int total = keep + wlen;
         int32_t* dst = p.idx + ((size_t)si.b * p.L + t) * p.S;
-        for (int i = wt; i < p.S; i += 128) dst[i] = i < total ? ib32[i] : -1;
+        for (int i = wt; i < p.S; i += 128) dst[i] = i < keep ? ib32[i] : (i < total ? wlo + (i - keep) : -1);
         wg_bar(wg);
       }
     }
@@ -668,7 +709,7 @@ static hs2_status run_t(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
                         cudaStream_t stream) {
   using FC = FaCfg<H, D>;
   using SC = ScCfg<H, D>;
-  if (topk > SC::CAP - 128) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (topk > SC::CAP - 128 || topk > 1024) return HS2_ERR_UNSUPPORTED_SHAPE;  // picks are sorted in 1024 slots
   const long long rows_total = (long long)B * L * H;
   if (rows_total >= (1LL << 31)) return HS2_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tmQ1, tmQ2, tmK, tmV;

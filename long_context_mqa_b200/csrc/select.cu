@@ -3,13 +3,17 @@
 //  1. threshold : (done by decode pass 2) from the 2048-bin histogram of score bits 30..20,
 //                 the bin beta that holds the k-th largest score; `above` = number of scores in
 //                 higher bins, `need` = k - above.
-//  2. collect   : every score in a bin above beta is selected outright; scores in bin beta
-//                 become 64-bit keys (score bits << 32 | ~index) -- unique, and larger key ==
-//                 higher score, then lower index. Extra CTAs of the same launch produce the
-//                 decode output: per (sequence, head), the sum of the per-segment output partials
-//                 of the CTAs whose tile ranges cover the sequence, rounded to bf16.
-//  3. final     : MSB-first 8-bit radix select of the `need` largest boundary keys, then the
-//                 forced window is appended and the <= 2048 indices are sorted ascending.
+//  2. collect   : every score in a bin above beta is selected outright -- its bit is set in
+//                 the sequence's selection bitmap (one bit per older token, cleared by pass 1);
+//                 scores in bin beta become 64-bit keys (score bits << 32 | ~index): unique, and
+//                 larger key == higher score, then lower index. Extra CTAs of the same launch
+//                 produce the decode output: per (sequence, head), the sum of the per-segment
+//                 output partials of the CTAs whose tile ranges cover the sequence.
+//  3. final     : MSB-first 8-bit radix select of the `need` largest boundary keys (starting at
+//                 the highest bit on which they differ, stopping as soon as the chosen bucket
+//                 holds exactly the remaining need) sets their bits; one pass over the bitmap
+//                 with a block-wide prefix sum writes the chosen indices in ascending order, and
+//                 the forced window (every index of which is larger) is appended.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -19,75 +23,44 @@ namespace sel {
 
 constexpr int NT = 1024;
 
-__device__ __forceinline__ void collect_one(const SelParams& p, int b, int* meta, int beta, int j, float score,
-                                            bool in_range, unsigned lane, unsigned lt_mask) {
-  int bin = -2;
-  uint32_t bits = 0;
-  if (in_range) {
-    bits = __float_as_uint(score);
-    bin = (int)((bits >> 20) & (NBINS - 1));
-  }
-  const bool up = bin > beta;
-  const bool eq = bin == beta;
-  const unsigned mu = __ballot_sync(0xffffffffu, up);
-  const unsigned me = __ballot_sync(0xffffffffu, eq);
-  if (mu) {
-    int base = 0;
-    const int leader = __ffs(mu) - 1;
-    if ((int)lane == leader) base = atomicAdd(&meta[3], __popc(mu));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (up) {
-      const int pos = base + __popc(mu & lt_mask);
-      if (pos < p.K) p.above[(size_t)b * p.K + pos] = j;
-      else report_status(p.st, kStatusBounds, 301);
-    }
-  }
-  if (me) {
-    int base = 0;
-    const int leader = __ffs(me) - 1;
-    if ((int)lane == leader) base = atomicAdd(&meta[4], __popc(me));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (eq) {
-      const int pos = base + __popc(me & lt_mask);
-      p.bnd[(size_t)b * p.ncand + pos] = ((unsigned long long)bits << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
-    }
-  }
-}
-
-// blockIdx.x < n_collect: every score of every older token -- above the boundary bin ->
-// selected; in it -> 64-bit key. blockIdx.x >= n_collect: output of head (blockIdx.x - n_collect).
+// blockIdx.x < n_collect: bitmap + boundary keys; blockIdx.x >= n_collect: output of head
+// (blockIdx.x - n_collect) of sequence blockIdx.y.
 __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_collect) {
   griddep_wait();
   griddep_launch_dependents();
   const int b = blockIdx.y;
   if ((int)blockIdx.x >= n_collect) {
     // CTAs c_lo..c_hi cover sequence b's tiles (contiguous split of the flattened tile space);
-    // slot = c * segmax + (b - first sequence of c)
+    // the partial of CTA c for b sits at slot c * segmax + (b - first sequence of c)
     __shared__ int slot_off[256];  // one entry per covering CTA (at most one CTA per SM)
-    __shared__ int n_slots;
+    __shared__ float part[128];
     const int h = blockIdx.x - n_collect;
-    if (threadIdx.x == 0) {
-      const long long x_lo = (long long)b * p.tps, x_hi = (long long)(b + 1) * p.tps - 1;
-      const int c_lo = (int)(((x_lo + 1) * p.G - 1) / p.total_tiles);
-      const int c_hi = (int)(((x_hi + 1) * p.G - 1) / p.total_tiles);
-      int n = 0;
-      for (int c = c_lo; c <= c_hi && n < 256; ++c, ++n) {
-        const long long ct0 = p.total_tiles * c / p.G;
-        slot_off[n] = c * p.segmax + (b - (int)(ct0 / p.tps));
-      }
-      n_slots = c_hi - c_lo + 1;
-    }
-    __syncthreads();
-    if (n_slots > 256) {  // more covering CTAs than SMs on any sm_100 part: not a valid split
+    const long long x_lo = (long long)b * p.tps, x_hi = (long long)(b + 1) * p.tps - 1;
+    const int c_lo = (int)(((x_lo + 1) * p.G - 1) / p.total_tiles);
+    const int c_hi = (int)(((x_hi + 1) * p.G - 1) / p.total_tiles);
+    const int n_slots = c_hi - c_lo + 1;
+    if (n_slots > 256 || p.D > 128) {
       if (threadIdx.x == 0) report_status(p.st, kStatusBounds, 303);
       return;
     }
-    for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
-      float acc = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < n_slots; ++i) acc += p.opart[((size_t)slot_off[i] * p.H + h) * p.D + d];
-      p.out[((size_t)b * p.H + h) * p.D + d] = __float2bfloat16_rn(acc);
+    for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
+      const int c = c_lo + i;
+      const long long ct0 = p.total_tiles * c / p.G;
+      slot_off[i] = c * p.segmax + (b - (int)(ct0 / p.tps));
     }
+    __syncthreads();
+    // two threads per output column, each summing half of the slots
+    const int d = threadIdx.x % 128, half = threadIdx.x / 128;
+    const int nh = (n_slots + 1) / 2;
+    const int s_lo = half ? nh : 0, s_hi = half ? n_slots : nh;
+    float acc = 0.f;
+    if (d < p.D) {
+#pragma unroll 8
+      for (int i = s_lo; i < s_hi; ++i) acc += p.opart[((size_t)slot_off[i] * p.H + h) * p.D + d];
+    }
+    if (half) part[d] = acc;
+    __syncthreads();
+    if (!half && d < p.D) p.out[((size_t)b * p.H + h) * p.D + d] = __float2bfloat16_rn(acc + part[d]);
     return;
   }
   int* meta = p.meta + b * META;
@@ -95,10 +68,11 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
   const unsigned lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   const float* sc = p.sc + (size_t)b * p.ncand;
+  unsigned* bm = p.bitmap + (size_t)b * p.words;
   const int stride = n_collect * 256 * 4;
   const int n_round = ((p.ncand + 127) / 128) * 128;
-  // four consecutive scores per thread per step (16-byte loads when the row is aligned)
   const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
+  // four consecutive scores per thread per step: one bitmap word, one 16-byte load
   for (int j0 = (blockIdx.x * 256 + threadIdx.x) * 4; j0 < n_round; j0 += stride) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (vec && j0 + 3 < p.ncand) {
@@ -108,32 +82,47 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
       for (int x = 0; x < 4; ++x)
         if (j0 + x < p.ncand) v[x] = sc[j0 + x];
     }
+    unsigned upmask = 0;
 #pragma unroll
-    for (int x = 0; x < 4; ++x) collect_one(p, b, meta, beta, j0 + x, v[x], j0 + x < p.ncand, lane, lt_mask);
+    for (int x = 0; x < 4; ++x) {
+      const int j = j0 + x;
+      const bool in_range = j < p.ncand;
+      const uint32_t bits = __float_as_uint(v[x]);
+      const int bin = in_range ? (int)((bits >> 20) & (NBINS - 1)) : -2;
+      if (in_range && bin > beta) upmask |= 1u << (j & 31);
+      const bool eq = in_range && bin == beta;
+      const unsigned me = __ballot_sync(0xffffffffu, eq);
+      if (me) {
+        int base = 0;
+        const int leader = __ffs(me) - 1;
+        if ((int)lane == leader) base = atomicAdd(&meta[4], __popc(me));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (eq) {
+          const int pos = base + __popc(me & lt_mask);
+          p.bnd[(size_t)b * p.ncand + pos] =
+              ((unsigned long long)bits << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
+        }
+      }
+    }
+    if (upmask) atomicOr(&bm[j0 >> 5], upmask);
   }
 }
 
 __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   griddep_wait();
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  __shared__ int list[2048];
   __shared__ unsigned dh[256];
-  __shared__ unsigned long long s_prefix, s_mask;
-  __shared__ int s_need, s_cnt;
+  __shared__ unsigned long long s_prefix, s_mask, s_and, s_or;
+  __shared__ int s_need, s_exact;
+  __shared__ unsigned wsum[32];
   const int* meta = p.meta + b * META;
-  const int n_above = meta[1];
   const int need = meta[2];
   const int n_bnd = meta[4];
   const unsigned long long* bnd = p.bnd + (size_t)b * p.ncand;
-  for (int i = tid; i < 2048; i += NT) list[i] = 0x7FFFFFFF;
-  __syncthreads();
-  for (int i = tid; i < n_above && i < p.K; i += NT) list[i] = p.above[(size_t)b * p.K + i];
-  if (tid == 0) { s_prefix = 0; s_mask = 0; s_need = need; s_cnt = 0; }
-  __syncthreads();
-  if (need > 0) {
+  unsigned* bm = p.bitmap + (size_t)b * p.words;
+  if (need > 0 && n_bnd > 0) {
     // bits on which every boundary key agrees need no pass: start at the highest differing bit
-    __shared__ unsigned long long s_and, s_or;
-    if (tid == 0) { s_and = ~0ull; s_or = 0ull; }
+    if (tid == 0) { s_and = ~0ull; s_or = 0ull; s_need = need; s_exact = 0; }
     __syncthreads();
     unsigned long long a_loc = ~0ull, o_loc = 0ull;
     for (int i = tid; i < n_bnd; i += NT) { const unsigned long long key = bnd[i]; a_loc &= key; o_loc |= key; }
@@ -144,11 +133,14 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
     if (lane == 0) { atomicAnd(&s_and, a_loc); atomicOr(&s_or, o_loc); }
     __syncthreads();
     const unsigned long long diff = s_and ^ s_or;
-    const int top = diff ? 63 - __clzll((long long)diff) : 0;  // highest differing bit
-    if (tid == 0) { s_prefix = s_and & ~((top >= 63) ? 0ull : ((2ull << top) - 1ull)); s_mask = (top >= 63) ? 0ull : ~((2ull << top) - 1ull); }
+    const int top = diff ? 63 - __clzll((long long)diff) : 0;
+    if (tid == 0) {
+      s_mask = top >= 63 ? 0ull : ~((2ull << top) - 1ull);
+      s_prefix = s_and & s_mask;
+    }
     __syncthreads();
-    // 8-bit digit windows [shift, shift + 8) from the top down; the last window is clamped at
-    // bit 0 (its bits above the previous window's are already fixed in the prefix)
+    // 8-bit digit windows from the top down; the last is clamped at bit 0 (its bits above the
+    // previous window are already fixed in the prefix)
     for (int sh_raw = top - 7;; sh_raw -= 8) {
       const int shift = sh_raw < 0 ? 0 : sh_raw;
       for (int i = tid; i < 256; i += NT) dh[i] = 0;
@@ -176,10 +168,10 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
           unsigned run = excl;
           for (int x = 0; x < 8; ++x) {
             if (run + cnt[x] >= k) {
-              const unsigned digit = 255u - 8u * lane - x;
               s_need = (int)(k - run);
-              s_prefix = prefix | ((unsigned long long)digit << shift);
+              s_prefix = prefix | ((unsigned long long)(255u - 8u * lane - x) << shift);
               s_mask = mask | (255ull << shift);
+              s_exact = run + cnt[x] == k;  // the whole bucket is taken: no further digit needed
               break;
             }
             run += cnt[x];
@@ -187,39 +179,61 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
         }
       }
       __syncthreads();
-      if (shift == 0) break;
+      if (shift == 0 || s_exact) break;
     }
-    // s_prefix is now the exact key of the need-th largest boundary entry
-    const unsigned long long thr = s_prefix;
+    // keys whose masked prefix is >= s_prefix are exactly the `need` largest boundary entries
+    const unsigned long long thr = s_prefix, fmask = s_mask;
     for (int i = tid; i < n_bnd; i += NT) {
       const unsigned long long key = bnd[i];
-      if (key >= thr) {
-        const int pos = atomicAdd(&s_cnt, 1);
-        if (n_above + pos < 2048) list[n_above + pos] = (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+      if ((key & fmask) >= thr) {
+        const uint32_t j = 0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull);
+        atomicOr(&bm[j >> 5], 1u << (j & 31));
       }
     }
-    __syncthreads();
   }
-  const int n_top = n_above + (need > 0 ? s_cnt : 0);
-  const int wlen = p.N < p.W ? p.N : p.W;
-  for (int i = tid; i < wlen; i += NT)
-    if (n_top + i < 2048) list[n_top + i] = p.N - wlen + i;
-  const int total = n_top + wlen;
-  const int expect = p.N < p.S ? p.N : p.S;
-  if (tid == 0 && total != expect) report_status(p.st, kStatusBounds, 302);
   __syncthreads();
-  // bitonic sort, ascending, 2048 slots
-  for (int k = 2; k <= 2048; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      const int i = 2 * tid - (tid & (j - 1));
-      const int l = i + j;
-      const int a = list[i], c = list[l];
-      const bool asc = (i & k) == 0;
-      if ((a > c) == asc) { list[i] = c; list[l] = a; }
-      __syncthreads();
+  // the bitmap in order: each thread owns a contiguous run of words; block-wide exclusive scan
+  const int per = (p.words + NT - 1) / NT;
+  const int w0 = tid * per, w1 = w0 + per < p.words ? w0 + per : p.words;
+  unsigned cnt = 0;
+  for (int i = w0; i < w1; ++i) cnt += __popc(__ldcg(&bm[i]));
+  unsigned incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    unsigned t = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    wsum[lane] = t;  // inclusive over warps
+  }
+  __syncthreads();
+  const unsigned total_top = wsum[31];
+  unsigned pos = incl - cnt + (w > 0 ? wsum[w - 1] : 0u);
+  int32_t* out = p.idx + (size_t)b * p.S;
+  for (int i = w0; i < w1; ++i) {
+    unsigned word = __ldcg(&bm[i]);
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (pos < (unsigned)p.S) out[pos] = i * 32 + bit;
+      ++pos;
     }
   }
-  for (int i = tid; i < p.S; i += NT) p.idx[(size_t)b * p.S + i] = (i < total && i < 2048) ? list[i] : -1;
+  const int wlen = p.N < p.W ? p.N : p.W;
+  const int expect_top = p.ncand < p.K ? p.ncand : p.K;
+  if (tid == 0 && (int)total_top != expect_top) report_status(p.st, kStatusBounds, 302);
+  for (int i = tid; i < p.S; i += NT) {
+    if (i >= (int)total_top && i < (int)total_top + wlen) out[i] = p.N - wlen + (i - (int)total_top);
+    else if (i >= (int)total_top + wlen) out[i] = -1;
+  }
 }
 
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream) {
