@@ -67,7 +67,8 @@ def _traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
+    """nvidia-smi clocks / throttle reasons, sampled every 50 ms by a reader thread; summary()
+    keeps the samples taken between start_region() and end_region()."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -76,30 +77,56 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.out = None
+        self.rows = []          # (monotonic time, csv line)
+        self.t_start = None
+        self.t_end = None
+        self._first = threading.Event()
+        self._thread = None
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.monotonic(), line))
+            self._first.set()
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._thread = threading.Thread(target=self._reader, daemon=True)
+            self._thread.start()
+            self._first.wait(timeout=5.0)   # sampling is running before the timed region opens
         except Exception:
             self.proc = None
         return self
+
+    def start_region(self):
+        self.t_start = time.monotonic()
+
+    def end_region(self):
+        self.t_end = time.monotonic()
+        # one more sample after the region, so a region shorter than the interval still has one
+        n = len(self.rows)
+        t0 = time.monotonic()
+        while self.proc is not None and len(self.rows) == n and time.monotonic() - t0 < 0.5:
+            time.sleep(0.01)
 
     def __exit__(self, *a):
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                self.out = ""
+            if self._thread is not None:
+                self._thread.join(timeout=2)
 
     def summary(self):
-        if not self.out:
+        lines = [ln for (t, ln) in self.rows
+                 if self.t_start is None or (t >= self.t_start and (self.t_end is None or t <= self.t_end + 0.06))]
+        if not lines:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        rows = [r for r in csv.reader(io.StringIO(self.out)) if len(r) >= 9]
+        rows = [r for r in csv.reader(io.StringIO("".join(lines))) if len(r) >= 9]
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -312,19 +339,21 @@ def run_gpu(args):
         for _ in range(args.warmup):
             step()
         _barrier(world)
-        hs2.profile_enable("dec_pass2")
+        hs2.profile_enable("dec_fused")
         launches0 = hs2.kernel_launches()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks.start_region()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         e1.synchronize()
+        clocks.end_region()
         launches = hs2.kernel_launches() - launches0
         hs2.profile_enable(None)
         _barrier(world)
     ms_total = _max_over_ranks(e0.elapsed_time(e1), world)
-    pass2_ms, pass2_n = hs2.profile_read("dec_pass2")
+    dec_ms, dec_n = hs2.profile_read("dec_fused")
     # per-kernel breakdown (separate short run with every launch timed by CUDA events)
     hs2.profile_enable("*")
     n_brk = min(args.steps, 50)
@@ -333,7 +362,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     hs2.profile_enable(None)
     breakdown = {}
-    for name in ("dec_pass1", "dec_pass2", "sel_collect", "sel_final", "sparse_attn"):
+    for name in ("dec_fused", "sel_collect", "sel_final", "sparse_attn"):
         kms, kn = hs2.profile_read(name)
         if kn:
             breakdown[name] = kms / n_brk
@@ -342,16 +371,16 @@ def run_gpu(args):
     ms_per_step = ms_total / args.steps
     value = world * args.steps / (ms_total / 1e3)
 
-    # ---------------- roofline of the dominant kernel (decode pass 2)
+    # ---------------- roofline of the dominant kernel (the fused decode kernel)
     ncand = wl.Lk - wl.window
-    pass2_bytes = wl.B * wl.Lk * wl.d * 2 * 2 + wl.B * ncand * 4   # K + V once, scores written
-    pass2_avg_s = pass2_ms / max(pass2_n, 1) / 1e3
-    pass2_gbs = pass2_bytes / pass2_avg_s / 1e9
-    traffic = _traffic("dec_pass2")
-    roofline = {"kernel": "dec_pass2", "bound": "hbm", "achieved": pass2_gbs, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": pass2_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": peaks["source"], "algorithmic_bytes_per_launch": pass2_bytes,
-                "avg_launch_ms": pass2_avg_s * 1e3}
+    dec_bytes = wl.B * wl.Lk * wl.d * 2 * 2 + wl.B * ncand * 4   # K + V once from HBM, scores written
+    dec_avg_s = dec_ms / max(dec_n, 1) / 1e3
+    dec_gbs = dec_bytes / dec_avg_s / 1e9
+    traffic = _traffic("dec_fused")
+    roofline = {"kernel": "dec_fused", "bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": peaks["source"], "algorithmic_bytes_per_launch": dec_bytes,
+                "avg_launch_ms": dec_avg_s * 1e3}
     step_bytes = (wl.B * wl.Lk * wl.d * 4 + (1 + wl.n_sparse) * wl.B * wl.H * wl.d * 4
                   + wl.n_sparse * wl.B * S * wl.d * 4 + wl.B * S * 4)
     step_roof = {"bound": "hbm", "algorithmic_bytes": step_bytes,

@@ -119,10 +119,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!wait_abortable(&full[s], (it / STAGES) & 1, limit, &abort_flag, p.st, 512)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES), sb = sa + A_BYTES;
+          const uint64_t da = sdesc(sa, 16, 1024), db = sdesc(sb, BK * 128, 1024);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t a = sdesc(sa + kk * 32, 16, 1024);
-            const uint64_t b = sdesc(sb + kk * 2048, BK * 128, 1024);
+            const uint64_t a = sdesc_at(da, kk * 32);
+            const uint64_t b = sdesc_at(db, kk * 2048);
             umma_bf16(tmem + ab * BN, a, b, IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);

@@ -1,36 +1,36 @@
 // Decode step of the full-attention + selection layer (one query token per sequence, the
-// query at position t = N-1 of an N-token K/V cache).
+// query at position t = N-1 of an N-token K/V cache), as one persistent kernel.
 //
 // Exact head-summed probabilities need each head's logsumexp over the whole row before any
-// token's score is final, so the cache is scanned twice:
+// token's score is final, so every tile of the cache is visited twice. The sequences are taken
+// in groups (Sched; by default one group holding all of them); per group:
 //
-//   pass 1  K only.  S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads).
-//           Two softmax warpgroups split the heads (32 each); every thread owns one key lane
-//           and keeps, per head, a reference r and a sum l of exp2(s*c - r). r is only moved
-//           (with the usual rescale of l) when a value exceeds it by more than 2^64, so the
-//           common step is one FFMA, one MUFU ex2, one FADD and one FMNMX per element. One
-//           cross-lane merge per work segment -> partial (m, l) per head. CTA 0 also clears the
-//           selection histogram for pass 2.
-//   pass 2  K and V.  Prologue: the segment's per-head lse from all pass-1 partials of that
-//           sequence (the CTA owning the sequence's first tile also writes the caller's lse).
-//           S^T again; p = exp2(s*c - lse2) exactly (no rescaling); the head sum is an in-thread
-//           reduction (the score of the thread's key); P^T (bf16) goes to shared memory as an
-//           MN-major operand and O^T += V^T P^T accumulates in TMEM. Two softmax warpgroups take
-//           alternate tiles. Scores of older tokens go to a global buffer and a 2048-bin
-//           histogram of their top bits (warp-aggregated shared atomics).
-//           The last CTA to finish a sequence scans that sequence's histogram for the bin of
-//           its k-th largest score.
-//   finish  (select.cu) sum of the output partials -> bf16 out; collect / final selection.
+//   phase 1  K only.  S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads).
+//            The two softmax warpgroups split the heads (32 each); every thread owns one key
+//            lane and keeps, per head, a reference r and a sum l of exp2(s*c - r). r only moves
+//            (with the usual rescale of l) when a value exceeds it by more than 2^64, so the
+//            common step is one FFMA, one MUFU ex2, one FADD and one FMNMX per element. One
+//            cross-lane merge per segment -> partial (m, l) per head.
+//   grid barrier (bounded): every phase-1 partial of the group is written.
+//   phase 2  K again (now from L2) and V. The segment's per-head lse from all partials of its
+//            sequence (the CTA owning the sequence's first tile also writes the caller's lse);
+//            S^T again; p = exp2(s*c - lse2) exactly (no rescaling); the head sum is an
+//            in-thread reduction (the score of the thread's key); P^T (bf16) goes to shared
+//            memory as an MN-major operand and O^T += V^T P^T accumulates in TMEM. The two
+//            warpgroups take alternate tiles. Scores of the older tokens go to a global buffer
+//            and a 2048-bin histogram of their top bits (warp-aggregated shared atomics); the
+//            last CTA to finish a sequence scans its histogram for the bin of the k-th score.
 //
-// Work split: the flattened (sequence, 128-key tile) space is cut into G contiguous ranges,
-// one per CTA (G = number of SMs); a range may cross a sequence boundary, so a CTA handles
-// one or more "segments", each producing one partial record. Pass 2 walks its range in
-// reverse order so the keys pass 1 touched last are re-read first (L2 hits).
+// Phase 2 walks a CTA's range backwards, so the K tiles phase 1 loaded last are re-read first
+// (those still in L2; a group small enough for L2 would re-read all of its K from there).
+// The grid is one CTA per SM, launched cooperatively (all CTAs co-resident). select.cu finishes
+// the step: output combine, collect, final selection.
 //
-// Warp roles: warp 0 = K (and Q) TMA producer, warp 1 = tcgen05 issuer and TMEM owner,
-// warp 2 = V producer (pass 2), warps 4..7 and 8..11 = the two softmax warpgroups (warp w
-// reads TMEM lanes 32*(w%4)..+31). Every wait is bounded; on timeout the kernel records it
-// in the status word and unwinds.
+// Warp roles (320 threads): warp 0 = TMA producer (Q per segment; K and V tiles through one
+// 5-slot ring, in the order the tensor core consumes them), warp 1 = tcgen05 issuer and TMEM
+// owner, warps 2..5 and 6..9 = softmax warpgroups 0 and 1 (warp w reads TMEM lanes
+// 32*(w%4)..+31). Every wait is bounded; on timeout the kernel records it in the status word
+// and unwinds with its barrier sequence intact.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -39,18 +39,12 @@ namespace hs2 {
 namespace dec {
 
 constexpr int TILE = 128;
-constexpr int NTHREADS = 384;
-constexpr int SM_WG0 = 4;     // first warp of softmax warpgroup 0
+constexpr int NTHREADS = 320;
+constexpr int SM_WG0 = 2;  // first warp of softmax warpgroup 0
+constexpr int RING = 5;    // K/V tile slots
+constexpr int NBINS = 2048;
 constexpr float REF_SLACK = 64.f;
 
-__device__ __forceinline__ void tile_range(const DecParams& p, int cta, long long& t0, long long& t1) {
-  t0 = p.total_tiles * cta / p.G;
-  t1 = p.total_tiles * (cta + 1) / p.G;
-}
-// CTA whose range holds flattened tile x
-__device__ __forceinline__ int cta_of_tile(const DecParams& p, long long x) {
-  return (int)(((x + 1) * p.G - 1) / p.total_tiles);
-}
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // bounded wait that also gives up when another role already aborted
@@ -78,261 +72,55 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, lo
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
 }
-
-// ------------------------------------------------------------------------------------------
-// pass 1: per-head (reference, sum) partials of exp2(s * c)
-// ------------------------------------------------------------------------------------------
-template <int H, int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    dec_pass1_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, DecParams p) {
-  constexpr int KST = 5;
-  constexpr int KT_BYTES = TILE * D * 2;
-  constexpr int Q_BYTES = H * D * 2;
-  constexpr int NKB = D / 64;
-  constexpr int HW = H / 2;  // heads per warpgroup
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                // 2 buffers
-  uint8_t* sK = smem + 2 * Q_BYTES;  // KST stages
-  __shared__ __align__(8) uint64_t k_full[KST], k_empty[KST], s_full[2], s_empty[2], q_full[2], q_empty[2];
-  __shared__ uint32_t tmem_base;
-  __shared__ volatile int abort_flag;
-  __shared__ float red[2][4][HW][2];
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x;
-  long long t0, t1;
-  tile_range(p, cta, t0, t1);
-  const long long limit = p.wait_ns;
-
-  if (cta == 0) {  // pass 2 accumulates into the selection histogram and per-sequence counters
-    for (int i = threadIdx.x; i < p.B * 2048; i += NTHREADS) p.hist[i] = 0u;
-    for (int i = threadIdx.x; i < p.B; i += NTHREADS) p.seq_done[i] = 0;
-  }
-  {  // the selection bitmap, cleared by all CTAs (the collect kernel sets bits)
-    const long long total = (long long)p.B * p.words;
-    const long long per = (total + p.G - 1) / p.G;
-    const long long w0 = per * cta, w1 = w0 + per < total ? w0 + per : total;
-    for (long long i = w0 + threadIdx.x; i < w1; i += NTHREADS) p.bitmap[i] = 0u;
-  }
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8);
-      mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
-    }
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-  griddep_launch_dependents();  // pass 2 may start streaming K/V into freed SMs
-
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmQ);
-      const uint64_t pol = policy_evict_last();  // pass 2 re-reads K: keep it in L2 if possible
-      uint32_t j = 0;
-      int seg = 0;
-      bool ok = true;
-      for (long long t = t0; t < t1 && ok; ++seg) {
-        const int b = (int)(t / p.tps);
-        const long long seg_end = t1 < (long long)(b + 1) * p.tps ? t1 : (long long)(b + 1) * p.tps;
-        const int qb = seg & 1;
-        if (!wait_bar(&q_empty[qb], ((seg >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 101)) { ok = false; break; }
-        mbar_expect_tx(&q_full[qb], Q_BYTES);
-        for (int kb = 0; kb < NKB; ++kb) tma_load_3d(sQ + qb * Q_BYTES + kb * (H * 128), &tmQ, &q_full[qb], kb * 64, 0, b);
-        for (; t < seg_end; ++t, ++j) {
-          const int lt = (int)(t - (long long)b * p.tps);
-          const int s = j % KST;
-          if (!wait_bar(&k_empty[s], ((j / KST) & 1) ^ 1, limit, &abort_flag, p.st, 102)) { ok = false; break; }
-          mbar_expect_tx(&k_full[s], KT_BYTES);
-          for (int kb = 0; kb < NKB; ++kb)
-            tma_load_3d_hint(sK + s * KT_BYTES + kb * (TILE * 128), &tmK, &k_full[s], kb * 64, lt * TILE, b, pol);
-        }
-      }
-      if (!ok)  // let the copies already issued land before the CTA exits
-        for (uint32_t jj = (j > KST ? j - KST : 0); jj < j; ++jj) mbar_wait(&k_full[jj % KST], (jj / KST) & 1, limit);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(128, H, 0, 0);
-      uint32_t j = 0;
-      int seg = 0;
-      bool ok = true;
-      for (long long t = t0; t < t1 && ok; ++seg) {
-        const int b = (int)(t / p.tps);
-        const long long seg_end = t1 < (long long)(b + 1) * p.tps ? t1 : (long long)(b + 1) * p.tps;
-        const int qb = seg & 1;
-        if (!wait_bar(&q_full[qb], (seg >> 1) & 1, limit, &abort_flag, p.st, 111)) { ok = false; break; }
-        const uint32_t qaddr = smem_u32(sQ + qb * Q_BYTES);
-        for (; t < seg_end; ++t, ++j) {
-          const int s = j % KST, buf = j & 1;
-          if (!wait_bar(&k_full[s], (j / KST) & 1, limit, &abort_flag, p.st, 112)) { ok = false; break; }
-          if (!wait_bar(&s_empty[buf], ((j >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 113)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kaddr = smem_u32(sK + s * KT_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = sdesc(kaddr + (kk / 4) * (TILE * 128) + (kk % 4) * 32, 16, 1024);
-            const uint64_t bq = sdesc(qaddr + (kk / 4) * (H * 128) + (kk % 4) * 32, 16, 1024);
-            umma_bf16(tmem + buf * H, a, bq, IDESC, kk > 0);
-          }
-          umma_commit(&s_full[buf]);
-          umma_commit(&k_empty[s]);
-        }
-        umma_commit(&q_empty[qb]);
-      }
-    }
-  } else if (warp >= SM_WG0) {
-    const int wg = (warp - SM_WG0) / 4;  // heads [wg*HW, wg*HW + HW)
-    const int wq = (warp - SM_WG0) % 4;
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const int wg_tid = wq * 32 + lane;
-    const float c = p.c;
-    uint32_t j = 0;
-    for (long long t = t0; t < t1;) {
-      const int b = (int)(t / p.tps);
-      const long long seg_end = t1 < (long long)(b + 1) * p.tps ? t1 : (long long)(b + 1) * p.tps;
-      const int slot = cta * p.segmax + (b - (int)(t0 / p.tps));
-      const long long seg_first = t;
-      float r[HW], l[HW];
-#pragma unroll
-      for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
-      // after a failed wait every later wait returns at once: keep the loop and barrier
-      // structure identical across warps, skip only the work
-      bool ok = !abort_flag;
-      for (; t < seg_end; ++t, ++j) {
-        const int lt = (int)(t - (long long)b * p.tps);
-        const int buf = j & 1;
-        if (!ok) continue;
-        if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 121)) { ok = false; continue; }
-        tc_fence_after();
-        float v[HW];
-        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + buf * H + wg * HW, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[buf]);
-        const bool valid = lt * TILE + row < p.N;
-        if (t == seg_first) {
-          // a lane's first key of the segment sets its references (invalid lanes only occur in
-          // a sequence's partial last tile, which is then the segment's only tile)
-#pragma unroll
-          for (int h = 0; h < HW; ++h) {
-            r[h] = valid ? v[h] * c : -INFINITY;
-            l[h] = valid ? 1.f : 0.f;
-          }
-          continue;
-        }
-        float dmax = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < HW; ++h) {
-          v[h] = valid ? fmaf(v[h], c, -r[h]) : -INFINITY;  // exponent relative to the reference
-          dmax = fmaxf(dmax, v[h]);
-        }
-        if (__any_sync(0xffffffffu, dmax > REF_SLACK)) {
-          // rare: move the reference of the heads that outgrew it (always on a lane's first key)
-#pragma unroll
-          for (int h = 0; h < HW; ++h) {
-            const float d = v[h];
-            if (d > REF_SLACK) {
-              l[h] = l[h] * fast_exp2(-d) + 1.f;
-              r[h] = r[h] + d;
-            } else {
-              l[h] += fast_exp2(d);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < HW; ++h) l[h] += fast_exp2(v[h]);
-        }
-      }
-      // merge the 128 lanes: warp shuffle, then the 4 warps through shared memory
-#pragma unroll
-      for (int h = 0; h < HW; ++h) {
-        float mm = r[h], ll = l[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, mm, off);
-          const float l2 = __shfl_xor_sync(0xffffffffu, ll, off);
-          const float mx = fmaxf(mm, m2);
-          const float a1 = mm == -INFINITY ? 0.f : fast_exp2(mm - mx);
-          const float a2 = m2 == -INFINITY ? 0.f : fast_exp2(m2 - mx);
-          ll = ll * a1 + l2 * a2;
-          mm = mx;
-        }
-        if (lane == 0) { red[wg][wq][h][0] = mm; red[wg][wq][h][1] = ll; }
-      }
-      named_bar(1 + wg, 128);
-      if (wg_tid < HW) {
-        float mm = red[wg][0][wg_tid][0], ll = red[wg][0][wg_tid][1];
-        for (int w = 1; w < 4; ++w) {
-          const float m2 = red[wg][w][wg_tid][0], l2 = red[wg][w][wg_tid][1];
-          const float mx = fmaxf(mm, m2);
-          const float a1 = mm == -INFINITY ? 0.f : fast_exp2(mm - mx);
-          const float a2 = m2 == -INFINITY ? 0.f : fast_exp2(m2 - mx);
-          ll = ll * a1 + l2 * a2;
-          mm = mx;
-        }
-        p.ml[(size_t)slot * 2 * H + wg * HW + wg_tid] = mm;
-        p.ml[(size_t)slot * 2 * H + H + wg * HW + wg_tid] = ll;
-      }
-      named_bar(1 + wg, 128);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 128); }
+// (m, l) <- merge of two (max, sum of exp2(x - max)) pairs
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+  const float mx = fmaxf(m, m2);
+  const float a1 = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+  const float a2 = m2 == -INFINITY ? 0.f : fast_exp2(m2 - mx);
+  l = l * a1 + l2 * a2;
+  m = mx;
 }
 
-// ------------------------------------------------------------------------------------------
-// pass 2: exact probabilities, output partials, head-summed scores, histogram
-// ------------------------------------------------------------------------------------------
 template <int H, int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    dec_pass2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    dec_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, DecParams p) {
-  static_assert(H == 64 && D == 128, "decode pass 2 is instantiated for 64 heads x 128");
-  constexpr int KST = 2, VST = 3;
+  static_assert(H == 64 && D == 128, "the decode kernel is instantiated for 64 heads x 128");
   constexpr int KT_BYTES = TILE * D * 2;
   constexpr int Q_BYTES = H * D * 2;
   constexpr int P_BYTES = TILE * H * 2;
   constexpr int NKB = D / 64;
-  constexpr int NBINS = 2048;
+  constexpr int HW = H / 2;  // heads per warpgroup in phase 1
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                           // 1 x Q
-  uint8_t* sK = sQ + Q_BYTES;                   // KST x K tile
-  uint8_t* sV = sK + KST * KT_BYTES;            // VST x V tile
-  uint8_t* sP = sV + VST * KT_BYTES;            // 2 x P^T
+  uint8_t* sQ = smem;                  // Q of the current segment
+  uint8_t* sR = sQ + Q_BYTES;          // RING tiles (K or V)
+  uint8_t* sP = sR + RING * KT_BYTES;  // P^T of warpgroup 0 / 1
   uint32_t* shist = (uint32_t*)(sP + 2 * P_BYTES);
-  __shared__ __align__(8) uint64_t k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], s_empty[2],
-      p_full[2], p_empty[2], q_full, q_empty, o_full, o_empty;
+  __shared__ __align__(8) uint64_t r_full[RING], r_empty[RING], s_full[2], s_empty[2], p_full[2], p_empty[2], q_full,
+      q_empty, o_full, o_empty;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ __align__(16) float slse[H];
+  __shared__ __align__(16) float red[8][H][2];  // merge scratch (phase-1 view: [2][4][HW][2])
   __shared__ int s_last;
   __shared__ unsigned s_wtot[8];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  long long t0, t1;
-  tile_range(p, cta, t0, t1);
+  const Sched S = p.sch;
   const long long limit = p.wait_ns;
-  const uint32_t tS = 0, tO = 2 * H;  // TMEM column offsets
+  // TMEM columns. Every product is split over two accumulators (even / odd 16-wide k-steps)
+  // so that consecutive MMAs do not wait on one another: S buffer b half x at (2b + x) * H,
+  // O^T half x at 4H + x * H. Readers add the two halves.
+  const uint32_t tS = 0, tO = 4 * H;
 
   for (int i = threadIdx.x; i < NBINS; i += NTHREADS) shist[i] = 0;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-    for (int i = 0; i < VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    for (int i = 0; i < RING; ++i) { mbar_init(&r_full[i], 1); mbar_init(&r_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
+      // phase 1: all 8 softmax warps release an S buffer; phase 2: the 4 warps of its owner, x2
+      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8);
       mbar_init(&p_full[i], 4); mbar_init(&p_empty[i], 1);
     }
     mbar_init(&q_full, 1); mbar_init(&q_empty, 1);
@@ -340,291 +128,455 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   griddep_launch_dependents();
-  // Launched early (programmatic dependent launch): the producers and the tensor core only read
-  // K, V and Q, so they start at once; the softmax warps wait for pass 1 to complete before they
-  // read its partials or touch the histogram / counters it cleared.
 
-  // segments are walked from the end of the range backwards, tiles likewise
   if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmQ);
-      const uint64_t pol = policy_evict_first();
-      uint32_t j = 0;
-      int seg = 0;
+      tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV); tma_prefetch_desc(&tmQ);
+      const uint64_t keep = policy_evict_last(), once = policy_evict_first();
+      uint32_t ri = 0, nq = 0;
       bool ok = true;
-      for (long long t = t1 - 1; t >= t0 && ok; ++seg) {
-        const int b = (int)(t / p.tps);
-        const long long seg_lo = t0 > (long long)b * p.tps ? t0 : (long long)b * p.tps;
-        if (!wait_bar(&q_empty, (seg & 1) ^ 1, limit, &abort_flag, p.st, 201)) { ok = false; break; }
+      auto load_q = [&](int b) -> bool {
+        if (!wait_bar(&q_empty, (nq & 1) ^ 1, limit, &abort_flag, p.st, 201)) return false;
         mbar_expect_tx(&q_full, Q_BYTES);
         for (int kb = 0; kb < NKB; ++kb) tma_load_3d(sQ + kb * (H * 128), &tmQ, &q_full, kb * 64, 0, b);
-        for (; t >= seg_lo; --t, ++j) {
-          const int lt = (int)(t - (long long)b * p.tps);
-          const int s = j % KST;
-          if (!wait_bar(&k_empty[s], ((j / KST) & 1) ^ 1, limit, &abort_flag, p.st, 202)) { ok = false; break; }
-          mbar_expect_tx(&k_full[s], KT_BYTES);
-          for (int kb = 0; kb < NKB; ++kb)
-            tma_load_3d_hint(sK + s * KT_BYTES + kb * (TILE * 128), &tmK, &k_full[s], kb * 64, lt * TILE, b, pol);
+        ++nq;
+        return true;
+      };
+      auto load_tile = [&](const CUtensorMap* m, int lt, int b, uint64_t pol) -> bool {
+        const int s = ri % RING;
+        if (!wait_bar(&r_empty[s], ((ri / RING) & 1) ^ 1, limit, &abort_flag, p.st, 202)) return false;
+        mbar_expect_tx(&r_full[s], KT_BYTES);
+        for (int kb = 0; kb < NKB; ++kb)
+          tma_load_3d_hint(sR + s * KT_BYTES + kb * (TILE * 128), m, &r_full[s], kb * 64, lt * TILE, b, pol);
+        ++ri;
+        return true;
+      };
+      for (int g = 0; g < S.n_groups && ok; ++g) {
+        long long t0, t1;
+        S.range(g, cta, t0, t1);
+        for (long long t = t0; t < t1 && ok;) {  // phase 1: K, ascending
+          const int b = (int)(t / S.tps);
+          const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          if (!load_q(b)) { ok = false; break; }
+          for (; t < seg_end; ++t)
+            if (!load_tile(&tmK, (int)(t - (long long)b * S.tps), b, keep)) { ok = false; break; }
+        }
+        for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: descending
+          const int b = (int)(t / S.tps);
+          const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          if (!load_q(b)) { ok = false; break; }
+          // in the order the tensor core consumes them: S of a tile needs its K, then the PV of
+          // the tile before it (the next higher one) needs that tile's V
+          const long long seg_hi = t;
+          for (; t >= seg_lo; --t) {
+            const int lt = (int)(t - (long long)b * S.tps);
+            if (!load_tile(&tmK, lt, b, once)) { ok = false; break; }
+            if (t < seg_hi && !load_tile(&tmV, lt + 1, b, once)) { ok = false; break; }
+          }
+          if (ok && !load_tile(&tmV, (int)(seg_lo - (long long)b * S.tps), b, once)) { ok = false; break; }
         }
       }
-      if (!ok)
-        for (uint32_t jj = (j > KST ? j - KST : 0); jj < j; ++jj) mbar_wait(&k_full[jj % KST], (jj / KST) & 1, limit);
-    }
-  } else if (warp == 2) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmV);
-      const uint64_t pol = policy_evict_first();
-      uint32_t j = 0;
-      bool ok = true;
-      for (long long t = t1 - 1; t >= t0 && ok; --t, ++j) {
-        const int b = (int)(t / p.tps);
-        const int lt = (int)(t - (long long)b * p.tps);
-        const int s = j % VST;
-        if (!wait_bar(&v_empty[s], ((j / VST) & 1) ^ 1, limit, &abort_flag, p.st, 203)) { ok = false; break; }
-        mbar_expect_tx(&v_full[s], KT_BYTES);
-        for (int kb = 0; kb < NKB; ++kb)
-          tma_load_3d_hint(sV + s * KT_BYTES + kb * (TILE * 128), &tmV, &v_full[s], kb * 64, lt * TILE, b, pol);
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        for (uint32_t x = (ri > RING ? ri - RING : 0); x < ri; ++x) mbar_wait(&r_full[x % RING], (x / RING) & 1, limit);
+        if (nq > 0) mbar_wait(&q_full, (nq - 1) & 1, limit);
       }
-      if (!ok)
-        for (uint32_t jj = (j > VST ? j - VST : 0); jj < j; ++jj) mbar_wait(&v_full[jj % VST], (jj / VST) & 1, limit);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, H, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16(D, H, 1, 1);
-      uint32_t j = 0;
-      int seg = 0;
+      uint32_t ri = 0, j = 0, nq = 0, seg2 = 0;
+      uint32_t npu[2] = {0, 0};  // PV uses of each P buffer
       bool ok = true;
-      auto issue_pv = [&](uint32_t jj, bool first, int segi) -> bool {
-        const int buf = jj & 1, s = jj % VST;
-        if (!wait_bar(&p_full[buf], (jj >> 1) & 1, limit, &abort_flag, p.st, 214)) return false;
-        if (!wait_bar(&v_full[s], (jj / VST) & 1, limit, &abort_flag, p.st, 215)) return false;
-        if (first && !wait_bar(&o_empty, (segi & 1) ^ 1, limit, &abort_flag, p.st, 216)) return false;
+      auto issue_s = [&](uint32_t kidx) -> bool {
+        const int s = kidx % RING, buf = j & 1;
+        if (!wait_bar(&r_full[s], (kidx / RING) & 1, limit, &abort_flag, p.st, 211)) return false;
+        if (!wait_bar(&s_empty[buf], ((j >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 212)) return false;
         tc_fence_after();
-        const uint32_t vaddr = smem_u32(sV + s * KT_BYTES), paddr = smem_u32(sP + buf * P_BYTES);
+        const uint64_t ka = sdesc(smem_u32(sR + s * KT_BYTES), 16, 1024), qa = sdesc(smem_u32(sQ), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < TILE / 16; ++kk) {
-          const uint64_t a = sdesc(vaddr + kk * 2048, TILE * 128, 1024);
-          const uint64_t bb = sdesc(paddr + kk * 2048, TILE * 128, 1024);
-          umma_bf16(tmem + tO, a, bb, IDESC_O, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
+          const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
+          umma_bf16(tmem + tS + (2 * buf + (kk & 1)) * H, a, bq, IDESC_S, kk > 1);
         }
-        umma_commit(&p_empty[buf]);
-        umma_commit(&v_empty[s]);
+        umma_commit(&s_full[buf]);
+        umma_commit(&r_empty[s]);
         return true;
       };
-      for (long long t = t1 - 1; t >= t0 && ok; ++seg) {
-        const int b = (int)(t / p.tps);
-        const long long seg_lo = t0 > (long long)b * p.tps ? t0 : (long long)b * p.tps;
-        if (!wait_bar(&q_full, seg & 1, limit, &abort_flag, p.st, 211)) { ok = false; break; }
-        const uint32_t qaddr = smem_u32(sQ);
-        int n_in_seg = 0;
-        for (; t >= seg_lo; --t, ++j, ++n_in_seg) {
-          const int s = j % KST, buf = j & 1;
-          if (!wait_bar(&k_full[s], (j / KST) & 1, limit, &abort_flag, p.st, 212)) { ok = false; break; }
-          if (!wait_bar(&s_empty[buf], ((j >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kaddr = smem_u32(sK + s * KT_BYTES);
+      auto issue_pv = [&](uint32_t jj, uint32_t vidx, bool first) -> bool {
+        const int buf = jj & 1, s = vidx % RING;
+        if (!wait_bar(&p_full[buf], npu[buf] & 1, limit, &abort_flag, p.st, 214)) return false;
+        if (!wait_bar(&r_full[s], (vidx / RING) & 1, limit, &abort_flag, p.st, 215)) return false;
+        if (first && !wait_bar(&o_empty, (seg2 & 1) ^ 1, limit, &abort_flag, p.st, 216)) return false;
+        tc_fence_after();
+        const uint64_t va = sdesc(smem_u32(sR + s * KT_BYTES), TILE * 128, 1024);
+        const uint64_t pa = sdesc(smem_u32(sP + buf * P_BYTES), TILE * 128, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = sdesc(kaddr + (kk / 4) * (TILE * 128) + (kk % 4) * 32, 16, 1024);
-            const uint64_t bq = sdesc(qaddr + (kk / 4) * (H * 128) + (kk % 4) * 32, 16, 1024);
-            umma_bf16(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
-          }
-          umma_commit(&s_full[buf]);
-          umma_commit(&k_empty[s]);
-          if (n_in_seg > 0 && !issue_pv(j - 1, n_in_seg == 1, seg)) { ok = false; break; }
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          const uint64_t a = sdesc_at(va, kk * 2048);
+          const uint64_t bb = sdesc_at(pa, kk * 2048);
+          umma_bf16(tmem + tO + (kk & 1) * H, a, bb, IDESC_O, (first && kk < 2) ? 0u : 1u);
         }
-        if (!ok) break;
-        umma_commit(&q_empty);
-        if (!issue_pv(j - 1, n_in_seg == 1, seg)) { ok = false; break; }
-        umma_commit(&o_full);
+        umma_commit(&p_empty[buf]);
+        umma_commit(&r_empty[s]);
+        npu[buf]++;
+        return true;
+      };
+      for (int g = 0; g < S.n_groups && ok; ++g) {
+        long long t0, t1;
+        S.range(g, cta, t0, t1);
+        for (long long t = t0; t < t1 && ok;) {  // phase 1
+          const int b = (int)(t / S.tps);
+          const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
+          for (; t < seg_end; ++t, ++j)
+            if (!issue_s(ri++)) { ok = false; break; }
+          if (!ok) break;
+          umma_commit(&q_empty);
+          ++nq;
+        }
+        for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: S(t) then PV of the tile before
+          const int b = (int)(t / S.tps);
+          const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
+          int n = 0;
+          uint32_t pj = 0;
+          for (; t >= seg_lo; --t, ++j, ++n) {
+            if (!issue_s(ri++)) { ok = false; break; }
+            if (n > 0 && !issue_pv(pj, ri++, n == 1)) { ok = false; break; }
+            pj = j;
+          }
+          if (!ok) break;
+          umma_commit(&q_empty);
+          ++nq;
+          if (!issue_pv(pj, ri++, n == 1)) { ok = false; break; }
+          umma_commit(&o_full);
+          ++seg2;
+        }
       }
     }
-  } else if (warp >= SM_WG0) {
-    const int wg = (warp - SM_WG0) / 4;    // takes tiles with (j & 1) == wg
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - SM_WG0) / 4;
     const int wq = (warp - SM_WG0) % 4;
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;   // key within the tile == TMEM lane == P^T row
-    const int wg_tid = wq * 32 + lane;
-    const int all_tid = wg * 128 + wg_tid;  // 0..255 over both warpgroups
+    const int row = quarter * 32 + lane;            // key within the tile == TMEM lane == P^T row
+    const int all_tid = wg * 128 + wq * 32 + lane;  // 0..255 over both warpgroups
+    const int swarp = all_tid >> 5;                 // 0..7
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float c = p.c;
     const int ncand = p.N - p.W > 0 ? p.N - p.W : 0;
-    griddep_wait();
-    uint32_t j = 0;
-    int seg = 0;
+    float(*red1)[4][HW][2] = reinterpret_cast<float(*)[4][HW][2]>(&red[0][0][0]);
+    // state the selection accumulates into, cleared before this CTA's first grid-barrier arrival
+    if (cta == 0) {
+      for (int i = all_tid; i < p.B * NBINS; i += 256) p.hist[i] = 0u;
+      for (int i = all_tid; i < p.B; i += 256) p.seq_done[i] = 0;
+    }
+    {  // the selection bitmap (the collect kernel sets bits after this kernel)
+      const long long total = (long long)p.B * p.words;
+      const long long per = (total + S.G - 1) / S.G;
+      const long long w0 = per * cta, w1 = w0 + per < total ? w0 + per : total;
+      for (long long i = w0 + all_tid; i < w1; i += 256) p.bitmap[i] = 0u;
+    }
+    uint32_t j = 0, npu = 0, seg2 = 0;
     bool ok = true;
     // after a failed wait every later wait returns at once: the loop and named-barrier
     // structure stays identical across all 8 warps, only the work is skipped
-    for (long long t = t1 - 1; t >= t0; ++seg) {
-      const int b = (int)(t / p.tps);
-      const long long seg_lo = t0 > (long long)b * p.tps ? t0 : (long long)b * p.tps;
-      const int slot = cta * p.segmax + (b - (int)(t0 / p.tps));
-      // the sequence's lse from every pass-1 partial record of it
-      if (all_tid < H) {
-        const int h = all_tid;
-        const int c_lo = cta_of_tile(p, (long long)b * p.tps), c_hi = cta_of_tile(p, (long long)(b + 1) * p.tps - 1);
-        float M = -INFINITY, L = 0.f;
-        for (int cc = c_lo; cc <= c_hi; ++cc) {
-          const long long ct0 = p.total_tiles * cc / p.G;
-          const int sl = cc * p.segmax + (b - (int)(ct0 / p.tps));
-          const float m = p.ml[(size_t)sl * 2 * H + h], l = p.ml[(size_t)sl * 2 * H + H + h];
-          if (!(l > 0.f)) continue;
-          const float mx = fmaxf(M, m);
-          L = L * (M == -INFINITY ? 0.f : exp2f(M - mx)) + l * exp2f(m - mx);
-          M = mx;
+    for (int g = 0; g < S.n_groups; ++g) {
+      long long t0, t1;
+      S.range(g, cta, t0, t1);
+      // ---------------------------------------------------------------- phase 1
+      for (long long t = t0; t < t1;) {
+        const int b = (int)(t / S.tps);
+        const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+        const long long seg_first = t;
+        float r[HW], l[HW];
+#pragma unroll
+        for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
+        for (; t < seg_end; ++t, ++j) {
+          if (!ok) continue;
+          const int buf = j & 1;
+          if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
+          tc_fence_after();
+          float v[HW], v2[HW];
+          tmem_ld32(tmem + lane_base + tS + 2 * buf * H + wg * HW, v);
+          tmem_ld32(tmem + lane_base + tS + (2 * buf + 1) * H + wg * HW, v2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < HW; h += 2) fadd2(v[h], v[h + 1], v[h], v[h + 1], v2[h], v2[h + 1]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_empty[buf]);
+          const bool valid = (t - (long long)b * S.tps) * TILE + row < p.N;
+          if (t == seg_first) {
+            // a lane's first key of the segment sets its references (invalid lanes only occur in
+            // a sequence's partial last tile, which then is the segment's only tile)
+#pragma unroll
+            for (int h = 0; h < HW; ++h) {
+              r[h] = valid ? v[h] * c : -INFINITY;
+              l[h] = valid ? 1.f : 0.f;
+            }
+            continue;
+          }
+          float dmax = -INFINITY;
+#pragma unroll
+          for (int h = 0; h < HW; ++h) {
+            v[h] = valid ? fmaf(v[h], c, -r[h]) : -INFINITY;  // exponent relative to the reference
+            dmax = fmaxf(dmax, v[h]);
+          }
+          if (__any_sync(0xffffffffu, dmax > REF_SLACK)) {
+            // rare: move the reference of the heads that outgrew it
+#pragma unroll
+            for (int h = 0; h < HW; ++h) {
+              const float d = v[h];
+              if (d > REF_SLACK) {
+                l[h] = l[h] * fast_exp2(-d) + 1.f;
+                r[h] = r[h] + d;
+              } else {
+                l[h] += fast_exp2(d);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < HW; ++h) l[h] += fast_exp2(v[h]);
+          }
         }
-        const float lse2 = M + log2f(L);
-        slse[h] = lse2;
-        if (cta == c_lo) p.lse_out[b * H + h] = lse2 * 0.69314718055994531f;
+        // merge the 128 lanes of each warpgroup. Within a warp a reduce-scatter: at each step a
+        // lane keeps half of its heads and merges in its partner's copy of that half, so after
+        // 16 + 8 + 4 + 2 + 1 exchanges lane i holds head i of the warpgroup's 32. Then the 4
+        // warps through shared memory.
+#pragma unroll
+        for (int half = 16; half >= 1; half >>= 1) {
+          const bool up = (lane & half) != 0;
+#pragma unroll
+          for (int i = 0; i < half; ++i) {
+            const float sm = up ? r[i] : r[i + half], sl = up ? l[i] : l[i + half];
+            float km = up ? r[i + half] : r[i], kl = up ? l[i + half] : l[i];
+            merge_ml(km, kl, __shfl_xor_sync(0xffffffffu, sm, half), __shfl_xor_sync(0xffffffffu, sl, half));
+            r[i] = km;
+            l[i] = kl;
+          }
+        }
+        red1[wg][wq][lane][0] = r[0];
+        red1[wg][wq][lane][1] = l[0];
+        named_bar(3, 256);
+        if (all_tid < H) {
+          const int hg = all_tid / HW, hh = all_tid % HW;
+          float mm = red1[hg][0][hh][0], ll = red1[hg][0][hh][1];
+          for (int w = 1; w < 4; ++w) merge_ml(mm, ll, red1[hg][w][hh][0], red1[hg][w][hh][1]);
+          const size_t sl = (size_t)S.slot(b, cta, S.cta_of(g, (long long)b * S.tps));
+          p.ml[sl * 2 * H + all_tid] = mm;
+          p.ml[sl * 2 * H + H + all_tid] = ll;
+        }
+        named_bar(3, 256);
+      }
+      // ---------------------------------------------------------------- grid barrier
+      named_bar(3, 256);
+      if (all_tid == 0) {
+        __threadfence();
+        atomicAdd(p.gbar, 1u);
+        const unsigned target = (unsigned)S.G * (unsigned)(g + 1);
+        const long long tw = globaltimer_ns();
+        while (*(volatile unsigned*)p.gbar < target) {
+          if (abort_flag) break;
+          if (globaltimer_ns() - tw > limit) {
+            abort_flag = 1;
+            report_status(p.st, kStatusTimeout, 230);
+            break;
+          }
+        }
+        __threadfence();
       }
       named_bar(3, 256);
-      const long long n_seg = t - seg_lo + 1;
-      for (long long x = 0; x < n_seg; ++x, --t, ++j) {
-        if ((int)(j & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
-        const int lt = (int)(t - (long long)b * p.tps);
-        const int buf = j & 1;
-        if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
-        tc_fence_after();
-        float v[H];
+      if (abort_flag) ok = false;
+      // ---------------------------------------------------------------- phase 2
+      for (long long t = t1 - 1; t >= t0;) {
+        const int b = (int)(t / S.tps);
+        const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+        int sg, c_lo, c_hi;
+        S.covering(b, sg, c_lo, c_hi);
+        {  // the sequence's lse from every phase-1 partial of it: 16 threads per partial record
+           // (4 heads each), 16 records per round, then a shuffle and a shared-memory merge
+          const int q4 = all_tid & 15;
+          float M[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, L[4] = {0.f, 0.f, 0.f, 0.f};
+          const float* rec = p.ml + (size_t)S.slot(b, c_lo, c_lo) * 2 * H + 4 * q4;
+          const int n_rec = c_hi - c_lo + 1;
+#pragma unroll 4
+          for (int i = all_tid >> 4; i < n_rec; i += 16) {
+            const float4 m4 = __ldcg(reinterpret_cast<const float4*>(rec + (size_t)i * 2 * H));
+            const float4 l4 = __ldcg(reinterpret_cast<const float4*>(rec + (size_t)i * 2 * H + H));
+            merge_ml(M[0], L[0], m4.x, l4.x);
+            merge_ml(M[1], L[1], m4.y, l4.y);
+            merge_ml(M[2], L[2], m4.z, l4.z);
+            merge_ml(M[3], L[3], m4.w, l4.w);
+          }
 #pragma unroll
-        for (int cc = 0; cc < H / 32; ++cc) {
-          float tmp[32];
-          tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + tS + buf * H + cc * 32, tmp);
-#pragma unroll
-          for (int x2 = 0; x2 < 32; ++x2) v[cc * 32 + x2] = tmp[x2];
+          for (int x = 0; x < 4; ++x) {
+            merge_ml(M[x], L[x], __shfl_xor_sync(0xffffffffu, M[x], 16), __shfl_xor_sync(0xffffffffu, L[x], 16));
+            if (lane < 16) { red[swarp][4 * q4 + x][0] = M[x]; red[swarp][4 * q4 + x][1] = L[x]; }
+          }
+          named_bar(3, 256);
+          if (all_tid < H) {
+            const int h = all_tid;
+            float mm = red[0][h][0], ll = red[0][h][1];
+            for (int w = 1; w < 8; ++w) merge_ml(mm, ll, red[w][h][0], red[w][h][1]);
+            const float lse2 = mm + log2f(ll);
+            slse[h] = lse2;
+            if (cta == c_lo) p.lse_out[b * H + h] = lse2 * 0.69314718055994531f;
+          }
+          named_bar(3, 256);
         }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[buf]);
-        const int key = lt * TILE + row;
-        const bool valid = key < p.N;
-        float score0 = 0.f, score1 = 0.f;
-        uint32_t pk[H / 2];
-#pragma unroll
-        for (int h = 0; h < H; h += 4) {
-          const float4 ls = *reinterpret_cast<const float4*>(&slse[h]);
-          const float p0 = valid ? fast_exp2(fmaf(v[h], c, -ls.x)) : 0.f;
-          const float p1 = valid ? fast_exp2(fmaf(v[h + 1], c, -ls.y)) : 0.f;
-          const float p2 = valid ? fast_exp2(fmaf(v[h + 2], c, -ls.z)) : 0.f;
-          const float p3 = valid ? fast_exp2(fmaf(v[h + 3], c, -ls.w)) : 0.f;
-          score0 += p0 + p1;
-          score1 += p2 + p3;
-          pk[h / 2] = pack_bf16x2(p0, p1);
-          pk[h / 2 + 1] = pack_bf16x2(p2, p3);
-        }
-        const float score = score0 + score1;
-        if (!warp_wait_bar(&p_empty[buf], ((j >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
-        const uint32_t prow = smem_u32(sP + buf * P_BYTES);
-#pragma unroll
-        for (int ch = 0; ch < H / 8; ++ch)
-          st_shared_v4(prow + sw128_off(row, ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
-        const bool is_cand = valid && key < ncand;
-        if (is_cand) p.sc[(size_t)b * ncand + key] = score;
-        const unsigned bin = (__float_as_uint(score) >> 20) & (NBINS - 1);
-        const unsigned act = __ballot_sync(0xffffffffu, is_cand);
-        if (is_cand) {
-          const unsigned peers = __match_any_sync(act, bin);
-          if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&shist[bin], (unsigned)__popc(peers));
-        }
-      }
-      // segment done: warpgroup 0 fetches O^T (lane = output column d, one TMEM column per head)
-      if (wg == 0 && ok) {
-        if (!warp_wait_bar(&o_full, seg & 1, limit, &abort_flag, p.st, 223)) { ok = false; }
-        if (ok) {
+        const long long n_seg = t - seg_lo + 1;
+        for (long long x = 0; x < n_seg; ++x, --t, ++j) {
+          if ((int)(j & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
+          const int lt = (int)(t - (long long)b * S.tps);
+          const int buf = j & 1;  // == wg
+          if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
           tc_fence_after();
-          float* dst = p.opart + (size_t)slot * H * D;
+          float v[H];
 #pragma unroll
           for (int cc = 0; cc < H / 32; ++cc) {
-            float o[32];
-            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + tO + cc * 32, o);
+            float ta[32], tb[32];
+            tmem_ld32(tmem + lane_base + tS + 2 * buf * H + cc * 32, ta);
+            tmem_ld32(tmem + lane_base + tS + (2 * buf + 1) * H + cc * 32, tb);
             tmem_ld_wait();
 #pragma unroll
-            for (int x2 = 0; x2 < 32; ++x2) dst[(cc * 32 + x2) * D + row] = o[x2];
+            for (int x2 = 0; x2 < 32; x2 += 2) fadd2(v[cc * 32 + x2], v[cc * 32 + x2 + 1], ta[x2], ta[x2 + 1], tb[x2], tb[x2 + 1]);
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&o_empty);
+          if (lane == 0) mbar_arrive_cnt(&s_empty[buf], 2);
+          const int key = lt * TILE + row;
+          const bool valid = key < p.N;
+          float sa = 0.f, sb = 0.f;
+          uint32_t pk[H / 2];
+#pragma unroll
+          for (int h = 0; h < H; h += 4) {
+            const float4 ls = *reinterpret_cast<const float4*>(&slse[h]);
+            float e0, e1, e2, e3;
+            ffma2(e0, e1, v[h], v[h + 1], c, c, -ls.x, -ls.y);
+            ffma2(e2, e3, v[h + 2], v[h + 3], c, c, -ls.z, -ls.w);
+            const float p0 = valid ? fast_exp2(e0) : 0.f, p1 = valid ? fast_exp2(e1) : 0.f;
+            const float p2 = valid ? fast_exp2(e2) : 0.f, p3 = valid ? fast_exp2(e3) : 0.f;
+            fadd2(sa, sb, sa, sb, p0, p1);
+            fadd2(sa, sb, sa, sb, p2, p3);
+            pk[h / 2] = pack_bf16x2(p0, p1);
+            pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+          }
+          const float score = sa + sb;
+          if (!warp_wait_bar(&p_empty[buf], (npu & 1) ^ 1, limit, &abort_flag, p.st, 223)) { ok = false; continue; }
+          const uint32_t prow = smem_u32(sP + buf * P_BYTES);
+#pragma unroll
+          for (int ch = 0; ch < H / 8; ++ch)
+            st_shared_v4(prow + sw128_off(row, ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[buf]);
+          ++npu;
+          const bool is_cand = valid && key < ncand;
+          if (is_cand) p.sc[(size_t)b * ncand + key] = score;
+          const unsigned bin = (__float_as_uint(score) >> 20) & (NBINS - 1);
+          const unsigned act = __ballot_sync(0xffffffffu, is_cand);
+          if (is_cand) {
+            const unsigned peers = __match_any_sync(act, bin);
+            if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&shist[bin], (unsigned)__popc(peers));
+          }
         }
-      }
-      // flush this sequence's histogram (both warpgroups are done with the segment)
-      named_bar(3, 256);
-      for (int i = all_tid; i < NBINS; i += 256) {
-        const uint32_t cnt = shist[i];
-        if (cnt) { atomicAdd(&p.hist[(size_t)b * NBINS + i], cnt); shist[i] = 0; }
-      }
-      __threadfence();
-      named_bar(3, 256);
-      // the last CTA to finish this sequence finds the bin of its k-th largest score
-      if (all_tid == 0) {
-        const int c_lo = cta_of_tile(p, (long long)b * p.tps), c_hi = cta_of_tile(p, (long long)(b + 1) * p.tps - 1);
-        s_last = atomicAdd(&p.seq_done[b], 1) == c_hi - c_lo;
-      }
-      named_bar(3, 256);
-      if (s_last) {
+        // segment done: warpgroup 0 fetches O^T (lane = output column d, one TMEM column per head)
+        if (wg == 0 && ok) {
+          if (!warp_wait_bar(&o_full, seg2 & 1, limit, &abort_flag, p.st, 224)) ok = false;
+          if (ok) {
+            tc_fence_after();
+            float* dst = p.opart + (size_t)S.slot(b, cta, c_lo) * H * D;
+#pragma unroll
+            for (int cc = 0; cc < H / 32; ++cc) {
+              float o[32], o2[32];
+              tmem_ld32(tmem + lane_base + tO + cc * 32, o);
+              tmem_ld32(tmem + lane_base + tO + H + cc * 32, o2);
+              tmem_ld_wait();
+#pragma unroll
+              for (int x2 = 0; x2 < 32; ++x2) dst[(cc * 32 + x2) * D + row] = o[x2] + o2[x2];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_empty);
+          }
+        }
+        ++seg2;
+        // flush this sequence's histogram (both warpgroups are done with the segment)
+        named_bar(3, 256);
+        for (int i = all_tid; i < NBINS; i += 256) {
+          const uint32_t cnt = shist[i];
+          if (cnt) { atomicAdd(&p.hist[(size_t)b * NBINS + i], cnt); shist[i] = 0; }
+        }
         __threadfence();
-        int* meta = p.meta + b * 8;
-        const int K = p.K_sel;
-        if (ncand <= K || K == 0) {
-          if (all_tid == 0) {
-            meta[0] = K == 0 ? NBINS : -1;  // -1: every older token; NBINS: none
-            meta[1] = K == 0 ? 0 : ncand;
-            meta[2] = 0; meta[3] = 0; meta[4] = 0;
-          }
-        } else {
-          // thread i owns bins hi..hi-7 (descending); block-inclusive scan of their counts
-          const int hi = NBINS - 1 - 8 * all_tid;
-          unsigned cnt8[8], local = 0;
+        named_bar(3, 256);
+        // the last CTA to finish this sequence finds the bin of its k-th largest score
+        if (all_tid == 0) s_last = atomicAdd(&p.seq_done[b], 1) == c_hi - c_lo;
+        named_bar(3, 256);
+        if (s_last) {
+          __threadfence();
+          int* meta = p.meta + b * 8;
+          const int K = p.K_sel;
+          if (ncand <= K || K == 0) {
+            if (all_tid == 0) {
+              meta[0] = K == 0 ? NBINS : -1;  // -1: every older token; NBINS: none
+              meta[1] = K == 0 ? 0 : ncand;
+              meta[2] = 0; meta[3] = 0; meta[4] = 0;
+            }
+          } else {
+            // thread i owns bins hi..hi-7 (descending); block-inclusive scan of their counts
+            const int hi = NBINS - 1 - 8 * all_tid;
+            unsigned cnt8[8], local = 0;
 #pragma unroll
-          for (int x = 0; x < 8; ++x) { cnt8[x] = __ldcg(&p.hist[(size_t)b * NBINS + hi - x]); local += cnt8[x]; }
-          unsigned incl = local;
+            for (int x = 0; x < 8; ++x) { cnt8[x] = __ldcg(&p.hist[(size_t)b * NBINS + hi - x]); local += cnt8[x]; }
+            unsigned incl = local;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const unsigned nb = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += nb;
-          }
-          const int wv = all_tid >> 5;
-          if (lane == 31) s_wtot[wv] = incl;
-          named_bar(3, 256);
-          unsigned add = 0;
-          for (int x = 0; x < wv; ++x) add += s_wtot[x];
-          incl += add;
-          const unsigned excl = incl - local;
-          if (excl < (unsigned)K && incl >= (unsigned)K) {
-            unsigned run = excl;
-            for (int x = 0; x < 8; ++x) {
-              if (run + cnt8[x] >= (unsigned)K) {
-                meta[0] = hi - x; meta[1] = (int)run; meta[2] = (int)(K - run); meta[3] = 0; meta[4] = 0;
-                break;
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned nb = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += nb;
+            }
+            if (lane == 31) s_wtot[swarp] = incl;
+            named_bar(3, 256);
+            unsigned add = 0;
+            for (int x = 0; x < swarp; ++x) add += s_wtot[x];
+            incl += add;
+            const unsigned excl = incl - local;
+            if (excl < (unsigned)K && incl >= (unsigned)K) {
+              unsigned run = excl;
+              for (int x = 0; x < 8; ++x) {
+                if (run + cnt8[x] >= (unsigned)K) {
+                  meta[0] = hi - x; meta[1] = (int)run; meta[2] = (int)(K - run); meta[3] = 0; meta[4] = 0;
+                  break;
+                }
+                run += cnt8[x];
               }
-              run += cnt8[x];
             }
           }
         }
+        named_bar(3, 256);
       }
-      named_bar(3, 256);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 256); }
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
 // ------------------------------------------------------------------------------------------
-// host launcher
+// host side
 // ------------------------------------------------------------------------------------------
-size_t pass1_smem_bytes(int H, int D) { return 1024 + 2 * (size_t)H * D * 2 + 5 * (size_t)TILE * D * 2; }
-size_t pass2_smem_bytes(int H, int D) {
-  return 1024 + (size_t)H * D * 2 + 5 * (size_t)TILE * D * 2 + 2 * (size_t)TILE * H * 2 + 2048 * 4;
+size_t fused_smem_bytes(int H, int D) {
+  return 1024 + (size_t)H * D * 2 + RING * (size_t)TILE * D * 2 + 2 * (size_t)TILE * H * 2 + NBINS * 4;
 }
 
 cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
@@ -632,21 +584,26 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
   constexpr int H = 64, D = 128;
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(dec_pass1_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)pass1_smem_bytes(H, D));
-    cudaFuncSetAttribute(dec_pass2_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)pass2_smem_bytes(H, D));
+    cudaFuncSetAttribute(dec_fused_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)fused_smem_bytes(H, D));
     configured = true;
   }
+  cudaError_t e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned), stream);
+  if (e != cudaSuccess) return e;
+  // every CTA waits for all others at the grid barrier, so they must all be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.sch.G);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = fused_smem_bytes(H, D);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   {
-    LaunchScope ls("dec_pass1", stream);
-    dec_pass1_kernel<H, D><<<p.G, NTHREADS, pass1_smem_bytes(H, D), stream>>>(tmK, tmQ, p);
-  }
-  cudaError_t e;
-  {
-    LaunchScope ls("dec_pass2", stream);
-    e = launch_k(dec_pass2_kernel<H, D>, dim3(p.G), dim3(NTHREADS), pass2_smem_bytes(H, D), stream, true, tmK, tmV,
-                 tmQ, p);
+    LaunchScope ls("dec_fused", stream);
+    e = cudaLaunchKernelEx(&cfg, dec_fused_kernel<H, D>, tmK, tmV, tmQ, p);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

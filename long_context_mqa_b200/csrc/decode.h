@@ -5,35 +5,33 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "decode_sched.h"
+
 namespace hs2 {
 
 struct DevStatus;
 
 namespace dec {
-// Parameters of the decode (one query per sequence) full-attention + selection kernels.
+// Parameters of the fused decode (one query per sequence) full-attention + selection kernel.
 struct DecParams {
   int B, N, W, K;          // sequences, cache length, window, top-k
-  int tps;                 // 128-key tiles per sequence
-  long long total_tiles;   // B * tps
-  int G;                   // CTAs of the two scan passes
-  int segmax;              // partial records per CTA
+  Sched sch;               // groups of sequences x contiguous tile ranges per CTA
   float c;                 // scale * log2(e)
   long long wait_ns;       // bound of every device-side wait
-  float* ml;               // [G*segmax][2][H] pass-1 partial (max, sum), log2 domain
-  float* lse2;             // [B][H] row logsumexp, log2 domain
+  float* ml;               // [n_groups*G*segmax][2][H] phase-1 partial (max, sum), log2 domain
   float* lse_out;          // [B][H] natural log (caller's lse)
-  float* opart;            // [G*segmax][H][D] pass-2 partial outputs
+  float* opart;            // [n_groups*G*segmax][H][D] phase-2 partial outputs
   float* sc;               // [B][N-W] head-summed scores of the older tokens
   unsigned* hist;          // [B][2048] histogram of score bits 30..20
-  int* seq_done;           // [B] pass-2 CTAs done with each sequence's histogram
-  unsigned* bitmap;        // [B][words] selection bitmap of the older tokens (cleared by pass 1)
+  int* seq_done;           // [B] CTAs done with each sequence's histogram
+  unsigned* bitmap;        // [B][words] selection bitmap of the older tokens (cleared here)
   int words;               // ceil((N - W) / 32)
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
+  unsigned* gbar;          // grid-barrier arrivals (zeroed before every launch)
   DevStatus* st;
 };
-size_t pass1_smem_bytes(int H, int D);
-size_t pass2_smem_bytes(int H, int D);
+size_t fused_smem_bytes(int H, int D);
 cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                                const DecParams& p, cudaStream_t stream);
 }  // namespace dec
@@ -54,10 +52,10 @@ struct SelParams {
   int32_t* idx;                  // [B][S] output
   DevStatus* st;
   // output partials of the decode passes, summed into out by the threshold kernel
-  const float* opart;            // [G*segmax][H][D]
+  const float* opart;            // partial outputs of the decode kernel, at Sched::slot
   __nv_bfloat16* out;            // [B][H][D]
-  int H, D, G, segmax, tps;
-  long long total_tiles;
+  int H, D;
+  dec::Sched sch;
 };
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
 }  // namespace sel

@@ -151,31 +151,53 @@ struct DecodeWs {
   int* meta;
   unsigned long long* bnd;
   size_t bytes;
+  bool ok;  // the schedule's index arithmetic fits (a group of at most 2^32 / G tiles)
 };
+
+// K bytes per decode group. Default: all sequences in one group (a single grid barrier); with the
+// current phase-2 pipeline the L2 reuse of smaller groups does not pay for their extra barriers
+// and pipeline refills. HS2_DEC_GROUP_MB sets a budget (about 72 fits the 126 MB L2).
+static double dec_group_budget_bytes() {
+  static double v = -1.0;
+  if (v < 0) {
+    v = 1e18;
+    const char* e = getenv("HS2_DEC_GROUP_MB");
+    if (e && atof(e) > 0) v = atof(e) * 1024 * 1024;
+  }
+  return v;
+}
 
 static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K, int sms) {
   DecodeWs w{};
   dec::DecParams& p = w.p;
   p.B = B; p.N = N; p.W = W; p.K = K;
-  p.tps = (N + 127) / 128;
-  p.total_tiles = (long long)B * p.tps;
-  if (sms > 256) sms = 256;  // the output combine keeps one table entry per covering CTA
-  p.G = (int)(p.total_tiles < sms ? p.total_tiles : sms);
-  int segmax = 1;
-  for (int cta = 0; cta < p.G; ++cta) {
-    const long long t0 = p.total_tiles * cta / p.G, t1 = p.total_tiles * (cta + 1) / p.G;
-    if (t1 > t0) {
-      const int segs = (int)((t1 - 1) / p.tps - t0 / p.tps + 1);
-      if (segs > segmax) segmax = segs;
-    }
+  // Sequences are grouped so that a group's K cache (bf16) stays well inside the 126 MB L2
+  // between the two phases of the decode kernel.
+  dec::Sched& s = p.sch;
+  s.B = B;
+  s.tps = (N + 127) / 128;
+  const double k_bytes = (double)N * D * 2.0;
+  long long gs = (long long)(dec_group_budget_bytes() / k_bytes);
+  s.gs = (int)(gs < 1 ? 1 : (gs > B ? B : gs));
+  s.n_groups = (B + s.gs - 1) / s.gs;
+  if (sms > 256) sms = 256;  // keeps the schedule's 32-bit tile arithmetic in range
+  const long long g_tiles = (long long)s.gs * s.tps;
+  s.G = (int)(g_tiles < sms ? g_tiles : sms);
+  int cmax = 1;
+  for (int b = 0; b < B; ++b) {
+    int g, lo, hi;
+    s.covering(b, g, lo, hi);
+    if (hi - lo + 1 > cmax) cmax = hi - lo + 1;
   }
-  p.segmax = segmax;
+  s.cmax = cmax;
+  w.ok = (unsigned long long)g_tiles * (unsigned long long)s.G < (1ull << 32);
+  const size_t n_slots = (size_t)B * cmax;
   const int ncand = N - W > 0 ? N - W : 0;
   Carve c{(uint8_t*)ws, 0};
   p.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
-  p.ml = c.take<float>((size_t)p.G * segmax * 2 * H);
-  p.lse2 = c.take<float>((size_t)B * H);
-  p.opart = c.take<float>((size_t)p.G * segmax * H * D);
+  p.gbar = c.take<unsigned>(1);
+  p.ml = c.take<float>(n_slots * 2 * H);
+  p.opart = c.take<float>(n_slots * H * D);
   p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
   p.seq_done = c.take<int>((size_t)B);
@@ -279,6 +301,7 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
   if (Lq == 1) {
     if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
     DecodeWs w = carve_decode(workspace, B, Lk, H, d, window, topk, sms);
+    if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
     if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
     w.p.c = c;
     w.p.wait_ns = wait_limit_ns();
@@ -292,8 +315,7 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
     sel::SelParams sp;
     sp.opart = w.p.opart;
     sp.out = reinterpret_cast<__nv_bfloat16*>(out);
-    sp.H = H; sp.D = d; sp.G = w.p.G; sp.segmax = w.p.segmax; sp.tps = w.p.tps;
-    sp.total_tiles = w.p.total_tiles;
+    sp.H = H; sp.D = d; sp.sch = w.p.sch;
     sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
     sp.ncand = Lk - window > 0 ? Lk - window : 0;
     sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.bnd = w.bnd;

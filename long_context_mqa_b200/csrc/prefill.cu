@@ -175,12 +175,12 @@ __global__ void __launch_bounds__(NT, 1)
         if (!wait_abortable(&r_full[s], (kslot_idx / C::RING) & 1, limit, &abort_flag, p.st, 611)) return false;
         if (!wait_abortable(&s_empty[w], (ns[w] & 1) ^ 1, limit, &abort_flag, p.st, 612)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(smem + C::OFF_Q + w * C::Q_BYTES);
-        const uint32_t ka = smem_u32(smem + C::OFF_RING + s * C::KV_BYTES);
+        const uint64_t qa = sdesc(smem_u32(smem + C::OFF_Q + w * C::Q_BYTES), 16, 1024);
+        const uint64_t ka = sdesc(smem_u32(smem + C::OFF_RING + s * C::KV_BYTES), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc(qa + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
-          const uint64_t bk = sdesc(ka + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+          const uint64_t a = sdesc_at(qa, (kk / 4) * (128 * 128) + (kk % 4) * 32);
+          const uint64_t bk = sdesc_at(ka, (kk / 4) * (128 * 128) + (kk % 4) * 32);
           umma_bf16(tmem + tS + 128 * w, a, bk, IDESC_S, kk > 0);
         }
         umma_commit(&s_full[w]);
@@ -192,12 +192,12 @@ __global__ void __launch_bounds__(NT, 1)
         if (!wait_abortable(&p_full[w], npv[w] & 1, limit, &abort_flag, p.st, 613)) return false;
         if (!wait_abortable(&r_full[s], (vslot_idx / C::RING) & 1, limit, &abort_flag, p.st, 614)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + C::OFF_P + w * C::P_BYTES);
-        const uint32_t va = smem_u32(smem + C::OFF_RING + s * C::KV_BYTES);
+        const uint64_t pa = sdesc(smem_u32(smem + C::OFF_P + w * C::P_BYTES), 16, 1024);
+        const uint64_t va = sdesc(smem_u32(smem + C::OFF_RING + s * C::KV_BYTES), 128 * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t a = sdesc(pa + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
-          const uint64_t bv = sdesc(va + kk * 2048, 128 * 128, 1024);
+          const uint64_t a = sdesc_at(pa, (kk / 4) * (128 * 128) + (kk % 4) * 32);
+          const uint64_t bv = sdesc_at(va, kk * 2048);
           umma_bf16(tmem + tO + D * w, a, bv, IDESC_O, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&pv_done[w]);
@@ -544,17 +544,17 @@ __global__ void __launch_bounds__(NT, 1)
         if (si.n_tiles == 0) continue;
         if (!wait_abortable(&q_full, it & 1, limit, &abort_flag, p.st, 711)) { ok = false; break; }
         ++it;
-        const uint32_t qa = smem_u32(smem + C::OFF_Q);
+        const uint64_t qd = sdesc(smem_u32(smem + C::OFF_Q), 16, 1024);
         for (int j = si.n_tiles - 1; j >= 0; --j, ++kt) {
           const int s = kt % C::KST, buf = kt & 1;
           if (!wait_abortable(&k_full[s], (kt / C::KST) & 1, limit, &abort_flag, p.st, 712)) { ok = false; break; }
           if (!wait_abortable(&s_empty[buf], ((kt >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 713)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t ka = smem_u32(smem + C::OFF_K + s * C::KT_BYTES);
+          const uint64_t ka = sdesc(smem_u32(smem + C::OFF_K + s * C::KT_BYTES), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = sdesc(ka + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
-            const uint64_t bq = sdesc(qa + (kk / 4) * (256 * 128) + (kk % 4) * 32, 16, 1024);
+            const uint64_t a = sdesc_at(ka, (kk / 4) * (128 * 128) + (kk % 4) * 32);
+            const uint64_t bq = sdesc_at(qd, (kk / 4) * (256 * 128) + (kk % 4) * 32);
             umma_bf16(tmem + buf * 256, a, bq, IDESC, kk > 0);
           }
           umma_commit(&s_full[buf]);

@@ -30,37 +30,37 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
   griddep_launch_dependents();
   const int b = blockIdx.y;
   if ((int)blockIdx.x >= n_collect) {
-    // CTAs c_lo..c_hi cover sequence b's tiles (contiguous split of the flattened tile space);
-    // the partial of CTA c for b sits at slot c * segmax + (b - first sequence of c)
-    __shared__ int slot_off[256];  // one entry per covering CTA (at most one CTA per SM)
-    __shared__ float part[128];
+    // the decode kernel's CTAs c_lo..c_hi (of sequence b's group) left one partial each, in
+    // consecutive records from slot b * cmax
+    __shared__ __align__(16) float4 part[8][32];
     const int h = blockIdx.x - n_collect;
-    const long long x_lo = (long long)b * p.tps, x_hi = (long long)(b + 1) * p.tps - 1;
-    const int c_lo = (int)(((x_lo + 1) * p.G - 1) / p.total_tiles);
-    const int c_hi = (int)(((x_hi + 1) * p.G - 1) / p.total_tiles);
+    int g, c_lo, c_hi;
+    p.sch.covering(b, g, c_lo, c_hi);
     const int n_slots = c_hi - c_lo + 1;
-    if (n_slots > 256 || p.D > 128) {
+    if (n_slots > p.sch.cmax || p.D != 128) {
       if (threadIdx.x == 0) report_status(p.st, kStatusBounds, 303);
       return;
     }
-    for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
-      const int c = c_lo + i;
-      const long long ct0 = p.total_tiles * c / p.G;
-      slot_off[i] = c * p.segmax + (b - (int)(ct0 / p.tps));
+    const float* rec = p.opart + ((size_t)p.sch.slot(b, c_lo, c_lo) * p.H + h) * p.D;
+    // lane = 4 output columns, warp w sums the partials w, w + 8, ...
+    const int d4 = threadIdx.x & 31, w = threadIdx.x >> 5;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int i = w; i < n_slots; i += 8) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(rec + (size_t)i * p.H * p.D) + d4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    part[w][d4] = acc;
     __syncthreads();
-    // two threads per output column, each summing half of the slots
-    const int d = threadIdx.x % 128, half = threadIdx.x / 128;
-    const int nh = (n_slots + 1) / 2;
-    const int s_lo = half ? nh : 0, s_hi = half ? n_slots : nh;
-    float acc = 0.f;
-    if (d < p.D) {
-#pragma unroll 8
-      for (int i = s_lo; i < s_hi; ++i) acc += p.opart[((size_t)slot_off[i] * p.H + h) * p.D + d];
+    if (w == 0) {
+      for (int x = 1; x < 8; ++x) {
+        const float4 v = part[x][d4];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * d4;
+      reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x, acc.y);
+      reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z, acc.w);
     }
-    if (half) part[d] = acc;
-    __syncthreads();
-    if (!half && d < p.D) p.out[((size_t)b * p.H + h) * p.D + d] = __float2bfloat16_rn(acc + part[d]);
     return;
   }
   int* meta = p.meta + b * META;

@@ -122,11 +122,11 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t IDESC = idesc_bf16(MH, TILE, 0, 0);
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+      const uint64_t qa = sdesc(smem_u32(sQ), 16, 1024), ka = sdesc(smem_u32(sK), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t a = sdesc(qa + (kk / 4) * (MH * 128) + (kk % 4) * 32, 16, 1024);
-        const uint64_t bk = sdesc(ka + (kk / 4) * (TILE * 128) + (kk % 4) * 32, 16, 1024);
+        const uint64_t a = sdesc_at(qa, (kk / 4) * (MH * 128) + (kk % 4) * 32);
+        const uint64_t bk = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
         umma_bf16(tmem + tS, a, bk, IDESC, kk > 0);
       }
       umma_commit(&mma_bar);
@@ -204,11 +204,11 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t IDESC = idesc_bf16(MH, D, 0, 1);
-      const uint32_t pa = smem_u32(sP), va = smem_u32(sV);
+      const uint64_t pa = sdesc(smem_u32(sP), 16, 1024), va = sdesc(smem_u32(sV), TILE * 128, 1024);
 #pragma unroll
       for (int kk = 0; kk < TILE / 16; ++kk) {
-        const uint64_t a = sdesc(pa + (kk / 4) * (MH * 128) + (kk % 4) * 32, 16, 1024);
-        const uint64_t bv = sdesc(va + kk * 2048, TILE * 128, 1024);
+        const uint64_t a = sdesc_at(pa, (kk / 4) * (MH * 128) + (kk % 4) * 32);
+        const uint64_t bv = sdesc_at(va, kk * 2048);
         umma_bf16(tmem + tO, a, bv, IDESC, (t == 0 && kk == 0) ? 0u : 1u);
       }
       umma_commit(&mma_bar);

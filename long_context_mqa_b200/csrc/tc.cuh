@@ -60,6 +60,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
                : "memory");
 }
+// one arrival that counts as `count` (the barrier's expected count is fixed at init)
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+               "r"(count)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
                    smem_u32(bar)),
@@ -170,6 +176,14 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)(layout & 7u) << 61;
   return d;
+}
+
+// The descriptor of an operand `byte_off` bytes further on: only the start-address field (bits
+// 0-13, address >> 4) changes, and shared-memory addresses stay below 256 KB, so it never carries.
+// Building each k-step's descriptor this way keeps the issuing thread's dependent ALU work to one
+// add per MMA, which matters: a single thread issues every tcgen05.mma of the CTA.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t base, uint32_t byte_off) {
+  return base + (uint64_t)(byte_off >> 4);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
