@@ -110,10 +110,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int cta = blockIdx.x;
   const Sched S = p.sch;
   const long long limit = p.wait_ns;
-  // TMEM columns. Every product is split over two accumulators (even / odd 16-wide k-steps)
-  // so that consecutive MMAs do not wait on one another: S buffer b half x at (2b + x) * H,
-  // O^T half x at 4H + x * H. Readers add the two halves.
-  const uint32_t tS = 0, tO = 4 * H;
+  const uint32_t tS = 0, tO = 2 * H;  // TMEM columns: S buffers 0..2H-1, O^T 2H..3H-1
 
   for (int i = threadIdx.x; i < NBINS; i += NTHREADS) shist[i] = 0;
   if (threadIdx.x == 0) {
@@ -128,7 +125,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -193,23 +190,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, H, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16(D, H, 1, 1);
-      uint32_t ri = 0, j = 0, nq = 0, seg2 = 0;
+      // js counts S tiles (the TMEM S buffer is js & 1), jp phase-2 tiles (their P buffer / owner)
+      uint32_t ri = 0, js = 0, jp = 0, nq = 0, seg2 = 0;
       uint32_t npu[2] = {0, 0};  // PV uses of each P buffer
       bool ok = true;
       auto issue_s = [&](uint32_t kidx) -> bool {
-        const int s = kidx % RING, buf = j & 1;
+        const int s = kidx % RING, buf = js & 1;
         if (!wait_bar(&r_full[s], (kidx / RING) & 1, limit, &abort_flag, p.st, 211)) return false;
-        if (!wait_bar(&s_empty[buf], ((j >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 212)) return false;
+        if (!wait_bar(&s_empty[buf], ((js >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 212)) return false;
         tc_fence_after();
         const uint64_t ka = sdesc(smem_u32(sR + s * KT_BYTES), 16, 1024), qa = sdesc(smem_u32(sQ), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t a = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
           const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
-          umma_bf16(tmem + tS + (2 * buf + (kk & 1)) * H, a, bq, IDESC_S, kk > 1);
+          umma_bf16(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
         }
         umma_commit(&s_full[buf]);
         umma_commit(&r_empty[s]);
+        ++js;
         return true;
       };
       auto issue_pv = [&](uint32_t jj, uint32_t vidx, bool first) -> bool {
@@ -224,7 +223,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int kk = 0; kk < TILE / 16; ++kk) {
           const uint64_t a = sdesc_at(va, kk * 2048);
           const uint64_t bb = sdesc_at(pa, kk * 2048);
-          umma_bf16(tmem + tO + (kk & 1) * H, a, bb, IDESC_O, (first && kk < 2) ? 0u : 1u);
+          umma_bf16(tmem + tO, a, bb, IDESC_O, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&p_empty[buf]);
         umma_commit(&r_empty[s]);
@@ -238,29 +237,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int b = (int)(t / S.tps);
           const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
-          for (; t < seg_end; ++t, ++j)
+          for (; t < seg_end; ++t)
             if (!issue_s(ri++)) { ok = false; break; }
           if (!ok) break;
           umma_commit(&q_empty);
           ++nq;
         }
-        for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: S(t) then PV of the tile before
+        for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2
           const int b = (int)(t / S.tps);
           const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
+          // S of a tile, then PV of the tile before it
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
-          int n = 0;
-          uint32_t pj = 0;
-          for (; t >= seg_lo; --t, ++j, ++n) {
-            if (!issue_s(ri++)) { ok = false; break; }
-            if (n > 0 && !issue_pv(pj, ri++, n == 1)) { ok = false; break; }
-            pj = j;
+          for (uint32_t x = 0; x < n; ++x, ++jp) {
+            if (!issue_s(base + (x == 0 ? 0u : 2 * x - 1))) { ok = false; break; }
+            if (x > 0 && !issue_pv(jp - 1, base + 2 * x, x == 1)) { ok = false; break; }
           }
           if (!ok) break;
           umma_commit(&q_empty);
           ++nq;
-          if (!issue_pv(pj, ri++, n == 1)) { ok = false; break; }
+          if (!issue_pv(jp - 1, base + 2 * n - 1, n == 1)) { ok = false; break; }
           umma_commit(&o_full);
           ++seg2;
+          ri = base + 2 * n;
+          t = seg_lo - 1;
         }
       }
     }
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const long long w0 = per * cta, w1 = w0 + per < total ? w0 + per : total;
       for (long long i = w0 + all_tid; i < w1; i += 256) p.bitmap[i] = 0u;
     }
-    uint32_t j = 0, npu = 0, seg2 = 0;
+    uint32_t js = 0, jp = 0, ri = 0, npu = 0, seg2 = 0;  // as in the tcgen05 issuer
     bool ok = true;
     // after a failed wait every later wait returns at once: the loop and named-barrier
     // structure stays identical across all 8 warps, only the work is skipped
@@ -302,17 +302,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float r[HW], l[HW];
 #pragma unroll
         for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
-        for (; t < seg_end; ++t, ++j) {
+        for (; t < seg_end; ++t, ++js) {
           if (!ok) continue;
-          const int buf = j & 1;
-          if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
+          const int buf = js & 1;
+          if (!warp_wait_bar(&s_full[buf], (js >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
           tc_fence_after();
-          float v[HW], v2[HW];
-          tmem_ld32(tmem + lane_base + tS + 2 * buf * H + wg * HW, v);
-          tmem_ld32(tmem + lane_base + tS + (2 * buf + 1) * H + wg * HW, v2);
+          float v[HW];
+          tmem_ld32(tmem + lane_base + tS + buf * H + wg * HW, v);
           tmem_ld_wait();
-#pragma unroll
-          for (int h = 0; h < HW; h += 2) fadd2(v[h], v[h + 1], v[h], v[h + 1], v2[h], v2[h + 1]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[buf]);
@@ -379,6 +376,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         named_bar(3, 256);
       }
+      ri += (uint32_t)(t1 - t0);  // the phase-1 K items of the ring
       // ---------------------------------------------------------------- grid barrier
       named_bar(3, 256);
       if (all_tid == 0) {
@@ -435,26 +433,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           named_bar(3, 256);
         }
-        const long long n_seg = t - seg_lo + 1;
-        for (long long x = 0; x < n_seg; ++x, --t, ++j) {
-          if ((int)(j & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
+        const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
+        for (uint32_t x = 0; x < n; ++x, --t, ++jp, ++js) {
+          if ((int)(jp & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
           const int lt = (int)(t - (long long)b * S.tps);
-          const int buf = j & 1;  // == wg
-          if (!warp_wait_bar(&s_full[buf], (j >> 1) & 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
+          const int buf = jp & 1;   // == wg: this warpgroup's P buffer
+          const int sbi = js & 1;   // the TMEM S buffer of this tile
+          if (!warp_wait_bar(&s_full[sbi], (js >> 1) & 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
           tc_fence_after();
           float v[H];
 #pragma unroll
           for (int cc = 0; cc < H / 32; ++cc) {
-            float ta[32], tb[32];
-            tmem_ld32(tmem + lane_base + tS + 2 * buf * H + cc * 32, ta);
-            tmem_ld32(tmem + lane_base + tS + (2 * buf + 1) * H + cc * 32, tb);
-            tmem_ld_wait();
+            float tmp[32];
+            tmem_ld32(tmem + lane_base + tS + sbi * H + cc * 32, tmp);
 #pragma unroll
-            for (int x2 = 0; x2 < 32; x2 += 2) fadd2(v[cc * 32 + x2], v[cc * 32 + x2 + 1], ta[x2], ta[x2 + 1], tb[x2], tb[x2 + 1]);
+            for (int x2 = 0; x2 < 32; ++x2) v[cc * 32 + x2] = tmp[x2];
           }
+          tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cnt(&s_empty[buf], 2);
+          if (lane == 0) mbar_arrive_cnt(&s_empty[sbi], 2);
           const int key = lt * TILE + row;
           const bool valid = key < p.N;
           float sa = 0.f, sb = 0.f;
@@ -491,6 +489,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&shist[bin], (unsigned)__popc(peers));
           }
         }
+        ri = base + 2 * n;
         // segment done: warpgroup 0 fetches O^T (lane = output column d, one TMEM column per head)
         if (wg == 0 && ok) {
           if (!warp_wait_bar(&o_full, seg2 & 1, limit, &abort_flag, p.st, 224)) ok = false;
@@ -499,12 +498,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float* dst = p.opart + (size_t)S.slot(b, cta, c_lo) * H * D;
 #pragma unroll
             for (int cc = 0; cc < H / 32; ++cc) {
-              float o[32], o2[32];
+              float o[32];
               tmem_ld32(tmem + lane_base + tO + cc * 32, o);
-              tmem_ld32(tmem + lane_base + tO + H + cc * 32, o2);
               tmem_ld_wait();
 #pragma unroll
-              for (int x2 = 0; x2 < 32; ++x2) dst[(cc * 32 + x2) * D + row] = o[x2] + o2[x2];
+              for (int x2 = 0; x2 < 32; ++x2) dst[(cc * 32 + x2) * D + row] = o[x2];
             }
             tc_fence_before();
             __syncwarp();
@@ -569,7 +567,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 256); }
 }
 
 // ------------------------------------------------------------------------------------------

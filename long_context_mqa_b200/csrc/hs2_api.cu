@@ -154,31 +154,17 @@ struct DecodeWs {
   bool ok;  // the schedule's index arithmetic fits (a group of at most 2^32 / G tiles)
 };
 
-// K bytes per decode group. Default: all sequences in one group (a single grid barrier); with the
-// current phase-2 pipeline the L2 reuse of smaller groups does not pay for their extra barriers
-// and pipeline refills. HS2_DEC_GROUP_MB sets a budget (about 72 fits the 126 MB L2).
-static double dec_group_budget_bytes() {
-  static double v = -1.0;
-  if (v < 0) {
-    v = 1e18;
-    const char* e = getenv("HS2_DEC_GROUP_MB");
-    if (e && atof(e) > 0) v = atof(e) * 1024 * 1024;
-  }
-  return v;
-}
-
 static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K, int sms) {
   DecodeWs w{};
   dec::DecParams& p = w.p;
   p.B = B; p.N = N; p.W = W; p.K = K;
-  // Sequences are grouped so that a group's K cache (bf16) stays well inside the 126 MB L2
-  // between the two phases of the decode kernel.
+  // One group of all sequences. (The schedule can split them into groups small enough for a
+  // group's K to stay in L2 between the phases; measured on B200 the per-group grid barrier,
+  // pipeline drain and refill cost more than the HBM re-reads they save.)
   dec::Sched& s = p.sch;
   s.B = B;
   s.tps = (N + 127) / 128;
-  const double k_bytes = (double)N * D * 2.0;
-  long long gs = (long long)(dec_group_budget_bytes() / k_bytes);
-  s.gs = (int)(gs < 1 ? 1 : (gs > B ? B : gs));
+  s.gs = B;
   s.n_groups = (B + s.gs - 1) / s.gs;
   if (sms > 256) sms = 256;  // keeps the schedule's 32-bit tile arithmetic in range
   const long long g_tiles = (long long)s.gs * s.tps;
