@@ -318,21 +318,13 @@ def run_gpu(args):
     ws_sp_bytes = hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S)
     ws_sp = [torch.zeros(ws_sp_bytes, dtype=torch.uint8, device=dev) for _ in range(wl.n_sparse)]
     stream = torch.cuda.current_stream()
-    # the sparse layers of a hybrid block only depend on the full layer's indices: each runs on
-    # its own stream (and workspace) and the main stream joins them before the next step
-    side = [torch.cuda.Stream(device=dev) for _ in range(wl.n_sparse)]
-    ev_idx = torch.cuda.Event()
-    ev_done = [torch.cuda.Event() for _ in range(wl.n_sparse)]
 
     def step():
+        # one hybrid block: the full-attention layer selects, then its sparse layers run one after
+        # another (in the model each sparse layer's query comes from the previous layer's output)
         hs2.full_attn_select(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws_full)
-        ev_idx.record(stream)
         for i in range(wl.n_sparse):
-            side[i].wait_event(ev_idx)
-            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i], stream=side[i])
-            ev_done[i].record(side[i])
-        for i in range(wl.n_sparse):
-            stream.wait_event(ev_done[i])
+            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i])
 
     # ---------------- device-resident throughput
     with ClockSampler(local) as clocks:

@@ -126,9 +126,10 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const h
  * device memory -- e.g. a plugin's enqueue hook inside an inference runtime that forbids
  * allocation on that path and offers no scratch buffer, or a process whose device-memory
  * budget is fixed up front. Same arguments and results as hs2_sparse_attn, minus the
- * workspace: the scratch is a 16 MiB array inside the library, held by every GPU that loads
+ * workspace: the scratch is a 4 KiB array inside the library, held by every GPU that loads
  * it until process exit. Returns HS2_ERR_WORKSPACE (nothing launched) when the shape needs
- * more scratch than that (hs2_sparse_attn_workspace_bytes(...) > 16 MiB). The first call on
+ * more scratch than that (hs2_sparse_attn_workspace_bytes(...) > 4 KiB; with the current
+ * kernels every supported shape needs only its 256-byte status word). The first call on
  * each device performs a one-time set-up (it looks up the array's device address) and should
  * come before any stream capture. All calls share the array: calls whose GPU work overlaps
  * (e.g. on different streams) race. The device status word of these calls is internal.

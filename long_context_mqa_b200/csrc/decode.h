@@ -65,13 +65,11 @@ struct SpParams {
   const __nv_bfloat16 *Q, *K, *V;
   const int32_t* idx;
   int B, Lq, Lk, S;
-  int nsplit, split_slots;    // slots of idx handled per CTA (multiple of 128)
+  int nsplit, split_slots;    // CTAs per query row (a cluster when > 1, at most 16) and the
+                              // idx slots each handles (a multiple of 128)
   float c;                    // scale * log2(e)
   __nv_bfloat16* out;
   float* lse;                 // may be null
-  float* opart;               // [B*Lq*nsplit][H][D] (nsplit > 1)
-  float* mlpart;              // [B*Lq*nsplit][2][H]
-  int* counters;              // [B*Lq] split arrivals (zeroed before every launch)
   long long wait_ns;
   DevStatus* st;
 };

@@ -201,25 +201,19 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
 static size_t carve_sparse(void* ws, int B, int Lq, int H, int D, int S, int sms, sparse::SpParams* p) {
   const long long rows = (long long)B * Lq;
   const int tiles = (S + 127) / 128;
-  int nsplit = 1;
-  if (rows < sms && tiles > 1) nsplit = tiles;  // few rows: one 128-slot tile per CTA
+  // few query rows (decode): split each row's index list over a cluster of CTAs (at most 16),
+  // which merge their partial results through distributed shared memory
+  int nsplit = 1, per = tiles;
+  if (rows < sms && tiles > 1) {
+    per = (tiles + 15) / 16;
+    nsplit = (tiles + per - 1) / per;
+  }
   Carve c{(uint8_t*)ws, 0};
   DevStatus* st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
-  float* opart = nullptr;
-  float* mlpart = nullptr;
-  int* counters = nullptr;
-  if (nsplit > 1) {
-    opart = c.take<float>((size_t)rows * nsplit * H * D);
-    mlpart = c.take<float>((size_t)rows * nsplit * 2 * H);
-    counters = c.take<int>((size_t)rows);
-  }
   if (p) {
     p->st = st;
-    p->opart = opart;
-    p->mlpart = mlpart;
-    p->counters = counters;
     p->nsplit = nsplit;
-    p->split_slots = nsplit > 1 ? 128 : tiles * 128;
+    p->split_slots = per * 128;
   }
   return c.off;
 }

@@ -6,14 +6,15 @@
 // cudaMalloc afterwards. They can pass inputs and outputs, but not the workspace hs2_sparse_attn
 // asks for. This entry point uses instead a scratch array that lives in the library itself.
 //
-// The array below is a file-scope __device__ object of kScratchBytes (16 MiB): every GPU on
-// which this library's code is loaded holds those 16 MiB until the process exits. Host code
+// The array below is a file-scope __device__ object of kScratchBytes (4 KiB): every GPU on
+// which this library's code is loaded holds it until the process exits. The sparse kernels need
+// only their 256-byte status word from a workspace (split rows merge in distributed shared
+// memory), so every supported shape fits; larger needs are still rejected, not overrun. Host code
 // cannot use the array's name as a device address (it is a host-side stand-in), so the first
 // call on each device looks the address up with cudaGetSymbolAddress while that device is
 // current, and caches it per device. That first call on a device should therefore happen before
 // any stream capture. All calls share the one array and it keeps what the last call left there:
-// each call clears the status word it needs at zero; the split partials are fully overwritten
-// before they are read. Calls whose GPU work overlaps (for example on two streams) race on the
+// each call clears the status word it needs at zero. Calls whose GPU work overlaps (for example on two streams) race on the
 // array. Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
 #include <mutex>
 
@@ -22,7 +23,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB per device
+constexpr size_t kScratchBytes = 4096;  // per device
 __device__ __align__(256) unsigned char g_sparse_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -51,7 +52,7 @@ extern "C" hs2_status hs2_sparse_attn_noalloc(const hs2_bf16* Q, const hs2_bf16*
   if (!Q || !K || !V || !idx || !out) return HS2_ERR_INVALID_ARG;
   const size_t need = hs2_sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S);
   if (need == 0) return HS2_ERR_INVALID_ARG;
-  if (need > kScratchBytes) return HS2_ERR_WORKSPACE;  // shape needs more than the 16 MiB scratch
+  if (need > kScratchBytes) return HS2_ERR_WORKSPACE;  // shape needs more than the scratch holds
   void* scratch = nullptr;
   const hs2_status st = scratch_for_current_device(&scratch);
   if (st != HS2_OK) return st;

@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
 
 __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   griddep_wait();
+  griddep_launch_dependents();
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   __shared__ unsigned dh[256];
   __shared__ unsigned long long s_prefix, s_mask, s_and, s_or;

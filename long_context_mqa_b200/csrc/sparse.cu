@@ -10,9 +10,13 @@
 //   O += P V_sel             tcgen05, M = 64 heads, N = d, P (bf16) K-major in shared memory
 // TMEM rows of an M = 64 accumulator sit in lanes 0..15 of each 32-lane quarter, so thread
 // (warp q, lane l < 16) owns head row 16 q + l. Two CTAs share an SM, so one CTA's gathers
-// overlap the other's math. With one split the CTA writes the final bf16 output (and lse); with
-// several, every split writes an unnormalised partial and the split that arrives last on the
-// row's counter merges them (few query rows, as in decode).
+// overlap the other's math. With one split the CTA writes the final bf16 output (and lse). With
+// few query rows (decode) a row's index list is split over a cluster of CTAs; head h of the row
+// is merged by cluster rank h % n: after a first cluster barrier (every CTA is done with its K/V
+// tiles) each CTA stores its unnormalised O rows into their owners' shared memory and its
+// per-head (max, sum) into every CTA's, and after a second barrier each CTA merges its heads
+// from local shared memory. Launched as a programmatic dependent: the prologue overlaps the
+// previous kernel's tail and every global read waits for it.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -49,8 +53,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ unsigned vmask[TILE / 32];
-  __shared__ int s_last;
-  __shared__ float wgt[33 * MH];  // merge weights [nsplit][64] and 1/L [64] (nsplit <= 32)
+  __shared__ float wgt[17 * MH];  // merge weights [nsplit][heads of this rank] and their 1/L
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x;  // flattened query row b * Lq + i
@@ -68,6 +71,9 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   const bool owns = lane < 16 && head < H;  // a real head
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
+  // every input may come from the kernels before this one on the stream
+  griddep_wait();
+  griddep_launch_dependents();
   // ---- query -> shared (K-major, 128B swizzle): rows 0..H-1 by cp.async, padding rows zero
   {
     const __nv_bfloat16* q = p.Q + (size_t)r * H * D;
@@ -224,15 +230,16 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   }
   cp_async_wait_all();
   if (__syncthreads_or(bad) && tid == 0) report_status(p.st, kStatusBounds, 403);
-  // ---- epilogue: this thread's O row
-  if (ntiles > 0 && ok) {  // block-uniform
+  // ---- epilogue
+  const bool have = ntiles > 0 && ok;  // block-uniform
+  if (p.nsplit == 1) {
+    if (have) {
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      float o[32];
-      tmem_ld32(tmem + lane_base + tO + cc * 32, o);
-      tmem_ld_wait();
-      if (owns) {
-        if (p.nsplit == 1) {
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + tO + cc * 32, o);
+        tmem_ld_wait();
+        if (owns) {
           const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
           uint32_t pk[16];
 #pragma unroll
@@ -240,82 +247,92 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)r * H + head) * D + cc * 32);
 #pragma unroll
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.opart + (((size_t)r * p.nsplit + split) * H + head) * D + cc * 32);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) dst[x] = make_float4(o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
         }
       }
     }
-  } else if (owns && p.nsplit > 1) {
-    float* dst = p.opart + (((size_t)r * p.nsplit + split) * H + head) * D;
-    for (int x = 0; x < D; ++x) dst[x] = 0.f;
+    if (owns && p.lse) p.lse[(size_t)r * H + head] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
+    return;
   }
-  if (owns) {
-    if (p.nsplit == 1) {
-      if (p.lse) p.lse[(size_t)r * H + head] = (m_run + log2f(l_run)) * 0.69314718055994531f;
-    } else {
-      float* ml = p.mlpart + ((size_t)r * p.nsplit + split) * 2 * H;
-      ml[head] = l_run > 0.f ? m_run : -INFINITY;
-      ml[H + head] = l_run;
+  // cluster merge. Exchange buffers in the (now free) K/V tile region of every CTA:
+  //   xO[s][k][D]  O row of head rank + k*n from split s      (HPR = ceil(H / n) heads per rank)
+  //   xm[s][MH], xl[s][MH]  split s's max (log2 units) and sum per head
+  const int n = p.nsplit;
+  const uint32_t rank = cluster_ctarank();
+  const int HPR = (H + n - 1) / n;
+  float* xO = reinterpret_cast<float*>(sK);
+  float* xm = xO + (size_t)n * HPR * D;
+  float* xl = xm + n * MH;
+  // (n * HPR * D + 2 * n * MH) floats <= (H + n) * D + 32 * MH floats fit in the 2 tile buffers
+  static_assert((H + 16) * D * 4 + 32 * MH * 4 <= 2 * Lay::KT_BYTES, "exchange buffers fit");
+  cluster_sync_all();  // every CTA of the row is done with its K and V tiles
+  {
+    const int owner = head % n, k = head / n;
+    const uint32_t o_dst = dsmem_addr(smem_u32(xO + ((size_t)split * HPR + k) * D), owner);
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      float o[32];
+      if (have) {
+        tmem_ld32(tmem + lane_base + tO + cc * 32, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o[x] = 0.f;
+      }
+      if (owns) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) st_dsmem_v4(o_dst + (cc * 32 + 4 * x) * 4, o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
+      }
+    }
+    if (owns) {
+      const float mv = l_run > 0.f && have ? m_run : -INFINITY, lv = have ? l_run : 0.f;
+      const uint32_t m_loc = smem_u32(xm + split * MH + head), l_loc = smem_u32(xl + split * MH + head);
+      for (int s2 = 0; s2 < n; ++s2) {
+        st_dsmem_f32(dsmem_addr(m_loc, s2), mv);
+        st_dsmem_f32(dsmem_addr(l_loc, s2), lv);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
-  if (p.nsplit > 1) {
-    // the split that arrives last on this row's counter merges the row's partials
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&p.counters[r], 1) == p.nsplit - 1;
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      const float* mlr = p.mlpart + (size_t)r * p.nsplit * 2 * H;
-      if (tid < H) {
-        float M = -INFINITY, L = 0.f;
-        for (int s2 = 0; s2 < p.nsplit; ++s2)
-          if (__ldcg(&mlr[s2 * 2 * H + H + tid]) > 0.f) M = fmaxf(M, __ldcg(&mlr[s2 * 2 * H + tid]));
-        for (int s2 = 0; s2 < p.nsplit; ++s2) {
-          const float l = __ldcg(&mlr[s2 * 2 * H + H + tid]);
-          const float w = l > 0.f ? exp2f(__ldcg(&mlr[s2 * 2 * H + tid]) - M) : 0.f;
-          wgt[s2 * MH + tid] = w;
-          L += l * w;
-        }
-        wgt[p.nsplit * MH + tid] = L > 0.f ? 1.f / L : 0.f;
-        if (p.lse) p.lse[(size_t)r * H + tid] = (M + log2f(L)) * 0.69314718055994531f;
+  cluster_sync_all();  // all partials have landed; nothing reads another CTA's memory after this
+  // merge weights of this rank's heads (thread k < HPR: head rank + k*n)
+  if (tid < HPR) {
+    const int h = (int)rank + tid * n;
+    if (h < H) {
+      float M = -INFINITY, L = 0.f;
+      for (int s2 = 0; s2 < n; ++s2)
+        if (xl[s2 * MH + h] > 0.f) M = fmaxf(M, xm[s2 * MH + h]);
+      for (int s2 = 0; s2 < n; ++s2) {
+        const float l = xl[s2 * MH + h];
+        const float w = l > 0.f ? exp2f(xm[s2 * MH + h] - M) : 0.f;
+        wgt[s2 * MH + tid] = w;
+        L += l * w;
       }
-      __syncthreads();
-      // every thread owns EPT float4 columns; a split's loads are all issued before any is used
-      const float4* op = reinterpret_cast<const float4*>(p.opart + (size_t)r * p.nsplit * H * D);
-      constexpr int EPT_ALL = H * D / 4 / NT;
-      constexpr int EPT = EPT_ALL > 8 ? 8 : EPT_ALL;
-#pragma unroll 1
-      for (int base = 0; base < EPT_ALL; base += EPT) {
-        float4 acc[EPT];
-#pragma unroll
-        for (int q2 = 0; q2 < EPT; ++q2) acc[q2] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s2 = 0; s2 < p.nsplit; ++s2) {
-          float4 v4[EPT];
-#pragma unroll
-          for (int q2 = 0; q2 < EPT; ++q2) v4[q2] = __ldcg(&op[(size_t)s2 * (H * D / 4) + tid + (base + q2) * NT]);
-#pragma unroll
-          for (int q2 = 0; q2 < EPT; ++q2) {
-            const float w = wgt[s2 * MH + (tid + (base + q2) * NT) / (D / 4)];
-            acc[q2].x += w * v4[q2].x; acc[q2].y += w * v4[q2].y; acc[q2].z += w * v4[q2].z; acc[q2].w += w * v4[q2].w;
-          }
-        }
-#pragma unroll
-        for (int q2 = 0; q2 < EPT; ++q2) {
-          const int e = tid + (base + q2) * NT;
-          const float inv = wgt[p.nsplit * MH + e / (D / 4)];
-          uint2 o2;
-          o2.x = pack_bf16x2(acc[q2].x * inv, acc[q2].y * inv);
-          o2.y = pack_bf16x2(acc[q2].z * inv, acc[q2].w * inv);
-          reinterpret_cast<uint2*>(p.out + (size_t)r * H * D)[e] = o2;
-        }
-      }
+      wgt[16 * MH + tid] = L > 0.f ? 1.f / L : 0.f;
+      if (p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
     }
+  }
+  __syncthreads();
+  // this rank's heads, 4 columns per thread per step
+  for (int e4 = tid; e4 < HPR * D / 4; e4 += NT) {
+    const int k = e4 / (D / 4), d4 = e4 % (D / 4);
+    const int h = (int)rank + k * n;
+    if (h >= H) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s2 = 0; s2 < n; ++s2) {
+      const float w = wgt[s2 * MH + k];
+      const float4 v4 = reinterpret_cast<const float4*>(xO + ((size_t)s2 * HPR + k) * D)[d4];
+      acc.x += w * v4.x; acc.y += w * v4.y; acc.z += w * v4.z; acc.w += w * v4.w;
+    }
+    const float inv = wgt[16 * MH + k];
+    uint2 o2;
+    o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(p.out + ((size_t)r * H + h) * D)[d4] = o2;
   }
 }
 
@@ -330,18 +347,32 @@ static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SpLayout<H, D>::BYTES);
+    cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     configured = true;
   }
   const int rows = p.B * p.Lq;
-  if (p.nsplit > 1 && cudaMemsetAsync(p.counters, 0, (size_t)rows * sizeof(int), stream) != cudaSuccess)
-    return cudaErrorUnknown;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows, p.nsplit);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = SpLayout<H, D>::BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of one row form a cluster
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = p.nsplit;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = p.nsplit > 1 ? attr : attr + 1;
+  cfg.numAttrs = p.nsplit > 1 ? 2 : 1;
   LaunchScope ls("sparse_attn", stream);
-  sparse_attn_kernel<H, D><<<dim3(rows, p.nsplit), NT, SpLayout<H, D>::BYTES, stream>>>(p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H, D>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse(const SpParams& p, int H, int D, cudaStream_t stream) {
-  if (p.nsplit > 32) return cudaErrorInvalidValue;  // merge-weight table holds 32 splits
+  if (p.nsplit < 1 || p.nsplit > 16) return cudaErrorInvalidValue;  // merge table and cluster size
   if (H == 64 && D == 128) return launch_t<64, 128>(p, stream);
   if (H == 16 && D == 64) return launch_t<16, 64>(p, stream);
   return cudaErrorInvalidValue;

@@ -2,10 +2,11 @@
 
 Such callers (for example a plugin whose enqueue hook runs inside an inference runtime that
 forbids device allocation there and provides no scratch buffer) use this entry point, which
-keeps its scratch in a 16 MiB array inside the library instead of a caller workspace. These
+keeps its scratch in a 4 KiB array inside the library instead of a caller workspace. These
 tests call it through the C ABI and require the same results as hs2_sparse_attn (which is
-given its own workspace), on two calls in a row, and a clear error for shapes whose scratch
-would not fit.
+given its own workspace), on two calls in a row, including shapes whose rows split over a
+cluster; and that every supported shape's workspace fits the scratch, while an invalid shape
+is refused before anything is launched.
 """
 import ctypes
 
@@ -50,12 +51,13 @@ def test_noalloc_matches_workspace_entry_point_two_calls_in_a_row():
         np.testing.assert_allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), rtol=0, atol=2e-3)
 
 
-def test_noalloc_rejects_shapes_beyond_its_scratch():
+def test_noalloc_scratch_covers_every_shape_and_refuses_invalid_ones():
     hs2, f = _entry()
-    # 100 query rows split 9 ways need ~30 MB of fp32 partials: more than the 16 MiB scratch
-    assert hs2.sparse_attn_workspace_bytes(100, 1, 8, 64, 128, 1152) > 16 << 20
+    # split rows merge in distributed shared memory: only the status word is needed
+    for B, Lq, S in [(1, 1, 128), (8, 1, 1152), (100, 1, 1152), (147, 1, 2048), (1, 32768, 1152)]:
+        assert 0 < hs2.sparse_attn_workspace_bytes(B, Lq, 8, 64, 128, S) <= 4096
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     i = torch.zeros(16, dtype=torch.int32, device="cuda")
-    rc = f(x.data_ptr(), x.data_ptr(), x.data_ptr(), i.data_ptr(), 100, 1, 8, 64, 128, 1152, 0.1, x.data_ptr(), None,
+    rc = f(x.data_ptr(), x.data_ptr(), x.data_ptr(), i.data_ptr(), 0, 1, 8, 64, 128, 1152, 0.1, x.data_ptr(), None,
            torch.cuda.current_stream().cuda_stream)
-    assert rc == hs2.ERR_WORKSPACE
+    assert rc == hs2.ERR_INVALID_ARG
