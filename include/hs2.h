@@ -168,6 +168,12 @@ HS2_API hs2_status hs2_clear_device_status(void* workspace, hs2_stream stream);
 HS2_API void hs2_set_wait_limit_ns(long long limit_ns);
 HS2_API hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_ns, hs2_stream stream);
 
+/* hs2_selftest_exp2: evaluates, for the n device floats x[i] (n even), the software 2^x the
+ * score pass computes on the FMA pipes (into y_soft) and the hardware approximation (MUFU ex2,
+ * flushing subnormals) it is mixed with (into y_mufu), so a test can bound their error. No
+ * counterpart in the paper: a check of an arithmetic building block. */
+HS2_API hs2_status hs2_selftest_exp2(const float* x, float* y_soft, float* y_mufu, int n, hs2_stream stream);
+
 /* ---------------------------------------------------------------------------------
  * Diagnostics (never needed on the compute path)
  * ---------------------------------------------------------------------------------

@@ -69,6 +69,8 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_set_wait_limit_ns.restype = None
     lib.hs2_selftest_wait_timeout.argtypes = [P, sz, ll, P]
     lib.hs2_selftest_wait_timeout.restype = i32
+    lib.hs2_selftest_exp2.argtypes = [P, P, P, i32, P]
+    lib.hs2_selftest_exp2.restype = i32
     lib.hs2_kernel_launches.restype = ctypes.c_ulonglong
     lib.hs2_profile_enable.argtypes = [ctypes.c_char_p]
     lib.hs2_profile_enable.restype = None
@@ -231,6 +233,15 @@ def set_wait_limit_ns(ns: int) -> None:
 def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int, stream=None) -> None:
     _check(lib.hs2_selftest_wait_timeout(workspace.data_ptr(), workspace.numel(), int(limit_ns), _stream_ptr(stream)),
            "hs2_selftest_wait_timeout")
+
+
+def selftest_exp2(x: torch.Tensor, stream=None):
+    """(software 2^x, MUFU 2^x) of the device float32 tensor x (even length), see hs2.h."""
+    _need(x, "x", torch.float32, 1)
+    ys, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(lib.hs2_selftest_exp2(x.data_ptr(), ys.data_ptr(), ym.data_ptr(), x.numel(), _stream_ptr(stream)),
+           "hs2_selftest_exp2")
+    return ys, ym
 
 
 def kernel_launches() -> int:

@@ -392,6 +392,27 @@ hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_bytes, lo
   return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* ys, float* ym, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 >= n) return;
+  float a = x[i], b = x[i + 1];
+  ym[i] = fast_exp2(a);
+  ym[i + 1] = fast_exp2(b);
+  exp2_fma2(a, b);
+  ys[i] = a;
+  ys[i + 1] = b;
+}
+
+hs2_status hs2_selftest_exp2(const float* x, float* y_soft, float* y_mufu, int n, hs2_stream stream) {
+  if (!x || !y_soft || !y_mufu || n <= 0 || (n & 1)) return HS2_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  {
+    LaunchScope ls("selftest_exp2", reinterpret_cast<cudaStream_t>(stream));
+    selftest_exp2_kernel<<<(n / 2 + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y_soft, y_mufu, n);
+  }
+  return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
 unsigned long long hs2_kernel_launches(void) { return g_launches.load(); }
 
 void hs2_profile_enable(const char* kernel) {

@@ -34,6 +34,10 @@ namespace prefill {
 
 constexpr int NT = 320;
 constexpr float LOG2E = 1.4426950408889634f;
+// Of every 16 score-pass exponentials, how many exp2_fma2 computes on the FMA pipes instead of
+// the MUFU. Measured on B200 at L = 32k: 0 and 6 take the same time (the loop is not MUFU-bound),
+// so the MUFU does all of them.
+constexpr int SOFT_EXP2 = 0;
 
 struct PfParams {
   int B, L, H;
@@ -359,10 +363,10 @@ template <int H, int D>
 struct ScCfg {
   static constexpr int NQ = 256 / H;        // queries per item
   static constexpr int QW = NQ / 2;         // queries per warpgroup
-  static constexpr int CAP = H == 64 ? 2048 : 1152;  // candidate slots per query
+  static constexpr int CAP = H == 64 ? 1920 : 1152;  // candidate slots per query
   static constexpr int Q_BYTES = 256 * D * 2;
   static constexpr int KT_BYTES = 128 * D * 2;
-  static constexpr int KST = 2;
+  static constexpr int KST = H == 64 ? 3 : 2;        // K tiles in flight (from L2)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_C = OFF_K + KST * KT_BYTES;
@@ -596,29 +600,48 @@ __global__ void __launch_bounds__(NT, 1)
         if (ok) {
         tc_fence_after();
         const int key = j * 128 + row;
-#pragma unroll 1
+        // this warpgroup's 128 columns (QW queries x H heads) in one go: the TMEM load latency
+        // is paid once per tile, not once per 16 columns
+        float v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128, v0);
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 32, v1);
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 64, v2);
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 96, v3);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[buf]);  // the S buffer is free for the next tile
+        auto col = [&](int i) -> float { return i < 32 ? v0[i] : i < 64 ? v1[i - 32] : i < 96 ? v2[i - 64] : v3[i - 96]; };
+#pragma unroll
         for (int qq = 0; qq < C::QW; ++qq) {
           const int q = wg * C::QW + qq;
           const int t = si.tq0 + q;
           const bool cand = t < p.L && key <= t - p.W;
           if (!__any_sync(0xffffffffu, cand)) continue;  // warp-uniform: no lane has a candidate here
-          float sa = 0.f, sb = 0.f;
+          // the exponentials can be shared between the MUFU (ex2) and the FMA pipes (exp2_fma2);
+          // four independent pairs of partial sums keep the additions off one dependency chain
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int hc = 0; hc < H; hc += 16) {
-            float v[16];
-            tmem_ld16(tmem + lane_base + buf * 256 + q * H + hc, v);
-            tmem_ld_wait();
+            float e[16];
 #pragma unroll
             for (int x = 0; x < 16; x += 4) {
               const float4 nl = *reinterpret_cast<const float4*>(&slse2[q * H + hc + x]);  // -lse2
-              float e0, e1, e2, e3;
-              ffma2(e0, e1, v[x], v[x + 1], c, c, nl.x, nl.y);
-              ffma2(e2, e3, v[x + 2], v[x + 3], c, c, nl.z, nl.w);
-              fadd2(sa, sb, sa, sb, fast_exp2(e0), fast_exp2(e1));
-              fadd2(sa, sb, sa, sb, fast_exp2(e2), fast_exp2(e3));
+              const int i = qq * H + hc + x;
+              ffma2(e[x], e[x + 1], col(i), col(i + 1), c, c, nl.x, nl.y);
+              ffma2(e[x + 2], e[x + 3], col(i + 2), col(i + 3), c, c, nl.z, nl.w);
+            }
+#pragma unroll
+            for (int x = 0; x < SOFT_EXP2; x += 2) exp2_fma2(e[x], e[x + 1]);
+#pragma unroll
+            for (int x = SOFT_EXP2; x < 16; ++x) e[x] = fast_exp2(e[x]);
+#pragma unroll
+            for (int x = 0; x < 16; x += 2) {
+              const int a = (x / 2) % 4;
+              fadd2(acc[2 * a], acc[2 * a + 1], acc[2 * a], acc[2 * a + 1], e[x], e[x + 1]);
             }
           }
-          const float score = sa + sb;
+          const float score = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           const unsigned long long k64 =
               ((unsigned long long)__float_as_uint(score) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)key);
           const bool take = cand && k64 > theta[q];
@@ -631,9 +654,6 @@ __global__ void __launch_bounds__(NT, 1)
             if (take) cbuf[(size_t)q * C::CAP + base + __popc(m & lt_mask)] = k64;
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[buf]);
         }
         wg_bar(wg);
         for (int qq = 0; qq < C::QW; ++qq) {

@@ -325,6 +325,30 @@ __device__ __forceinline__ void fadd2(float& dx, float& dy, float ax, float ay, 
       : "f"(ax), "f"(ay), "f"(bx), "f"(by));
 }
 // max of 32 values (balanced tree)
+// 2^x for a pair of values on the FMA and integer pipes (no MUFU), to share the exponentials of
+// a MUFU-bound loop between both units. Cody and Waite's range reduction: 2^x = 2^j * 2^f with
+// j = round(x) (adding 1.5*2^23 leaves j in the low mantissa bits) and f = x - j in [-1/2, 1/2];
+// 2^f is a degree-5 polynomial whose coefficients minimise the maximum relative error on that
+// interval (fitted by Lawson's iteratively reweighted least squares in fit_exp2.py: 1.5e-7, about
+// 2.3e-7 with float32 Horner evaluation); 2^j is added to the exponent field. Inputs below -126
+// are clamped to -126 (2^-126 ~ 1.2e-38, a zero next to the sums it feeds); valid for x <= 127.
+__device__ __forceinline__ void exp2_fma2(float& a, float& b) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  const float xa = fmaxf(a, -126.f), xb = fmaxf(b, -126.f);
+  float ta, tb, ja, jb, fa, fb;
+  fadd2(ta, tb, xa, xb, kRound, kRound);
+  fadd2(ja, jb, ta, tb, -kRound, -kRound);
+  fadd2(fa, fb, xa, xb, -ja, -jb);
+  float pa = __uint_as_float(0x3aae0555u), pb = pa;  // c5
+  ffma2(pa, pb, pa, pb, fa, fb, __uint_as_float(0x3c1e8692u), __uint_as_float(0x3c1e8692u));  // c4
+  ffma2(pa, pb, pa, pb, fa, fb, __uint_as_float(0x3d635b72u), __uint_as_float(0x3d635b72u));  // c3
+  ffma2(pa, pb, pa, pb, fa, fb, __uint_as_float(0x3e75fc8au), __uint_as_float(0x3e75fc8au));  // c2
+  ffma2(pa, pb, pa, pb, fa, fb, __uint_as_float(0x3f317214u), __uint_as_float(0x3f317214u));  // c1
+  ffma2(pa, pb, pa, pb, fa, fb, __uint_as_float(0x3f800001u), __uint_as_float(0x3f800001u));  // c0
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
 __device__ __forceinline__ float max32(const float (&v)[32]) {
   float a[16];
 #pragma unroll
