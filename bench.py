@@ -289,6 +289,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph of the steps")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (small profiling cases)")
     ap.add_argument("--cache", type=int, default=0, help="override cache length (small profiling cases)")
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill full-attention + selection")
@@ -353,23 +354,48 @@ def run_gpu(args):
         for i in range(wl.n_sparse):
             hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i])
 
-    # ---------------- device-resident throughput
+    # ---------------- device-resident throughput: the K timed steps run as one CUDA graph (the
+    # library's timing events around each dec_fused launch become nodes of that graph)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    graph, graph_note = None, None
+    launches0 = hs2.kernel_launches()
+    if not args.eager:
+        try:
+            hs2.profile_enable("dec_fused")
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(args.steps):
+                    step()
+            hs2.profile_enable(None)
+            graph.replay()            # upload and warm the graph (untimed)
+            torch.cuda.synchronize()
+        except Exception as e:       # fall back to eager launches, said so in the line
+            hs2.profile_enable(None)
+            hs2.profile_read("dec_fused")
+            graph, graph_note = None, f"eager (graph capture failed: {e})"
+            torch.cuda.synchronize()
+    launches = hs2.kernel_launches() - launches0
     with ClockSampler(local) as clocks:
-        for _ in range(args.warmup):
-            step()
         _barrier(world)
-        hs2.profile_enable("dec_fused")
-        launches0 = hs2.kernel_launches()
+        if graph is None:
+            hs2.profile_enable("dec_fused")
+            launches0 = hs2.kernel_launches()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         clocks.start_region()
         e0.record(stream)
-        for _ in range(args.steps):
-            step()
+        if graph is not None:
+            graph.replay()
+        else:
+            for _ in range(args.steps):
+                step()
         e1.record(stream)
         e1.synchronize()
         clocks.end_region()
-        launches = hs2.kernel_launches() - launches0
-        hs2.profile_enable(None)
+        if graph is None:
+            launches = hs2.kernel_launches() - launches0
+            hs2.profile_enable(None)
         _barrier(world)
     ms_total = _max_over_ranks(e0.elapsed_time(e1), world)
     dec_ms, dec_n = hs2.profile_read("dec_fused")
@@ -381,7 +407,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     hs2.profile_enable(None)
     breakdown = {}
-    for name in ("dec_fused", "sel_collect", "sel_final", "sparse_attn"):
+    for name in ("dec_fused", "dec_redo", "sel_collect", "sel_rescore", "sel_final", "sparse_attn"):
         kms, kn = hs2.profile_read(name)
         if kn:
             breakdown[name] = kms / n_brk
@@ -463,7 +489,9 @@ def run_gpu(args):
                                    f"H={wl.H}, d={wl.d}, window {wl.window} + top-{wl.topk}, "
                                    f"{wl.n_sparse} sparse layers per step",
                        "global_batch": wl.B * world, "seq_len": wl.Lk, "parallelism": f"dp{world} (replicas)",
-                       "l2": "inputs larger than L2 (1.07 GB K+V per GPU), no flush"},
+                       "l2": "inputs larger than L2 (1.07 GB K+V per GPU), no flush",
+                       "launch": (f"the {args.steps} timed steps replayed as one CUDA graph" if graph is not None
+                                  else (graph_note or "eager launches"))},
             "roofline": roofline, "step_roofline": step_roof, "kernel_ms_per_step": breakdown,
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "note": "public Python API, pinned host inputs, result read every step"},

@@ -180,8 +180,10 @@ HS2_API hs2_status hs2_selftest_exp2(const float* x, float* y_soft, float* y_muf
  * hs2_kernel_launches: number of CUDA kernels this library has launched since it was
  * loaded (all devices, all streams).
  * hs2_profile_enable: NULL turns per-kernel timing off; "*" times every kernel; any other
- * string times only the kernel of that name (e.g. "dec_pass2", "sparse_attn"). While on,
- * the library records a pair of CUDA events around each matching launch on its stream.
+ * string times only the kernel of that name (e.g. "dec_fused", "sparse_attn"). While on,
+ * the library records a pair of CUDA events around each matching launch on its stream; on a
+ * stream being captured into a CUDA graph they become event-record nodes of the graph (the
+ * events then hold the latest replay's times, and must be read before the events are reused).
  * hs2_profile_read: waits for the recorded events of `kernel`, returns their summed
  * duration in milliseconds and the number of launches, and forgets them. Returns 0, or -1
  * if an event could not be read.

@@ -105,12 +105,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __shared__ __align__(16) float red[8][H][2];  // merge scratch (phase-1 view: [2][4][HW][2])
   __shared__ int s_last;
   __shared__ unsigned s_wtot[8];
+  __shared__ unsigned s_cnt2[8][2];
+  __shared__ float s_lmm[2][2];
+  __shared__ int s_band[3];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
   const Sched S = p.sch;
   const long long limit = p.wait_ns;
   const uint32_t tS = 0, tO = 2 * H;  // TMEM columns: S buffers 0..2H-1, O^T 2H..3H-1
+  // the exact redo runs only if the sampled launch before it flagged a sequence (every CTA reads
+  // the same final count, so the whole grid leaves together, before any barrier)
+  if (p.fallback && *(volatile const int*)&p.ovf[p.B] == 0) return;
+  // in the redo, only flagged sequences are processed (every role skips the same segments)
+  auto skip_seq = [&](int b) -> bool { return p.fallback && *(volatile const int*)&p.ovf[b] == 0; };
 
   for (int i = threadIdx.x; i < NBINS; i += NTHREADS) shist[i] = 0;
   if (threadIdx.x == 0) {
@@ -161,13 +169,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (long long t = t0; t < t1 && ok;) {  // phase 1: K, ascending
           const int b = (int)(t / S.tps);
           const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          if (skip_seq(b)) { t = seg_end; continue; }
           if (!load_q(b)) { ok = false; break; }
-          for (; t < seg_end; ++t)
-            if (!load_tile(&tmK, (int)(t - (long long)b * S.tps), b, keep)) { ok = false; break; }
+          for (; t < seg_end; ++t) {
+            const long long lt = t - (long long)b * S.tps;
+            if (lt % p.sample_stride == 0 && !load_tile(&tmK, (int)lt, b, keep)) { ok = false; break; }
+          }
         }
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: descending
           const int b = (int)(t / S.tps);
           const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          if (skip_seq(b)) { t = seg_lo - 1; continue; }
           if (!load_q(b)) { ok = false; break; }
           // in the order the tensor core consumes them: S of a tile needs its K, then the PV of
           // the tile before it (the next higher one) needs that tile's V
@@ -236,9 +248,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (long long t = t0; t < t1 && ok;) {  // phase 1
           const int b = (int)(t / S.tps);
           const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          if (skip_seq(b)) { t = seg_end; continue; }
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
           for (; t < seg_end; ++t)
-            if (!issue_s(ri++)) { ok = false; break; }
+            if ((t - (long long)b * S.tps) % p.sample_stride == 0 && !issue_s(ri++)) { ok = false; break; }
           if (!ok) break;
           umma_commit(&q_empty);
           ++nq;
@@ -246,6 +259,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2
           const int b = (int)(t / S.tps);
           const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          if (skip_seq(b)) { t = seg_lo - 1; continue; }
           const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
           // S of a tile, then PV of the tile before it
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
@@ -278,10 +292,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float(*red1)[4][HW][2] = reinterpret_cast<float(*)[4][HW][2]>(&red[0][0][0]);
     // state the selection accumulates into, cleared before this CTA's first grid-barrier arrival
     if (cta == 0) {
-      for (int i = all_tid; i < p.B * NBINS; i += 256) p.hist[i] = 0u;
-      for (int i = all_tid; i < p.B; i += 256) p.seq_done[i] = 0;
+      for (int i = all_tid; i < p.B * NBINS; i += 256)
+        if (!skip_seq(i / NBINS)) p.hist[i] = 0u;
+      for (int i = all_tid; i < p.B; i += 256)
+        if (!skip_seq(i)) p.seq_done[i] = 0;
+      if (!p.fallback)
+        for (int i = all_tid; i <= p.B; i += 256) p.ovf[i] = 0;
     }
-    {  // the selection bitmap (the collect kernel sets bits after this kernel)
+    if (!p.fallback) {  // the selection bitmap (the collect kernel sets bits after this kernel)
       const long long total = (long long)p.B * p.words;
       const long long per = (total + S.G - 1) / S.G;
       const long long w0 = per * cta, w1 = w0 + per < total ? w0 + per : total;
@@ -294,18 +312,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int g = 0; g < S.n_groups; ++g) {
       long long t0, t1;
       S.range(g, cta, t0, t1);
-      // ---------------------------------------------------------------- phase 1
+      // ---------------------------------------------------------------- phase 1 (sampled tiles)
+      uint32_t n1 = 0;  // K tiles phase 1 took through the ring
       for (long long t = t0; t < t1;) {
         const int b = (int)(t / S.tps);
         const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
-        const long long seg_first = t;
+        if (skip_seq(b)) { t = seg_end; continue; }  // uniform: every softmax warp skips it
+        bool first = true;
         float r[HW], l[HW];
 #pragma unroll
         for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
-        for (; t < seg_end; ++t, ++js) {
+        for (; t < seg_end; ++t) {
+          if ((t - (long long)b * S.tps) % p.sample_stride != 0) continue;
+          const uint32_t jt = js++;
+          ++n1;
           if (!ok) continue;
-          const int buf = js & 1;
-          if (!warp_wait_bar(&s_full[buf], (js >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
+          const int buf = jt & 1;
+          if (!warp_wait_bar(&s_full[buf], (jt >> 1) & 1, limit, &abort_flag, p.st, 221)) { ok = false; continue; }
           tc_fence_after();
           float v[HW];
           tmem_ld32(tmem + lane_base + tS + buf * H + wg * HW, v);
@@ -314,9 +337,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[buf]);
           const bool valid = (t - (long long)b * S.tps) * TILE + row < p.N;
-          if (t == seg_first) {
+          if (first) {
             // a lane's first key of the segment sets its references (invalid lanes only occur in
-            // a sequence's partial last tile, which then is the segment's only tile)
+            // a sequence's partial last tile, which then is the segment's last sampled tile)
+            first = false;
 #pragma unroll
             for (int h = 0; h < HW; ++h) {
               r[h] = valid ? v[h] * c : -INFINITY;
@@ -376,7 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         named_bar(3, 256);
       }
-      ri += (uint32_t)(t1 - t0);  // the phase-1 K items of the ring
+      ri += n1;  // the phase-1 K items of the ring
       // ---------------------------------------------------------------- grid barrier
       named_bar(3, 256);
       if (all_tid == 0) {
@@ -400,6 +424,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (long long t = t1 - 1; t >= t0;) {
         const int b = (int)(t / S.tps);
         const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+        if (skip_seq(b)) { t = seg_lo - 1; continue; }  // uniform: every softmax warp skips it
         int sg, c_lo, c_hi;
         S.covering(b, sg, c_lo, c_hi);
         {  // the sequence's lse from every phase-1 partial of it: 16 threads per partial record
@@ -428,12 +453,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float mm = red[0][h][0], ll = red[0][h][1];
             for (int w = 1; w < 8; ++w) merge_ml(mm, ll, red[w][h][0], red[w][h][1]);
             const float lse2 = mm + log2f(ll);
-            slse[h] = lse2;
-            if (cta == c_lo) p.lse_out[b * H + h] = lse2 * 0.69314718055994531f;
+            slse[h] = lse2;  // of the sampled tiles only: the reference of p' = exp2(s*c - lse2)
           }
           named_bar(3, 256);
         }
         const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
+        float la = 0.f, lb = 0.f;  // sums of p' over this warp's keys for heads 2*lane, 2*lane + 1
         for (uint32_t x = 0; x < n; ++x, --t, ++jp, ++js) {
           if ((int)(jp & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
           const int lt = (int)(t - (long long)b * S.tps);
@@ -469,8 +494,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fadd2(sa, sb, sa, sb, p2, p3);
             pk[h / 2] = pack_bf16x2(p0, p1);
             pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+            v[h] = p0; v[h + 1] = p1; v[h + 2] = p2; v[h + 3] = p3;
           }
           const float score = sa + sb;
+          // p' above 2^64 (or not finite): the sampled reference was far too low for this
+          // sequence; flag it for the exact redo (the sum is above 2^64 iff a term is)
+          if (__any_sync(0xffffffffu, valid && !(score <= 1.8446744e19f)) && lane == 0) {
+            if (atomicExch(&p.ovf[b], 1) == 0) atomicAdd(&p.ovf[p.B], 1);
+          }
           if (!warp_wait_bar(&p_empty[buf], (npu & 1) ^ 1, limit, &abort_flag, p.st, 223)) { ok = false; continue; }
           const uint32_t prow = smem_u32(sP + buf * P_BYTES);
 #pragma unroll
@@ -480,6 +511,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[buf]);
           ++npu;
+          // per-head sums over the warp's 32 keys by a reduce-scatter: at each step a lane keeps
+          // half of its values and adds its partner's copy of that half; at the end lane L holds
+          // heads 2L and 2L + 1
+#pragma unroll
+          for (int stp = 0; stp < 5; ++stp) {
+            const int cnt = 64 >> stp, dist = 16 >> stp;
+            const bool up = (lane & dist) != 0;
+#pragma unroll
+            for (int i = 0; i < cnt / 2; ++i) {
+              const float send = up ? v[i] : v[i + cnt / 2];
+              const float keep = up ? v[i + cnt / 2] : v[i];
+              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, dist);
+            }
+          }
+          la += v[0];
+          lb += v[1];
           const bool is_cand = valid && key < ncand;
           if (is_cand) p.sc[(size_t)b * ncand + key] = score;
           const unsigned bin = (__float_as_uint(score) >> 20) & (NBINS - 1);
@@ -490,6 +537,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         ri = base + 2 * n;
+        {  // this segment's per-head sums of p' over its keys: one record per (sequence, CTA)
+          float* rr = &red[0][0][0];  // [8 warps][64 heads]
+          rr[swarp * H + 2 * lane] = la;
+          rr[swarp * H + 2 * lane + 1] = lb;
+          named_bar(3, 256);
+          if (all_tid < H) {
+            float L = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) L += rr[w * H + all_tid];
+            p.lp[(size_t)S.slot(b, cta, c_lo) * H + all_tid] = L;
+          }
+        }
         // segment done: warpgroup 0 fetches O^T (lane = output column d, one TMEM column per head)
         if (wg == 0 && ok) {
           if (!warp_wait_bar(&o_full, seg2 & 1, limit, &abort_flag, p.st, 224)) ok = false;
@@ -522,14 +581,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (all_tid == 0) s_last = atomicAdd(&p.seq_done[b], 1) == c_hi - c_lo;
         named_bar(3, 256);
         if (s_last) {
+          // The last CTA of the sequence: exact per-head totals L'_h = sum_j p'_jh give the exact
+          // lse (lse2 = lse2' + log2 L'); the true score of key j is sum_h p'_jh / L'_h, so
+          // score'_j / max L' <= score_j <= score'_j / min L'. With rho = min L' / max L', a key
+          // whose score' is above (upper edge of the k-th score' bin) / rho is certainly chosen,
+          // one below rho * (lower edge) certainly not; the keys in between (the band) are
+          // re-scored exactly (sel_rescore) and the top "need" of them by exact score taken.
           __threadfence();
           int* meta = p.meta + b * 8;
           const int K = p.K_sel;
+          if (all_tid < H) {
+            const float* rec = p.lp + (size_t)S.slot(b, c_lo, c_lo) * H + all_tid;
+            float L = 0.f;
+            for (int i = 0; i <= c_hi - c_lo; ++i) L += __ldcg(rec + (size_t)i * H);
+            const float lse2 = slse[all_tid] + log2f(L);
+            p.lse_out[b * H + all_tid] = lse2 * 0.69314718055994531f;
+            p.lse2x[b * H + all_tid] = lse2;
+            p.lsum[b * H + all_tid] = L;
+            float mn = L, mx = L;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            }
+            if (lane == 0) { s_lmm[swarp][0] = mn; s_lmm[swarp][1] = mx; }
+          }
+          named_bar(3, 256);
           if (ncand <= K || K == 0) {
             if (all_tid == 0) {
-              meta[0] = K == 0 ? NBINS : -1;  // -1: every older token; NBINS: none
+              meta[0] = K == 0 ? NBINS : -1;  // every older token above bin -1, or none above NBINS
               meta[1] = K == 0 ? 0 : ncand;
-              meta[2] = 0; meta[3] = 0; meta[4] = 0;
+              meta[2] = 0;
+              meta[3] = NBINS + 1;            // empty band
+              meta[4] = 0; meta[5] = 0;
             }
           } else {
             // thread i owns bins hi..hi-7 (descending); block-inclusive scan of their counts
@@ -552,12 +636,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (excl < (unsigned)K && incl >= (unsigned)K) {
               unsigned run = excl;
               for (int x = 0; x < 8; ++x) {
-                if (run + cnt8[x] >= (unsigned)K) {
-                  meta[0] = hi - x; meta[1] = (int)run; meta[2] = (int)(K - run); meta[3] = 0; meta[4] = 0;
-                  break;
-                }
+                if (run + cnt8[x] >= (unsigned)K) { s_band[2] = hi - x; break; }
                 run += cnt8[x];
               }
+            }
+            named_bar(3, 256);
+            if (all_tid == 0) {
+              const float rho = fminf(s_lmm[0][0], s_lmm[1][0]) / fmaxf(s_lmm[0][1], s_lmm[1][1]);
+              const unsigned beta = (unsigned)s_band[2];
+              // score' of the k-th key lies in [lo, hi) of bin beta; slack for rounding of the sums
+              const float lo = __uint_as_float(beta << 20), up_e = __uint_as_float((beta + 1) << 20);
+              const float lower = rho * lo * (1.f - 3e-5f);
+              const float upper = up_e / rho * (1.f + 3e-5f);
+              const int b_lo = (int)((__float_as_uint(lower) >> 20) & (NBINS - 1));
+              int b_hi = (int)(__float_as_uint(upper) >> 20);
+              b_hi = b_hi > NBINS - 1 ? NBINS - 1 : b_hi;
+              s_band[0] = b_lo;
+              s_band[1] = b_hi;
+            }
+            named_bar(3, 256);
+            const int b_lo = s_band[0], b_hi = s_band[1];
+            unsigned above = 0, band = 0;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const int bin = hi - x;
+              if (bin > b_hi) above += cnt8[x];
+              else if (bin >= b_lo) band += cnt8[x];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              above += __shfl_xor_sync(0xffffffffu, above, off);
+              band += __shfl_xor_sync(0xffffffffu, band, off);
+            }
+            if (lane == 0) { s_cnt2[swarp][0] = above; s_cnt2[swarp][1] = band; }
+            named_bar(3, 256);
+            if (all_tid == 0) {
+              unsigned ab = 0, bd = 0;
+              for (int w = 0; w < 8; ++w) { ab += s_cnt2[w][0]; bd += s_cnt2[w][1]; }
+              meta[0] = b_hi;             // bins above: chosen outright
+              meta[1] = (int)ab;
+              meta[2] = K - (int)ab;      // to take from the band by exact score
+              meta[3] = b_lo;             // bins b_lo..b_hi: the band
+              meta[4] = 0;                // band keys collected so far
+              meta[5] = (int)bd;          // band size expected
             }
           }
         }
@@ -586,24 +707,33 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
                          (int)fused_smem_bytes(H, D));
     configured = true;
   }
-  cudaError_t e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned), stream);
-  if (e != cudaSuccess) return e;
-  // every CTA waits for all others at the grid barrier, so they must all be resident at once
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.sch.G);
-  cfg.blockDim = dim3(NTHREADS);
-  cfg.dynamicSmemBytes = fused_smem_bytes(H, D);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  {
-    LaunchScope ls("dec_fused", stream);
-    e = cudaLaunchKernelEx(&cfg, dec_fused_kernel<H, D>, tmK, tmV, tmQ, p);
+  // the sampled launch, then the exact redo of any sequence it flagged (normally none: the redo's
+  // CTAs read the flag count and leave at once). Every CTA waits for all others at the grid
+  // barrier, so both launches are cooperative.
+  for (int pass = 0; pass < 2; ++pass) {
+    DecParams q = p;
+    if (pass == 1) {
+      q.fallback = 1;
+      q.sample_stride = 1;
+    }
+    cudaError_t e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned), stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.sch.G);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = fused_smem_bytes(H, D);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+      LaunchScope ls(pass == 0 ? "dec_fused" : "dec_redo", stream);
+      e = cudaLaunchKernelEx(&cfg, dec_fused_kernel<H, D>, tmK, tmV, tmQ, q);
+    }
+    if (e != cudaSuccess) return e;
   }
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -29,6 +29,12 @@ struct DecParams {
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
   unsigned* gbar;          // grid-barrier arrivals (zeroed before every launch)
+  int sample_stride;       // phase 1 takes every sample_stride-th tile of each sequence
+  float* lp;               // [B*cmax][H] per-(sequence, CTA) sums of p' = exp2(s*c - lse2')
+  float* lsum;             // [B][H] their totals L'_h (the output is sum(O') / L')
+  float* lse2x;            // [B][H] exact lse, log2 units (for the exact re-score of the band)
+  int* ovf;                // [B + 1] sequences whose p' overflowed the sampled reference (and a count)
+  int fallback;            // 0: the sampled schedule; 1: redo the flagged sequences with every tile
   DevStatus* st;
 };
 size_t fused_smem_bytes(int H, int D);
@@ -38,7 +44,8 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
 
 namespace sel {
 constexpr int NBINS = 2048;
-constexpr int META = 8;  // ints per sequence: beta, above, need, (unused), cnt_bnd
+constexpr int META = 8;  // ints per sequence: bin above which all are in, their count, need, lowest band
+                         // bin, band keys collected, band size expected
 // Top-k selection over a materialised score vector per sequence (decode path).
 struct SelParams {
   int B, N, W, K, S;
@@ -51,11 +58,19 @@ struct SelParams {
   unsigned long long* bnd;       // [B][ncand] boundary-bin candidates (score bits << 32 | ~index)
   int32_t* idx;                  // [B][S] output
   DevStatus* st;
-  // output partials of the decode passes, summed into out by the threshold kernel
-  const float* opart;            // partial outputs of the decode kernel, at Sched::slot
+  // output records of the decode kernel, summed into out by the collect kernel's extra CTAs
+  const float* opart;            // unnormalised output records, at Sched::slot
+  const float* lsum;             // [B][H] totals L' dividing them
   __nv_bfloat16* out;            // [B][H][D]
   int H, D;
   dec::Sched sch;
+  // exact re-score of the band keys
+  const __nv_bfloat16* qry;      // [B][H][D] the decode queries
+  const __nv_bfloat16* kc;       // [B][N][D] the K cache
+  const float* lse2x;            // [B][H] exact lse, log2 units
+  float c;                       // scale * log2(e)
+  int sms;
+  long long wait_ns;             // bound of the re-score kernel's wait for its MMA
 };
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
 }  // namespace sel

@@ -106,6 +106,14 @@ static cudaEvent_t take_event() {
   return e;
 }
 
+// While a stream is being captured into a CUDA graph the timing events become event-record nodes
+// of the graph (they then hold the times of the graph's latest replay).
+static unsigned record_flags(cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return cudaEventRecordDefault;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+}
+
 LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : slot_(-1), stream_(stream), name_(name) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (!g_prof_on.load(std::memory_order_relaxed)) return;
@@ -113,7 +121,7 @@ LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : slot_(-1), str
   if (g_prof_filter != "*" && g_prof_filter != name) return;
   cudaEvent_t a = take_event();
   if (!a) return;
-  cudaEventRecord(a, stream);
+  cudaEventRecordWithFlags(a, stream, record_flags(stream));
   t_pending_start = a;
   slot_ = 0;
 }
@@ -123,7 +131,7 @@ LaunchScope::~LaunchScope() {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   cudaEvent_t b = take_event();
   if (!b) return;
-  cudaEventRecord(b, stream_);
+  cudaEventRecordWithFlags(b, stream_, record_flags(stream_));
   g_prof[name_].push_back({t_pending_start, b});
   t_pending_start = nullptr;
 }
@@ -184,6 +192,13 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   p.gbar = c.take<unsigned>(1);
   p.ml = c.take<float>(n_slots * 2 * H);
   p.opart = c.take<float>(n_slots * H * D);
+  p.lp = c.take<float>(n_slots * H);
+  p.lsum = c.take<float>((size_t)B * H);
+  p.lse2x = c.take<float>((size_t)B * H);
+  p.ovf = c.take<int>((size_t)B + 1);
+  p.fallback = 0;
+  // phase 1 estimates each head's logsumexp from about 128 tiles (16k keys) per sequence
+  p.sample_stride = s.tps / 128 > 1 ? s.tps / 128 : 1;
   p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
   p.seq_done = c.take<int>((size_t)B);
@@ -296,6 +311,13 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
     sp.opart = w.p.opart;
     sp.out = reinterpret_cast<__nv_bfloat16*>(out);
     sp.H = H; sp.D = d; sp.sch = w.p.sch;
+    sp.lsum = w.p.lsum;
+    sp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
+    sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
+    sp.lse2x = w.p.lse2x;
+    sp.c = c;
+    sp.sms = sms;
+    sp.wait_ns = w.p.wait_ns;
     sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
     sp.ncand = Lk - window > 0 ? Lk - window : 0;
     sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.bnd = w.bnd;

@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
         const float4 v = part[x][d4];
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
+      const float inv = 1.f / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
       __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * d4;
       reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x, acc.y);
       reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z, acc.w);
@@ -64,7 +66,7 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
     return;
   }
   int* meta = p.meta + b * META;
-  const int beta = meta[0];
+  const int beta = meta[0], beta_lo = meta[3];
   const unsigned lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   const float* sc = p.sc + (size_t)b * p.ncand;
@@ -90,22 +92,122 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_col
       const uint32_t bits = __float_as_uint(v[x]);
       const int bin = in_range ? (int)((bits >> 20) & (NBINS - 1)) : -2;
       if (in_range && bin > beta) upmask |= 1u << (j & 31);
-      const bool eq = in_range && bin == beta;
+      const bool eq = in_range && bin >= beta_lo && bin <= beta;  // the band: re-scored exactly
       const unsigned me = __ballot_sync(0xffffffffu, eq);
       if (me) {
         int base = 0;
         const int leader = __ffs(me) - 1;
         if ((int)lane == leader) base = atomicAdd(&meta[4], __popc(me));
         base = __shfl_sync(0xffffffffu, base, leader);
-        if (eq) {
-          const int pos = base + __popc(me & lt_mask);
-          p.bnd[(size_t)b * p.ncand + pos] =
-              ((unsigned long long)bits << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
-        }
+        if (eq) p.bnd[(size_t)b * p.ncand + base + __popc(me & lt_mask)] = (unsigned long long)(uint32_t)j;
       }
     }
     if (upmask) atomicOr(&bm[j0 >> 5], upmask);
   }
+}
+
+// The band keys of every sequence, 128 at a time: their K rows are gathered into shared memory,
+// S^T = K_band Q^T runs on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads), and each thread
+// turns its key's row into the exact score sum_h exp2(s*c - lse2_h) with the exact lse, then into
+// the 64-bit key (score bits << 32 | ~index) the final selection ranks. Persistent CTAs walk the
+// (sequence, tile) pairs of all sequences.
+__global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int H = 64, D = 128, TILE = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;               // [64 heads][128] K-major SW128 (two 64-column blocks)
+  uint8_t* sK = smem + H * D * 2;   // [128 keys][128] K-major SW128
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ __align__(16) float s_nl[H];  // -lse2 of the current sequence
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) { mbar_init(&mma_bar, 1); fence_mbar_init(); }
+  if (warp == 0) { tmem_alloc(&tmem_base, 64); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const float c = p.c;
+  int cur_b = -1;
+  uint32_t phase = 0;
+  bool ok = true;
+  // virtual tile v walks (sequence, tile) pairs in sequence order; b, base_t follow it
+  auto tiles_of = [&](int bb) { return (p.meta[bb * META + 4] + TILE - 1) / TILE; };
+  int b = 0, base_t = 0, nt_b = p.B > 0 ? tiles_of(0) : 0;
+  for (int v = blockIdx.x; ok; v += gridDim.x) {
+    while (b < p.B && v >= base_t + nt_b) {
+      base_t += nt_b;
+      ++b;
+      nt_b = b < p.B ? tiles_of(b) : 0;
+    }
+    if (b >= p.B) break;
+    const int tile = v - base_t;
+    const int n_band = p.meta[b * META + 4];
+    if (b != cur_b) {  // this sequence's query (64 heads) and exact lse
+      const __nv_bfloat16* q = p.qry + (size_t)b * H * D;
+      for (int i = tid; i < H * D / 8; i += 128) {
+        const int row = i / (D / 8), ch = i % (D / 8);
+        cp_async_16(smem_u32(sQ) + (ch / 8) * (H * 128) + sw128_off(row, ch % 8), q + row * D + ch * 8, true);
+      }
+      if (tid < H) s_nl[tid] = -p.lse2x[b * H + tid];
+      cur_b = b;
+    }
+    // gather the K rows of band slots tile*128 .. +127 (zero rows past the end)
+    const int slot = tile * TILE + tid;
+    const bool in = slot < n_band;
+    const int j = in ? (int)(uint32_t)p.bnd[(size_t)b * p.ncand + slot] : 0;
+    const bool valid = in && j >= 0 && j < p.ncand;
+    const __nv_bfloat16* kr = p.kc + ((size_t)b * p.N + (valid ? j : 0)) * D;
+#pragma unroll
+    for (int ch = 0; ch < D / 8; ++ch)
+      cp_async_16(smem_u32(sK) + (ch / 8) * (TILE * 128) + sw128_off(tid, ch % 8), kr + ch * 8, valid);
+    cp_async_commit();
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t IDESC = idesc_bf16(TILE, H, 0, 0);
+      const uint64_t ka = sdesc(smem_u32(sK), 16, 1024), qa = sdesc(smem_u32(sQ), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_bf16(tmem, sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32),
+                  sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32), IDESC, kk > 0);
+      umma_commit(&mma_bar);
+    }
+    bool w_ok = true;
+    if (tid == 0) w_ok = mbar_wait(&mma_bar, phase, p.wait_ns);
+    if (!__syncthreads_and(w_ok)) { if (tid == 0) report_status(p.st, kStatusTimeout, 311); ok = false; break; }
+    phase ^= 1;
+    tc_fence_after();
+    float sa = 0.f, sb = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < H / 32; ++cc) {
+      float sv[32];
+      tmem_ld32(tmem + lane_base + cc * 32, sv);
+      tmem_ld_wait();
+#pragma unroll
+      for (int x = 0; x < 32; x += 2) {
+        float e0, e1;
+        ffma2(e0, e1, sv[x], sv[x + 1], c, c, s_nl[cc * 32 + x], s_nl[cc * 32 + x + 1]);
+        fadd2(sa, sb, sa, sb, fast_exp2(e0), fast_exp2(e1));
+      }
+    }
+    if (in && !valid) report_status(p.st, kStatusBounds, 312);
+    if (in) {
+      const float score = sa + sb;
+      p.bnd[(size_t)b * p.ncand + slot] =
+          ((unsigned long long)__float_as_uint(score) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM and the K tile are reused by the next tile
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 64); }
 }
 
 __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
@@ -245,6 +347,20 @@ cudaError_t launch_select(const SelParams& p, cudaStream_t stream) {
     if (n_collect < 1) n_collect = 1;
     LaunchScope ls("sel_collect", stream);
     e = launch_k(sel_collect_kernel, dim3(n_collect + p.H, p.B), dim3(256), 0, stream, true, p, n_collect);
+  }
+  if (e != cudaSuccess) return e;
+  {
+    static bool configured = false;
+    constexpr int RS_SMEM = 1024 + 64 * 128 * 2 + 128 * 128 * 2;
+    if (!configured) {
+      cudaFuncSetAttribute(sel_rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RS_SMEM);
+      configured = true;
+    }
+    int grid = 2 * (p.sms > 0 ? p.sms : 148);
+    const int max_tiles = p.B * ((p.ncand + 127) / 128);
+    if (grid > max_tiles) grid = max_tiles > 0 ? max_tiles : 1;
+    LaunchScope ls("sel_rescore", stream);
+    e = launch_k(sel_rescore_kernel, dim3(grid), dim3(128), RS_SMEM, stream, true, p);
   }
   if (e != cudaSuccess) return e;
   {

@@ -88,3 +88,18 @@ def test_decode_full_size(hs2, name):
         torch.cuda.synchronize()
         ref = oracle.sparse_attn(qs, g.k, g.v, idx.cpu().numpy(), g.wl.scale)
         assert_out_close(bf16_to_f64(o2).reshape(ref["out"].shape), ref["out"], f"sparse layer {layer}")
+
+
+def test_decode_dominant_key_outside_the_phase1_sample_is_redone_exactly(hs2):
+    """Phase 1 estimates each head's logsumexp from a sample of the tiles (every 2nd tile here).
+    A key that head 0 prefers over all sampled keys by about 2^74 sits in an unsampled tile: its
+    unnormalised probability overflows the sampled reference, the sequence is flagged, and the
+    exact redo (every tile) must give the oracle's output, lse and selection."""
+    B, N, j = 2, 40000, 200  # 313 tiles per sequence: phase 1 takes tiles 0, 2, 4, ...; key 200 is in tile 1
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=N))
+    q0 = bf16_to_f64(to_torch_bf16(g.q[1, 0, 0]))
+    k_dom = 60.0 * q0 / np.linalg.norm(q0)
+    g.k[1, j] = synth.f32_to_bf16_bits(k_dom.astype(np.float32))
+    q, k, v, out, lse, idx = _run_full(hs2, g)
+    ora, st = _check_full(g, out, lse, idx)
+    assert j in set(idx.cpu().numpy()[1, 0].tolist())
