@@ -1,36 +1,40 @@
 // Decode step of the full-attention + selection layer (one query token per sequence, the
 // query at position t = N-1 of an N-token K/V cache), as one persistent kernel.
 //
-// Exact head-summed probabilities need each head's logsumexp over the whole row before any
-// token's score is final, so every tile of the cache is visited twice. The sequences are taken
-// in groups (Sched; by default one group holding all of them); per group:
+// The score of a key is sum_h p_h = sum_h exp(s_h - lse_h): each head's logsumexp over the whole
+// row is needed before any score is final. Instead of a full first pass over K for it, phase 1
+// estimates it from a sample of the tiles, phase 2 streams K and V once against that reference,
+// and the selection is made exact with bounds and a re-score of the few keys near the threshold:
 //
-//   phase 1  K only.  S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads).
-//            The two softmax warpgroups split the heads (32 each); every thread owns one key
-//            lane and keeps, per head, a reference r and a sum l of exp2(s*c - r). r only moves
-//            (with the usual rescale of l) when a value exceeds it by more than 2^64, so the
-//            common step is one FFMA, one MUFU ex2, one FADD and one FMNMX per element. One
-//            cross-lane merge per segment -> partial (m, l) per head.
-//   grid barrier (bounded): every phase-1 partial of the group is written.
-//   phase 2  K again (now from L2) and V. The segment's per-head lse from all partials of its
-//            sequence (the CTA owning the sequence's first tile also writes the caller's lse);
-//            S^T again; p = exp2(s*c - lse2) exactly (no rescaling); the head sum is an
-//            in-thread reduction (the score of the thread's key); P^T (bf16) goes to shared
-//            memory as an MN-major operand and O^T += V^T P^T accumulates in TMEM. The two
-//            warpgroups take alternate tiles. Scores of the older tokens go to a global buffer
-//            and a 2048-bin histogram of their top bits (warp-aggregated shared atomics); the
-//            last CTA to finish a sequence scans its histogram for the bin of the k-th score.
+//   phase 1  every sample_stride-th tile of each sequence (about 128 tiles), K only.
+//            S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads); the two
+//            softmax warpgroups split the heads (32 each); every thread owns one key lane and
+//            keeps, per head, a reference r and a sum l of exp2(s*c - r) (r moves only when a
+//            value exceeds it by 2^64); one reduce-scatter merge per segment -> (m, l) records.
+//   grid barrier (bounded).
+//   phase 2  K and V, each CTA's range backwards. The sequence's sampled lse2' per head from all
+//            its records; S^T again; p' = exp2(s*c - lse2') (no rescaling, p' >= p); the head
+//            sum score' is an in-thread reduction; P'^T (bf16) goes to shared memory as an
+//            MN-major operand and O'^T += V^T P'^T accumulates in TMEM; a warp reduce-scatter of
+//            p' accumulates the per-head totals L'_h = sum_j p'_jh. Scores go to a global buffer
+//            and a 2048-bin histogram of their bits 30..20. The two warpgroups take alternate
+//            tiles.
+//   tail     the last CTA to finish a sequence forms the exact lse = lse2' + log2 L' (out is
+//            sum O' / L' in the combine), and since score = sum_h p'_h / L'_h lies within
+//            [score' / max L', score' / min L'], it turns the bin of the k-th score' into a bin
+//            above which keys are certainly selected and one below which they certainly are
+//            not. select.cu collects the band between them, re-scores it exactly and selects.
 //
-// Phase 2 walks a CTA's range backwards, so the K tiles phase 1 loaded last are re-read first
-// (those still in L2; a group small enough for L2 would re-read all of its K from there).
-// The grid is one CTA per SM, launched cooperatively (all CTAs co-resident). select.cu finishes
-// the step: output combine, collect, final selection.
+// A sequence whose p' reaches 2^64 (a key far more probable than everything sampled) is flagged
+// and redone with every tile (sample_stride 1: the reference is then the exact lse) by a second
+// launch of this kernel, which leaves at once when nothing is flagged.
 //
-// Warp roles (320 threads): warp 0 = TMA producer (Q per segment; K and V tiles through one
-// 5-slot ring, in the order the tensor core consumes them), warp 1 = tcgen05 issuer and TMEM
-// owner, warps 2..5 and 6..9 = softmax warpgroups 0 and 1 (warp w reads TMEM lanes
-// 32*(w%4)..+31). Every wait is bounded; on timeout the kernel records it in the status word
-// and unwinds with its barrier sequence intact.
+// The grid is one CTA per SM, launched cooperatively (all CTAs co-resident). Warp roles
+// (320 threads): warp 0 = TMA producer (Q per segment; K and V tiles through one 5-slot ring,
+// in the order the tensor core consumes them), warp 1 = tcgen05 issuer and TMEM owner,
+// warps 2..5 and 6..9 = softmax warpgroups 0 and 1 (warp w reads TMEM lanes 32*(w%4)..+31).
+// Every wait is bounded; on timeout the kernel records it in the status word and unwinds with
+// its barrier sequence intact.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"

@@ -1,19 +1,22 @@
-// Exact top-k over a per-sequence score vector (decode path), ties to the lower index.
+// Exact top-k of the decode path, ties to the lower index, from the decode kernel's bounded
+// scores (score' with score' / max L' <= score <= score' / min L', see decode.cu).
 //
-//  1. threshold : (done by decode pass 2) from the 2048-bin histogram of score bits 30..20,
-//                 the bin beta that holds the k-th largest score; `above` = number of scores in
-//                 higher bins, `need` = k - above.
-//  2. collect   : every score in a bin above beta is selected outright -- its bit is set in
-//                 the sequence's selection bitmap (one bit per older token, cleared by pass 1);
-//                 scores in bin beta become 64-bit keys (score bits << 32 | ~index): unique, and
-//                 larger key == higher score, then lower index. Extra CTAs of the same launch
-//                 produce the decode output: per (sequence, head), the sum of the per-segment
-//                 output partials of the CTAs whose tile ranges cover the sequence.
-//  3. final     : MSB-first 8-bit radix select of the `need` largest boundary keys (starting at
-//                 the highest bit on which they differ, stopping as soon as the chosen bucket
-//                 holds exactly the remaining need) sets their bits; one pass over the bitmap
-//                 with a block-wide prefix sum writes the chosen indices in ascending order, and
-//                 the forced window (every index of which is larger) is appended.
+//  1. bounds   : (decode kernel, last CTA of a sequence) from the 2048-bin histogram of score'
+//                bits 30..20: bins above b_hi hold keys certainly selected (`above` of them),
+//                bins below b_lo keys certainly not; `need` = k - above are to come from the band
+//                b_lo..b_hi.
+//  2. collect  : every score' above b_hi sets its bit in the sequence's selection bitmap (one bit
+//                per older token, cleared by the decode kernel); band keys are listed by index.
+//                Extra CTAs of the same launch produce the decode output: per (sequence, head),
+//                the sum of the output records of the CTAs covering the sequence, divided by L'.
+//  3. rescore  : the band keys' K rows are gathered and their exact scores computed (tcgen05,
+//                exact lse), as unique 64-bit keys (score bits << 32 | ~index: larger key ==
+//                higher score, then lower index).
+//  4. final    : MSB-first 8-bit radix select of the `need` largest band keys (starting at the
+//                highest bit on which they differ, stopping as soon as the chosen bucket holds
+//                exactly the remaining need) sets their bits; one pass over the bitmap with a
+//                block-wide prefix sum writes the chosen indices in ascending order, and the
+//                forced window (every index of which is larger) is appended.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
