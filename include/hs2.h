@@ -31,8 +31,11 @@
  *    contiguous, 16-byte aligned, owned by the caller. bf16 values are passed as
  *    hs2_bf16 (the 16-bit pattern). Inputs are read only; outputs must not alias inputs.
  *  - `workspace` is caller-owned device scratch of at least the size the matching
- *    *_workspace_bytes query returns. Its first 16 bytes hold the device status word. The
- *    library never allocates, frees or synchronises inside the compute calls.
+ *    *_workspace_bytes query returns. Its first 256 bytes are the status block: the device
+ *    status word (first 16 bytes) and the counters of the decode kernel's grid barrier. Zero-
+ *    fill a workspace before its first use (cudaMemset, torch.zeros); every call leaves it
+ *    ready for the next one. After a device-side error, hs2_clear_device_status re-arms it.
+ *    The library never allocates, frees or synchronises inside the compute calls.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *    Arguments are validated on the host before anything is launched; a non-zero return
  *    means nothing was launched (HS2_ERR_CUDA: a launch failed).
@@ -156,7 +159,8 @@ HS2_API hs2_status hs2_bridge_kv_proj(const hs2_bf16* Hs, int T, int hidden, con
  * ---------------------------------------------------------------------------------
  * hs2_read_device_status: waits for `stream`, reads the status word of `workspace` and
  * returns HS2_OK, HS2_ERR_DEVICE_TIMEOUT or HS2_ERR_DEVICE_BOUNDS (HS2_ERR_CUDA if the
- * read failed). hs2_clear_device_status: resets the word (asynchronously, on `stream`).
+ * read failed). hs2_clear_device_status: zeroes the status block (the word and the grid
+ * barrier's counters; asynchronously, on `stream`).
  * hs2_set_wait_limit_ns: wall-time bound of every device-side wait of later launches
  * (default 2 s, or the environment variable HS2_WAIT_LIMIT_MS at first use).
  * hs2_selftest_wait_timeout: launches one kernel whose bounded wait is on a barrier that

@@ -85,6 +85,9 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
   m = mx;
 }
 
+// the first phase-1 (sampled) tile at or after local tile lt
+__device__ __forceinline__ int first_sample(int lt, int st) { return (lt + st - 1) / st * st; }
+
 template <int H, int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dec_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -118,6 +121,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const Sched S = p.sch;
   const long long limit = p.wait_ns;
   const uint32_t tS = 0, tO = 2 * H;  // TMEM columns: S buffers 0..2H-1, O^T 2H..3H-1
+  // launched as a programmatic dependent: nothing before this point touches global memory
+  griddep_wait();
   // the exact redo runs only if the sampled launch before it flagged a sequence (every CTA reads
   // the same final count, so the whole grid leaves together, before any barrier)
   if (p.fallback && *(volatile const int*)&p.ovf[p.B] == 0) return;
@@ -142,7 +147,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -175,10 +179,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
           if (skip_seq(b)) { t = seg_end; continue; }
           if (!load_q(b)) { ok = false; break; }
-          for (; t < seg_end; ++t) {
-            const long long lt = t - (long long)b * S.tps;
-            if (lt % p.sample_stride == 0 && !load_tile(&tmK, (int)lt, b, keep)) { ok = false; break; }
-          }
+          const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
+          for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi && ok; lt += st)
+            if (!load_tile(&tmK, lt, b, keep)) ok = false;
+          t = seg_end;
         }
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: descending
           const int b = (int)(t / S.tps);
@@ -254,8 +258,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
           if (skip_seq(b)) { t = seg_end; continue; }
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
-          for (; t < seg_end; ++t)
-            if ((t - (long long)b * S.tps) % p.sample_stride == 0 && !issue_s(ri++)) { ok = false; break; }
+          const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
+          for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi && ok; lt += st)
+            if (!issue_s(ri++)) ok = false;
+          t = seg_end;
           if (!ok) break;
           umma_commit(&q_empty);
           ++nq;
@@ -326,8 +332,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float r[HW], l[HW];
 #pragma unroll
         for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
-        for (; t < seg_end; ++t) {
-          if ((t - (long long)b * S.tps) % p.sample_stride != 0) continue;
+        const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
+        for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi; lt += st) {
           const uint32_t jt = js++;
           ++n1;
           if (!ok) continue;
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[buf]);
-          const bool valid = (t - (long long)b * S.tps) * TILE + row < p.N;
+          const bool valid = lt * TILE + row < p.N;
           if (first) {
             // a lane's first key of the segment sets its references (invalid lanes only occur in
             // a sequence's partial last tile, which then is the segment's last sampled tile)
@@ -375,6 +381,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int h = 0; h < HW; ++h) l[h] += fast_exp2(v[h]);
           }
         }
+        t = seg_end;
         // merge the 128 lanes of each warpgroup. Within a warp a reduce-scatter: at each step a
         // lane keeps half of its heads and merges in its partner's copy of that half, so after
         // 16 + 8 + 4 + 2 + 1 exchanges lane i holds head i of the warpgroup's 32. Then the 4
@@ -406,23 +413,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       ri += n1;  // the phase-1 K items of the ring
       // ---------------------------------------------------------------- grid barrier
+      // gbar[0] counts arrivals over the step's launches: zero when the sampled launch starts (a
+      // zero-filled workspace, then re-armed by the collect kernel after both launches)
       named_bar(3, 256);
       if (all_tid == 0) {
         __threadfence();
-        atomicAdd(p.gbar, 1u);
-        const unsigned target = (unsigned)S.G * (unsigned)(g + 1);
+        const unsigned target = (unsigned)S.G * (unsigned)(g + 1 + (p.fallback ? S.n_groups : 0));
+        const unsigned arrived = atomicAdd(&p.gbar[0], 1u);
+        if (arrived >= target) {  // a count left over: the workspace was not zero-filled
+          abort_flag = 1;
+          report_status(p.st, kStatusBounds, 231);
+        }
         const long long tw = globaltimer_ns();
-        while (*(volatile unsigned*)p.gbar < target) {
-          if (abort_flag) break;
+        while (!abort_flag && *(volatile unsigned*)&p.gbar[0] < target) {
           if (globaltimer_ns() - tw > limit) {
             abort_flag = 1;
             report_status(p.st, kStatusTimeout, 230);
-            break;
           }
         }
         __threadfence();
       }
       named_bar(3, 256);
+      // every CTA of this grid is resident: the next grid on the stream may start launching
+      // (earlier, its CTAs could take SMs this grid still needs)
+      if (g == 0) griddep_launch_dependents();
       if (abort_flag) ok = false;
       // ---------------------------------------------------------------- phase 2
       for (long long t = t1 - 1; t >= t0;) {
@@ -713,25 +727,27 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
   }
   // the sampled launch, then the exact redo of any sequence it flagged (normally none: the redo's
   // CTAs read the flag count and leave at once). Every CTA waits for all others at the grid
-  // barrier, so both launches are cooperative.
+  // barrier, so both launches are cooperative; both are also programmatic dependents of the
+  // work before them (their CTAs wait in griddepcontrol.wait), so the launch overlaps it.
   for (int pass = 0; pass < 2; ++pass) {
     DecParams q = p;
     if (pass == 1) {
       q.fallback = 1;
       q.sample_stride = 1;
     }
-    cudaError_t e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned), stream);
-    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.sch.G);
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = fused_smem_bytes(H, D);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
+    cudaError_t e;
     {
       LaunchScope ls(pass == 0 ? "dec_fused" : "dec_redo", stream);
       e = cudaLaunchKernelEx(&cfg, dec_fused_kernel<H, D>, tmK, tmV, tmQ, q);

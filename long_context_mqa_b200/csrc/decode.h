@@ -28,7 +28,8 @@ struct DecParams {
   int words;               // ceil((N - W) / 32)
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
-  unsigned* gbar;          // grid-barrier arrivals (zeroed before every launch)
+  unsigned* gbar;          // grid-barrier arrivals: zero when a step starts; the sampled launch
+                           // counts to G per group, the redo on from there (the collect kernel re-arms it)
   int sample_stride;       // phase 1 takes every sample_stride-th tile of each sequence
   float* lp;               // [B*cmax][H] per-(sequence, CTA) sums of p' = exp2(s*c - lse2')
   float* lsum;             // [B][H] their totals L'_h (the output is sum(O') / L')
@@ -70,6 +71,7 @@ struct SelParams {
   const float* lse2x;            // [B][H] exact lse, log2 units
   float c;                       // scale * log2(e)
   int sms;
+  unsigned* gbar;                // the decode kernel's grid-barrier counters, re-armed here
   long long wait_ns;             // bound of the re-score kernel's wait for its MMA
 };
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);

@@ -139,7 +139,8 @@ LaunchScope::~LaunchScope() {
 // ------------------------------------------------------------------------------------------
 // workspace carving
 // ------------------------------------------------------------------------------------------
-constexpr size_t kStatusBytes = 256;
+constexpr size_t kStatusBytes = 256;   // status word (16 bytes) + the decode grid barrier's counter
+constexpr size_t kBarrierOffset = 64;
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Carve {
@@ -189,7 +190,8 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   const int ncand = N - W > 0 ? N - W : 0;
   Carve c{(uint8_t*)ws, 0};
   p.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
-  p.gbar = c.take<unsigned>(1);
+  // the grid-barrier counter lives in the status block, so clearing the status re-arms it
+  p.gbar = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(p.st) + kBarrierOffset);
   p.ml = c.take<float>(n_slots * 2 * H);
   p.opart = c.take<float>(n_slots * H * D);
   p.lp = c.take<float>(n_slots * H);
@@ -315,6 +317,7 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
     sp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
     sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
     sp.lse2x = w.p.lse2x;
+    sp.gbar = w.p.gbar;
     sp.c = c;
     sp.sms = sms;
     sp.wait_ns = w.p.wait_ns;
@@ -397,7 +400,8 @@ hs2_status hs2_read_device_status(const void* workspace, hs2_stream stream) {
 
 hs2_status hs2_clear_device_status(void* workspace, hs2_stream stream) {
   if (!workspace) return HS2_ERR_WORKSPACE;
-  if (cudaMemsetAsync(workspace, 0, sizeof(DevStatus), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // the whole status block: the status word and the decode grid barrier's counters
+  if (cudaMemsetAsync(workspace, 0, kStatusBytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return HS2_ERR_CUDA;
   return HS2_OK;
 }

@@ -31,6 +31,8 @@ constexpr int NT = 1024;
 __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_collect) {
   griddep_wait();
   griddep_launch_dependents();
+  // both decode launches are complete: re-arm their grid barrier for the next step
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *(volatile unsigned*)p.gbar = 0u;
   const int b = blockIdx.y;
   if ((int)blockIdx.x >= n_collect) {
     // the decode kernel's CTAs c_lo..c_hi (of sequence b's group) left one partial each, in
