@@ -88,25 +88,32 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   if (warp == 0) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
   bool bad = false;
 
-  // thread `tid` gathers key row `tid` of tile t (K tile K-major; the V tile is read MN-major)
+  // gathers the key rows of tile t (K tile K-major; the V tile is read MN-major). Thread `tid`
+  // reads the index of row `tid`; the copies are coalesced: LPR consecutive lanes fetch the
+  // 16-byte chunks of one row (a whole row per group of lanes, RPS rows per warp step), the
+  // row's index passed by shuffle from the lane that read it.
   auto gather = [&](int t) {
+    constexpr int LPR = D * 2 / 16, RPS = 32 / LPR;
     const int slot = slot0 + t * TILE + tid;
     int j = -1;
     if (slot < slot1) j = idx_row[slot];
     const bool valid = j >= 0 && j < p.Lk;
     if (j != -1 && !valid) bad = true;
-    const __nv_bfloat16* kr = Kb + (size_t)(valid ? j : 0) * D;
-    const __nv_bfloat16* vr = Vb + (size_t)(valid ? j : 0) * D;
-    const uint32_t kd = smem_u32(sK), vd = smem_u32(sV);
-#pragma unroll
-    for (int ch = 0; ch < D / 8; ++ch) {
-      const uint32_t off = (ch / 8) * (TILE * 128) + sw128_off(tid, ch % 8);
-      cp_async_16(kd + off, kr + ch * 8, valid);
-      cp_async_16(vd + off, vr + ch * 8, valid);
-    }
-    cp_async_commit();
+    const int jv = valid ? j : -1;
     const unsigned m = __ballot_sync(0xffffffffu, valid);
     if (lane == 0) vmask[warp] = m;
+    const uint32_t kd = smem_u32(sK), vd = smem_u32(sV);
+    const int sub = lane / LPR, ch = lane % LPR;
+#pragma unroll
+    for (int it = 0; it < 32 / RPS; ++it) {
+      const int rr = it * RPS + sub;  // row within this warp's 32
+      const int jr = __shfl_sync(0xffffffffu, jv, rr);
+      const uint32_t off = (ch / 8) * (TILE * 128) + sw128_off(warp * 32 + rr, ch % 8);
+      const size_t src = (size_t)(jr >= 0 ? jr : 0) * D + ch * 8;
+      cp_async_16(kd + off, Kb + src, jr >= 0);
+      cp_async_16(vd + off, Vb + src, jr >= 0);
+    }
+    cp_async_commit();
   };
 
   const float c = p.c;
@@ -145,19 +152,20 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     phase ^= 1;
     if (!ok) break;
     tc_fence_after();
-    // ---- row max of the valid keys (every thread runs the warp-collective loads)
+    // ---- the row's 128 logits in registers (warp-collective loads, one wait); max of the valid
+    float sv[4][32];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + tS + cc * 32, sv[cc]);
+    tmem_ld_wait();
     float rmax = -INFINITY;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      float v[32];
-      tmem_ld32(tmem + lane_base + tS + cc * 32, v);
-      tmem_ld_wait();
       if (!all_valid) {
         const unsigned mk = vmask[cc];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) v[x] = (mk >> x) & 1u ? v[x] : -INFINITY;
+        for (int x = 0; x < 32; ++x) sv[cc][x] = (mk >> x) & 1u ? sv[cc][x] : -INFINITY;
       }
-      rmax = fmaxf(rmax, max32(v));
+      rmax = fmaxf(rmax, max32(sv[cc]));
     }
     const float mt = rmax * c;
     const bool raise = mt > -INFINITY && (m_run == -INFINITY || mt > m_run + RESCALE_SLACK);
@@ -181,9 +189,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     float la = 0.f, lb = 0.f;
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      float v[32];
-      tmem_ld32(tmem + lane_base + tS + cc * 32, v);
-      tmem_ld_wait();
+      const float* v = sv[cc];
       const unsigned mk = all_valid ? 0xFFFFFFFFu : vmask[cc];
       uint32_t pk[16];
 #pragma unroll
