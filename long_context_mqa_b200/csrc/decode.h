@@ -90,7 +90,7 @@ struct SpParams {
   long long wait_ns;
   DevStatus* st;
 };
-size_t sparse_smem_bytes(int H, int D);
+size_t sparse_smem_bytes(int H, int D, int nsplit);
 cudaError_t launch_sparse(const SpParams& p, int H, int D, cudaStream_t stream);
 }  // namespace sparse
 

@@ -9,14 +9,16 @@
 //                            in TMEM only when the max grows by more than 2^8
 //   O += P V_sel             tcgen05, M = 64 heads, N = d, P (bf16) K-major in shared memory
 // TMEM rows of an M = 64 accumulator sit in lanes 0..15 of each 32-lane quarter, so thread
-// (warp q, lane l < 16) owns head row 16 q + l. Two CTAs share an SM, so one CTA's gathers
-// overlap the other's math. With one split the CTA writes the final bf16 output (and lse). With
-// few query rows (decode) a row's index list is split over a cluster of CTAs; head h of the row
-// is merged by cluster rank h % n: after a first cluster barrier (every CTA is done with its K/V
-// tiles) each CTA stores its unnormalised O rows into their owners' shared memory and its
-// per-head (max, sum) into every CTA's, and after a second barrier each CTA merges its heads
-// from local shared memory. Launched as a programmatic dependent: the prologue overlaps the
-// previous kernel's tail and every global read waits for it.
+// (warp q, lane l < 16) owns head row 16 q + l; lane l + 16 takes over the upper half of that
+// row's keys for the softmax. Two CTAs share an SM, so one CTA's gathers overlap the other's
+// math. With one split the CTA writes the final bf16 output (and lse). With few query rows
+// (decode) a row's index list is split over a cluster of CTAs; head h of the row is merged by
+// cluster rank h % n: as soon as its own tiles are done (and every CTA of the cluster has
+// started: a cluster barrier arrived at the start, waited on here) each CTA stores its
+// unnormalised O rows into their owners' exchange buffers and its per-head (max, sum) into
+// every CTA's, and after a second cluster barrier each CTA merges its heads from local shared
+// memory. Launched as a programmatic dependent: the prologue overlaps the previous kernel's
+// tail and every global read waits for it.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -38,7 +40,15 @@ struct SpLayout {
   static constexpr int OFF_K = ((Q_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_V = OFF_K + KT_BYTES;
   static constexpr int OFF_P = OFF_V + KT_BYTES;
-  static constexpr int BYTES = OFF_P + P_BYTES + 1024;
+  static constexpr int OFF_X = OFF_P + P_BYTES;  // split-merge exchange buffers (clusters only)
+  // xO[n][HPR][D] + xm[n][MH] + xl[n][MH] floats, HPR = ceil(H / n) heads per cluster rank
+  __host__ __device__ static constexpr int x_bytes(int n) { return n > 1 ? (n * ((H + n - 1) / n) * D + 2 * n * MH) * 4 : 0; }
+  __host__ __device__ static constexpr int bytes(int n) { return OFF_X + x_bytes(n) + 1024; }
+  static constexpr int max_bytes() {
+    int m = bytes(1);
+    for (int n = 2; n <= 16; ++n) m = bytes(n) > m ? bytes(n) : m;
+    return m;
+  }
 };
 
 template <int H, int D>
@@ -67,13 +77,17 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   const __nv_bfloat16* Kb = p.K + (size_t)b * p.Lk * D;
   const __nv_bfloat16* Vb = p.V + (size_t)b * p.Lk * D;
   const uint32_t tS = 0, tO = 128;
-  const int head = warp * 16 + lane;        // the head row this thread owns (lanes 0..15)
-  const bool owns = lane < 16 && head < H;  // a real head
+  const int prow = warp * 16 + (lane & 15);  // the row this lane's pair works on
+  const int head = warp * 16 + lane;         // the head row this thread owns (lanes 0..15)
+  const bool owns = lane < 16 && head < H;   // a real head, written out by this lane
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   // every input may come from the kernels before this one on the stream
   griddep_wait();
   griddep_launch_dependents();
+  // first half of the cluster barrier that makes the other CTAs' shared memory safe to write
+  // (every CTA of the cluster has started); its wait comes just before the first remote store
+  if (p.nsplit > 1) cluster_arrive();
   // ---- query -> shared (K-major, 128B swizzle): rows 0..H-1 by cp.async, padding rows zero
   {
     const __nv_bfloat16* q = p.Q + (size_t)r * H * D;
@@ -152,21 +166,35 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     phase ^= 1;
     if (!ok) break;
     tc_fence_after();
-    // ---- the row's 128 logits in registers (warp-collective loads, one wait); max of the valid
-    float sv[4][32];
+    // ---- the row's 128 logits (warp-collective loads, one wait). Lanes 0..15 hold the head
+    // rows; lane l + 16 takes keys 64..127 of lane l's row (by shuffle), lane l keeps keys 0..63,
+    // so every lane exponentiates 64 keys. Both lanes of a pair keep the same running max.
+    const bool upper = lane >= 16;
+    float sv[2][32];
+    {
+      float s4[4][32];
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + tS + cc * 32, sv[cc]);
-    tmem_ld_wait();
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + tS + cc * 32, s4[cc]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float hi = __shfl_xor_sync(0xffffffffu, s4[2 + h2][x], 16);
+          sv[h2][x] = upper ? hi : s4[h2][x];
+        }
+    }
     float rmax = -INFINITY;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int h2 = 0; h2 < 2; ++h2) {
       if (!all_valid) {
-        const unsigned mk = vmask[cc];
+        const unsigned mk = vmask[(upper ? 2 : 0) + h2];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) sv[cc][x] = (mk >> x) & 1u ? sv[cc][x] : -INFINITY;
+        for (int x = 0; x < 32; ++x) sv[h2][x] = (mk >> x) & 1u ? sv[h2][x] : -INFINITY;
       }
-      rmax = fmaxf(rmax, max32(sv[cc]));
+      rmax = fmaxf(rmax, max32(sv[h2]));
     }
+    rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 16));
     const float mt = rmax * c;
     const bool raise = mt > -INFINITY && (m_run == -INFINITY || mt > m_run + RESCALE_SLACK);
     const float alpha = raise ? (m_run == -INFINITY ? 0.f : fast_exp2(m_run - mt)) : 1.f;
@@ -186,11 +214,11 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     }
     // ---- probabilities -> P row (K-major: row = head, K = the 128 keys)
     const float negm = m_run == -INFINITY ? 0.f : -m_run;
-    float la = 0.f, lb = 0.f;
+    float la = 0.f, lb = 0.f;  // this lane's half of the row sum (l_run is the half's running sum)
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const float* v = sv[cc];
-      const unsigned mk = all_valid ? 0xFFFFFFFFu : vmask[cc];
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float* v = sv[h2];
+      const unsigned mk = all_valid ? 0xFFFFFFFFu : vmask[(upper ? 2 : 0) + h2];
       uint32_t pk[16];
 #pragma unroll
       for (int x = 0; x < 32; x += 2) {
@@ -201,11 +229,11 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
         fadd2(la, lb, la, lb, p0, p1);
         pk[x / 2] = pack_bf16x2(p0, p1);
       }
-      if (lane < 16) {
-        const uint32_t blk = smem_u32(sP) + (cc / 2) * (MH * 128);
+      {  // keys 0..63 of the row in the first 128-byte block, keys 64..127 in the second
+        const uint32_t blk = smem_u32(sP) + (upper ? MH * 128 : 0);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          st_shared_v4(blk + sw128_off(head, (cc % 2) * 4 + q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          st_shared_v4(blk + sw128_off(prow, h2 * 4 + q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
     }
     l_run += la + lb;
@@ -238,6 +266,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   if (__syncthreads_or(bad) && tid == 0) report_status(p.st, kStatusBounds, 403);
   // ---- epilogue
   const bool have = ntiles > 0 && ok;  // block-uniform
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);  // the row's sum: both halves
   if (p.nsplit == 1) {
     if (have) {
 #pragma unroll
@@ -262,35 +291,37 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
     return;
   }
-  // cluster merge. Exchange buffers in the (now free) K/V tile region of every CTA:
+  // cluster merge. Exchange buffers in their own shared-memory region of every CTA:
   //   xO[s][k][D]  O row of head rank + k*n from split s      (HPR = ceil(H / n) heads per rank)
   //   xm[s][MH], xl[s][MH]  split s's max (log2 units) and sum per head
   const int n = p.nsplit;
   const uint32_t rank = cluster_ctarank();
   const int HPR = (H + n - 1) / n;
-  float* xO = reinterpret_cast<float*>(sK);
+  float* xO = reinterpret_cast<float*>(smem + Lay::OFF_X);
   float* xm = xO + (size_t)n * HPR * D;
   float* xl = xm + n * MH;
-  // (n * HPR * D + 2 * n * MH) floats <= (H + n) * D + 32 * MH floats fit in the 2 tile buffers
-  static_assert((H + 16) * D * 4 + 32 * MH * 4 <= 2 * Lay::KT_BYTES, "exchange buffers fit");
-  cluster_sync_all();  // every CTA of the row is done with its K and V tiles
   {
+    // this CTA's O rows (unnormalised), one TMEM wait, while the cluster barrier completes
+    float o[D / 32][32];
+    if (have) {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_base + tO + cc * 32, o[cc]);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o[cc][x] = 0.f;
+    }
+    cluster_wait();  // every CTA of the cluster has started: its shared memory can be written
     const int owner = head % n, k = head / n;
     const uint32_t o_dst = dsmem_addr(smem_u32(xO + ((size_t)split * HPR + k) * D), owner);
+    if (owns) {
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      float o[32];
-      if (have) {
-        tmem_ld32(tmem + lane_base + tO + cc * 32, o);
-        tmem_ld_wait();
-      } else {
+      for (int cc = 0; cc < D / 32; ++cc)
 #pragma unroll
-        for (int x = 0; x < 32; ++x) o[x] = 0.f;
-      }
-      if (owns) {
-#pragma unroll
-        for (int x = 0; x < 8; ++x) st_dsmem_v4(o_dst + (cc * 32 + 4 * x) * 4, o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
-      }
+        for (int x = 0; x < 8; ++x)
+          st_dsmem_v4(o_dst + (cc * 32 + 4 * x) * 4, o[cc][4 * x], o[cc][4 * x + 1], o[cc][4 * x + 2], o[cc][4 * x + 3]);
     }
     if (owns) {
       const float mv = l_run > 0.f && have ? m_run : -INFINITY, lv = have ? l_run : 0.f;
@@ -342,9 +373,9 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   }
 }
 
-size_t sparse_smem_bytes(int H, int D) {
-  if (H == 64 && D == 128) return SpLayout<64, 128>::BYTES;
-  if (H == 16 && D == 64) return SpLayout<16, 64>::BYTES;
+size_t sparse_smem_bytes(int H, int D, int nsplit) {
+  if (H == 64 && D == 128) return SpLayout<64, 128>::bytes(nsplit);
+  if (H == 16 && D == 64) return SpLayout<16, 64>::bytes(nsplit);
   return 0;
 }
 
@@ -352,7 +383,8 @@ template <int H, int D>
 static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SpLayout<H, D>::BYTES);
+    cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         SpLayout<H, D>::max_bytes());
     cudaFuncSetAttribute(sparse_attn_kernel<H, D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     configured = true;
   }
@@ -360,7 +392,7 @@ static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, p.nsplit);
   cfg.blockDim = dim3(NT);
-  cfg.dynamicSmemBytes = SpLayout<H, D>::BYTES;
+  cfg.dynamicSmemBytes = SpLayout<H, D>::bytes(p.nsplit);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of one row form a cluster

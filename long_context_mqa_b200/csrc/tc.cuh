@@ -171,6 +171,9 @@ __device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float a) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// the two halves of a cluster barrier (every thread of every CTA arrives once before waiting)
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Ampere-style 16-byte asynchronous copy (used for row gathers by index).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {
