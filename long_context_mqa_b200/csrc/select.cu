@@ -160,15 +160,24 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
       if (tid < H) s_nl[tid] = -p.lse2x[b * H + tid];
       cur_b = b;
     }
-    // gather the K rows of band slots tile*128 .. +127 (zero rows past the end)
+    // gather the K rows of band slots tile*128 .. +127 (zero rows past the end). Thread `tid`
+    // reads the index of row `tid`; the copies are coalesced, 16 lanes per row (the whole
+    // 256-byte row), the row's index passed by shuffle
     const int slot = tile * TILE + tid;
     const bool in = slot < n_band;
     const int j = in ? (int)(uint32_t)p.bnd[(size_t)b * p.ncand + slot] : 0;
     const bool valid = in && j >= 0 && j < p.ncand;
-    const __nv_bfloat16* kr = p.kc + ((size_t)b * p.N + (valid ? j : 0)) * D;
+    {
+      const __nv_bfloat16* kb = p.kc + (size_t)b * p.N * D;
+      const int jv = valid ? j : -1, sub = lane >> 4, ch = lane & 15;
 #pragma unroll
-    for (int ch = 0; ch < D / 8; ++ch)
-      cp_async_16(smem_u32(sK) + (ch / 8) * (TILE * 128) + sw128_off(tid, ch % 8), kr + ch * 8, valid);
+      for (int it = 0; it < 16; ++it) {
+        const int rr = 2 * it + sub;  // row within this warp's 32
+        const int jr = __shfl_sync(0xffffffffu, jv, rr);
+        cp_async_16(smem_u32(sK) + (ch / 8) * (TILE * 128) + sw128_off(warp * 32 + rr, ch % 8),
+                    kb + (size_t)(jr >= 0 ? jr : 0) * D + ch * 8, jr >= 0);
+      }
+    }
     cp_async_commit();
     cp_async_wait_all();
     fence_async_smem();
@@ -218,6 +227,8 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
 __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int KPT = 4;  // band keys held in registers per thread (bands up to NT * KPT keys)
+  constexpr int WPT = 8;  // bitmap words per thread per round of the ordered write-out
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   __shared__ unsigned dh[256];
   __shared__ unsigned long long s_prefix, s_mask, s_and, s_or;
@@ -229,11 +240,25 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   const unsigned long long* bnd = p.bnd + (size_t)b * p.ncand;
   unsigned* bm = p.bitmap + (size_t)b * p.words;
   if (need > 0 && n_bnd > 0) {
+    // the band keys, read once into registers when they fit (else every pass reads them again)
+    const bool in_regs = n_bnd <= NT * KPT;
+    unsigned long long kr[KPT];
+#pragma unroll
+    for (int x = 0; x < KPT; ++x) kr[x] = in_regs && tid + x * NT < n_bnd ? bnd[tid + x * NT] : 0ull;
+    auto visit = [&](auto&& f) {
+      if (in_regs) {
+#pragma unroll
+        for (int x = 0; x < KPT; ++x)
+          if (tid + x * NT < n_bnd) f(kr[x]);
+      } else {
+        for (int i = tid; i < n_bnd; i += NT) f(bnd[i]);
+      }
+    };
     // bits on which every boundary key agrees need no pass: start at the highest differing bit
     if (tid == 0) { s_and = ~0ull; s_or = 0ull; s_need = need; s_exact = 0; }
     __syncthreads();
     unsigned long long a_loc = ~0ull, o_loc = 0ull;
-    for (int i = tid; i < n_bnd; i += NT) { const unsigned long long key = bnd[i]; a_loc &= key; o_loc |= key; }
+    visit([&](unsigned long long key) { a_loc &= key; o_loc |= key; });
     for (int o = 16; o > 0; o >>= 1) {
       a_loc &= __shfl_xor_sync(0xffffffffu, a_loc, o);
       o_loc |= __shfl_xor_sync(0xffffffffu, o_loc, o);
@@ -254,10 +279,9 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
       for (int i = tid; i < 256; i += NT) dh[i] = 0;
       __syncthreads();
       const unsigned long long prefix = s_prefix, mask = s_mask;
-      for (int i = tid; i < n_bnd; i += NT) {
-        const unsigned long long key = bnd[i];
+      visit([&](unsigned long long key) {
         if ((key & mask) == prefix) atomicAdd(&dh[(key >> shift) & 255u], 1u);
-      }
+      });
       __syncthreads();
       if (w == 0) {
         // lane l owns digits 255-8l .. 248-8l (descending)
@@ -291,50 +315,58 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
     }
     // keys whose masked prefix is >= s_prefix are exactly the `need` largest boundary entries
     const unsigned long long thr = s_prefix, fmask = s_mask;
-    for (int i = tid; i < n_bnd; i += NT) {
-      const unsigned long long key = bnd[i];
+    visit([&](unsigned long long key) {
       if ((key & fmask) >= thr) {
         const uint32_t j = 0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull);
         atomicOr(&bm[j >> 5], 1u << (j & 31));
       }
-    }
+    });
   }
   __syncthreads();
-  // the bitmap in order: each thread owns a contiguous run of words; block-wide exclusive scan
-  const int per = (p.words + NT - 1) / NT;
-  const int w0 = tid * per, w1 = w0 + per < p.words ? w0 + per : p.words;
-  unsigned cnt = 0;
-  for (int i = w0; i < w1; ++i) cnt += __popc(__ldcg(&bm[i]));
-  unsigned incl = cnt;
+  // the bitmap in order, in rounds of NT * WPT words: each thread owns WPT consecutive words
+  // (loaded together), a block-wide exclusive scan of their counts gives its output position
+  int32_t* out = p.idx + (size_t)b * p.S;
+  unsigned done = 0;  // chosen indices written in earlier rounds
+  for (int base = 0; base < p.words; base += NT * WPT) {
+    const int w0 = base + tid * WPT;
+    unsigned wv[WPT], cnt = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) wsum[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    unsigned t = wsum[lane];
+    for (int x = 0; x < WPT; ++x) wv[x] = w0 + x < p.words ? __ldcg(&bm[w0 + x]) : 0u;
+#pragma unroll
+    for (int x = 0; x < WPT; ++x) cnt += __popc(wv[x]);
+    unsigned incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const unsigned n = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += n;
+      const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
     }
-    wsum[lane] = t;  // inclusive over warps
-  }
-  __syncthreads();
-  const unsigned total_top = wsum[31];
-  unsigned pos = incl - cnt + (w > 0 ? wsum[w - 1] : 0u);
-  int32_t* out = p.idx + (size_t)b * p.S;
-  for (int i = w0; i < w1; ++i) {
-    unsigned word = __ldcg(&bm[i]);
-    while (word) {
-      const int bit = __ffs(word) - 1;
-      word &= word - 1;
-      if (pos < (unsigned)p.S) out[pos] = i * 32 + bit;
-      ++pos;
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      unsigned t = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned n = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += n;
+      }
+      wsum[lane] = t;  // inclusive over warps
     }
+    __syncthreads();
+    unsigned pos = done + incl - cnt + (w > 0 ? wsum[w - 1] : 0u);
+#pragma unroll
+    for (int x = 0; x < WPT; ++x) {
+      unsigned word = wv[x];
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        if (pos < (unsigned)p.S) out[pos] = (w0 + x) * 32 + bit;
+        ++pos;
+      }
+    }
+    done += wsum[31];
+    __syncthreads();  // wsum is rewritten by the next round
   }
+  const unsigned total_top = done;
   const int wlen = p.N < p.W ? p.N : p.W;
   const int expect_top = p.ncand < p.K ? p.ncand : p.K;
   if (tid == 0 && (int)total_top != expect_top) report_status(p.st, kStatusBounds, 302);
