@@ -25,7 +25,7 @@ struct DecParams {
   unsigned* hist;          // [B][2048] histogram of score bits 30..20
   int* seq_done;           // [B] CTAs done with each sequence's histogram
   unsigned* bitmap;        // [B][words] selection bitmap of the older tokens (cleared here)
-  int words;               // ceil((N - W) / 32)
+  int words;               // ceil((N - W) / 32) rounded up to a multiple of 8 (32-byte rows)
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
   unsigned* gbar;          // grid-barrier arrivals: zero when a step starts; the sampled launch

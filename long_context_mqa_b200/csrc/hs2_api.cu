@@ -207,7 +207,7 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   w.meta = c.take<int>((size_t)B * sel::META);
   p.meta = w.meta;
   p.K_sel = K;
-  p.words = (ncand + 31) / 32;
+  p.words = ((ncand + 31) / 32 + 7) / 8 * 8;  // rows of 32-byte multiples (vector loads)
   p.bitmap = c.take<unsigned>((size_t)B * (p.words > 0 ? p.words : 1));
   w.bnd = c.take<unsigned long long>((size_t)B * (ncand > 0 ? ncand : 1));
   w.bytes = c.off;

@@ -324,14 +324,21 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   }
   __syncthreads();
   // the bitmap in order, in rounds of NT * WPT words: each thread owns WPT consecutive words
-  // (loaded together), a block-wide exclusive scan of their counts gives its output position
+  // (two 16-byte loads: the bitmap's row stride is a multiple of 8 words), a block-wide
+  // exclusive scan of their counts gives its output position
   int32_t* out = p.idx + (size_t)b * p.S;
   unsigned done = 0;  // chosen indices written in earlier rounds
   for (int base = 0; base < p.words; base += NT * WPT) {
     const int w0 = base + tid * WPT;
     unsigned wv[WPT], cnt = 0;
+    if (w0 < p.words) {
+      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(bm + w0));
+      const uint4 c4 = __ldcg(reinterpret_cast<const uint4*>(bm + w0 + 4));
+      wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w; wv[4] = c4.x; wv[5] = c4.y; wv[6] = c4.z; wv[7] = c4.w;
+    } else {
 #pragma unroll
-    for (int x = 0; x < WPT; ++x) wv[x] = w0 + x < p.words ? __ldcg(&bm[w0 + x]) : 0u;
+      for (int x = 0; x < WPT; ++x) wv[x] = 0u;
+    }
 #pragma unroll
     for (int x = 0; x < WPT; ++x) cnt += __popc(wv[x]);
     unsigned incl = cnt;
