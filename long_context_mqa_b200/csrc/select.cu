@@ -6,9 +6,8 @@
 //                bins below b_lo keys certainly not; `need` = k - above are to come from the band
 //                b_lo..b_hi.
 //  2. collect  : every score' above b_hi sets its bit in the sequence's selection bitmap (one bit
-//                per older token, cleared by the decode kernel); band keys are listed by index.
-//                Extra CTAs of the same launch produce the decode output: per (sequence, head),
-//                the sum of the output records of the CTAs covering the sequence, divided by L'.
+//                per older token, cleared by the decode kernel); band keys are listed by index
+//                (one list-counter update per warp).
 //  3. rescore  : the band keys' K rows are gathered and their exact scores computed (tcgen05,
 //                exact lse), as unique 64-bit keys (score bits << 32 | ~index: larger key ==
 //                higher score, then lower index).
@@ -16,7 +15,10 @@
 //                highest bit on which they differ, stopping as soon as the chosen bucket holds
 //                exactly the remaining need) sets their bits; one pass over the bitmap with a
 //                block-wide prefix sum writes the chosen indices in ascending order, and the
-//                forced window (every index of which is larger) is appended.
+//                forced window (every index of which is larger) is appended. Extra CTAs of the
+//                same launch produce the decode output (independent of the selection): per
+//                (sequence, head), the sum of the output records of the CTAs covering the
+//                sequence, divided by L'.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -26,96 +28,103 @@ namespace sel {
 
 constexpr int NT = 1024;
 
-// blockIdx.x < n_collect: bitmap + boundary keys; blockIdx.x >= n_collect: output of head
-// (blockIdx.x - n_collect) of sequence blockIdx.y.
-__global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p, int n_collect) {
+// The decode output of head h of sequence b, by one warp (lane = 4 columns): the decode kernel's
+// CTAs c_lo..c_hi covering the sequence left one unnormalised record each, in consecutive slots
+// from b * cmax; their sum divided by L'_h.
+__device__ __forceinline__ void combine_output(const SelParams& p, int b, int h, unsigned lane) {
+  int g, c_lo, c_hi;
+  p.sch.covering(b, g, c_lo, c_hi);
+  const int n_slots = c_hi - c_lo + 1;
+  if (n_slots > p.sch.cmax || p.D != 128) {
+    if (lane == 0) report_status(p.st, kStatusBounds, 303);
+    return;
+  }
+  const float4* rec = reinterpret_cast<const float4*>(p.opart + ((size_t)p.sch.slot(b, c_lo, c_lo) * p.H + h) * p.D) + lane;
+  const size_t rstride = (size_t)p.H * p.D / 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int i = 0; i < n_slots; ++i) {
+    const float4 v = __ldcg(rec + i * rstride);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  const float inv = 1.f / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
+  __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * lane;
+  reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+}
+
+// Scores one bitmap CTA of the collect kernel classifies: 256 threads x 8 steps x 4 scores.
+constexpr int COLLECT_CHUNK = 8192;
+
+// Bitmap + band keys of scores [blockIdx.x * COLLECT_CHUNK, +COLLECT_CHUNK) of sequence blockIdx.y.
+__global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p) {
   griddep_wait();
   griddep_launch_dependents();
   // both decode launches are complete: re-arm their grid barrier for the next step
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *(volatile unsigned*)p.gbar = 0u;
   const int b = blockIdx.y;
-  if ((int)blockIdx.x >= n_collect) {
-    // the decode kernel's CTAs c_lo..c_hi (of sequence b's group) left one partial each, in
-    // consecutive records from slot b * cmax
-    __shared__ __align__(16) float4 part[8][32];
-    const int h = blockIdx.x - n_collect;
-    int g, c_lo, c_hi;
-    p.sch.covering(b, g, c_lo, c_hi);
-    const int n_slots = c_hi - c_lo + 1;
-    if (n_slots > p.sch.cmax || p.D != 128) {
-      if (threadIdx.x == 0) report_status(p.st, kStatusBounds, 303);
-      return;
-    }
-    const float* rec = p.opart + ((size_t)p.sch.slot(b, c_lo, c_lo) * p.H + h) * p.D;
-    // lane = 4 output columns, warp w sums the partials w, w + 8, ...
-    const int d4 = threadIdx.x & 31, w = threadIdx.x >> 5;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int i = w; i < n_slots; i += 8) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(rec + (size_t)i * p.H * p.D) + d4);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    part[w][d4] = acc;
-    __syncthreads();
-    if (w == 0) {
-      for (int x = 1; x < 8; ++x) {
-        const float4 v = part[x][d4];
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      const float inv = 1.f / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
-      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-      __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * d4;
-      reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x, acc.y);
-      reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z, acc.w);
-    }
-    return;
-  }
+  const unsigned lane = threadIdx.x & 31;
   int* meta = p.meta + b * META;
   const int beta = meta[0], beta_lo = meta[3];
-  const unsigned lane = threadIdx.x & 31;
-  const unsigned lt_mask = (1u << lane) - 1u;
   const float* sc = p.sc + (size_t)b * p.ncand;
   unsigned* bm = p.bitmap + (size_t)b * p.words;
-  const int stride = n_collect * 256 * 4;
-  const int n_round = ((p.ncand + 127) / 128) * 128;
   const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
-  // four consecutive scores per thread per step: one bitmap word, one 16-byte load
-  for (int j0 = (blockIdx.x * 256 + threadIdx.x) * 4; j0 < n_round; j0 += stride) {
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (vec && j0 + 3 < p.ncand) {
-      const float4 f = *reinterpret_cast<const float4*>(sc + j0);
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
-      for (int x = 0; x < 4; ++x)
-        if (j0 + x < p.ncand) v[x] = sc[j0 + x];
-    }
-    unsigned upmask = 0;
+  const int c0 = blockIdx.x * COLLECT_CHUNK + threadIdx.x * 4;
+  // four consecutive scores per thread per step (one bitmap word, one 16-byte load); the loads
+  // of four steps are issued together. Band scores are marked in `band` (bit 4 * step + x) and
+  // appended at the end with one counter update per warp.
+  unsigned band = 0;
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int j = j0 + x;
-      const bool in_range = j < p.ncand;
-      const uint32_t bits = __float_as_uint(v[x]);
-      const int bin = in_range ? (int)((bits >> 20) & (NBINS - 1)) : -2;
-      if (in_range && bin > beta) upmask |= 1u << (j & 31);
-      const bool eq = in_range && bin >= beta_lo && bin <= beta;  // the band: re-scored exactly
-      const unsigned me = __ballot_sync(0xffffffffu, eq);
-      if (me) {
-        int base = 0;
-        const int leader = __ffs(me) - 1;
-        if ((int)lane == leader) base = atomicAdd(&meta[4], __popc(me));
-        base = __shfl_sync(0xffffffffu, base, leader);
-        if (eq) p.bnd[(size_t)b * p.ncand + base + __popc(me & lt_mask)] = (unsigned long long)(uint32_t)j;
+  for (int half = 0; half < 2; ++half) {
+    float v[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j0 = c0 + (half * 4 + k) * 1024;
+      if (vec && j0 + 3 < p.ncand) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + j0));
+        v[k][0] = f.x; v[k][1] = f.y; v[k][2] = f.z; v[k][3] = f.w;
+      } else {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) v[k][x] = j0 + x < p.ncand ? __ldcg(sc + j0 + x) : 0.f;
       }
     }
-    if (upmask) atomicOr(&bm[j0 >> 5], upmask);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j0 = c0 + (half * 4 + k) * 1024;
+      unsigned upmask = 0;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int j = j0 + x;
+        const bool in_range = j < p.ncand;
+        const uint32_t bits = __float_as_uint(v[k][x]);
+        const int bin = in_range ? (int)((bits >> 20) & (NBINS - 1)) : -2;
+        if (in_range && bin > beta) upmask |= 1u << (j & 31);
+        if (in_range && bin >= beta_lo && bin <= beta) band |= 1u << ((half * 4 + k) * 4 + x);  // re-scored exactly
+      }
+      if (upmask) atomicOr(&bm[j0 >> 5], upmask);
+    }
+  }
+  // the warp's band scores get consecutive slots of the sequence's band list
+  const unsigned nb = __popc(band);
+  unsigned incl = nb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= (unsigned)o) incl += n;
+  }
+  const unsigned total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total == 0) return;
+  unsigned base = 0;
+  if (lane == 31) base = (unsigned)atomicAdd(&meta[4], (int)total);
+  unsigned pos = __shfl_sync(0xffffffffu, base, 31) + incl - nb;
+  while (band) {
+    const int bit = __ffs(band) - 1;
+    band &= band - 1;
+    const int j = c0 + (bit >> 2) * 1024 + (bit & 3);
+    p.bnd[(size_t)b * p.ncand + pos++] = (unsigned long long)(uint32_t)j;
   }
 }
 
-// The band keys of every sequence, 128 at a time: their K rows are gathered into shared memory,
-// S^T = K_band Q^T runs on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads), and each thread
-// turns its key's row into the exact score sum_h exp2(s*c - lse2_h) with the exact lse, then into
-// the 64-bit key (score bits << 32 | ~index) the final selection ranks. Persistent CTAs walk the
-// (sequence, tile) pairs of all sequences.
 __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
   griddep_wait();
   griddep_launch_dependents();
@@ -227,6 +236,13 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
 __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
   griddep_wait();
   griddep_launch_dependents();
+  if ((int)blockIdx.x >= p.B) {
+    // the decode output (independent of the selection), a warp per head: NT / 32 heads per CTA
+    const int oc = blockIdx.x - p.B, per_seq = (p.H + NT / 32 - 1) / (NT / 32);
+    const int h = (oc % per_seq) * (NT / 32) + (int)(threadIdx.x >> 5);
+    if (h < p.H) combine_output(p, oc / per_seq, h, threadIdx.x & 31);
+    return;
+  }
   constexpr int KPT = 4;  // band keys held in registers per thread (bands up to NT * KPT keys)
   constexpr int WPT = 8;  // bitmap words per thread per round of the ordered write-out
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -386,11 +402,10 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream) {
   cudaError_t e;
   {
-    int n_collect = (p.ncand + 1023) / 1024;  // 256 threads x 4 scores
-    if (n_collect > 128) n_collect = 128;
+    int n_collect = (p.ncand + COLLECT_CHUNK - 1) / COLLECT_CHUNK;
     if (n_collect < 1) n_collect = 1;
     LaunchScope ls("sel_collect", stream);
-    e = launch_k(sel_collect_kernel, dim3(n_collect + p.H, p.B), dim3(256), 0, stream, true, p, n_collect);
+    e = launch_k(sel_collect_kernel, dim3(n_collect, p.B), dim3(256), 0, stream, true, p);
   }
   if (e != cudaSuccess) return e;
   {
@@ -409,7 +424,9 @@ cudaError_t launch_select(const SelParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   {
     LaunchScope ls("sel_final", stream);
-    e = launch_k(sel_final_kernel, dim3(p.B), dim3(NT), 0, stream, true, p);
+    // B selection CTAs, then the output CTAs
+    const int per_seq = (p.H + NT / 32 - 1) / (NT / 32);
+    e = launch_k(sel_final_kernel, dim3(p.B + p.B * per_seq), dim3(NT), 0, stream, true, p);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
