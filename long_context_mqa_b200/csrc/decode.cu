@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const Sched S = p.sch;
+  const Sched& S = p.sch;  // in parameter space (its start table is indexed at run time)
   const long long limit = p.wait_ns;
   const uint32_t tS = 0, tO = 2 * H;  // TMEM columns: S buffers 0..2H-1, O^T 2H..3H-1
   // launched as a programmatic dependent: nothing before this point touches global memory
@@ -608,10 +608,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __threadfence();
           int* meta = p.meta + b * 8;
           const int K = p.K_sel;
+          {  // L'_h over the sequence's records: 4 threads per head, their loads issued together
+            float(*tl)[H] = reinterpret_cast<float(*)[H]>(&red[0][0][0]);
+            const float* rec = p.lp + (size_t)S.slot(b, c_lo, c_lo) * H + (all_tid & (H - 1));
+            float L4 = 0.f;
+#pragma unroll 8
+            for (int i = all_tid / H; i <= c_hi - c_lo; i += 256 / H) L4 += __ldcg(rec + (size_t)i * H);
+            tl[all_tid / H][all_tid & (H - 1)] = L4;
+          }
+          named_bar(3, 256);
           if (all_tid < H) {
-            const float* rec = p.lp + (size_t)S.slot(b, c_lo, c_lo) * H + all_tid;
-            float L = 0.f;
-            for (int i = 0; i <= c_hi - c_lo; ++i) L += __ldcg(rec + (size_t)i * H);
+            const float(*tl)[H] = reinterpret_cast<const float(*)[H]>(&red[0][0][0]);
+            const float L = (tl[0][all_tid] + tl[1][all_tid]) + (tl[2][all_tid] + tl[3][all_tid]);
             const float lse2 = slse[all_tid] + log2f(L);
             p.lse_out[b * H + all_tid] = lse2 * 0.69314718055994531f;
             p.lse2x[b * H + all_tid] = lse2;

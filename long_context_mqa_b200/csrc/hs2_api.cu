@@ -163,6 +163,10 @@ struct DecodeWs {
   bool ok;  // the schedule's index arithmetic fits (a group of at most 2^32 / G tiles)
 };
 
+// Tiles a decode CTA gives up for crossing a sequence boundary (its second segment's drain,
+// record and logsumexp cost about this many tiles of streaming; measured on B200: ~6 us).
+constexpr int kBoundaryTiles = 4;
+
 static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K, int sms) {
   DecodeWs w{};
   dec::DecParams& p = w.p;
@@ -175,9 +179,12 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   s.tps = (N + 127) / 128;
   s.gs = B;
   s.n_groups = (B + s.gs - 1) / s.gs;
-  if (sms > 256) sms = 256;  // keeps the schedule's 32-bit tile arithmetic in range
+  if (sms > dec::kMaxCtas) sms = dec::kMaxCtas;  // the schedule's start table
   const long long g_tiles = (long long)s.gs * s.tps;
+  w.ok = g_tiles < (1ll << 31);  // 32-bit tile arithmetic inside the group
+  if (!w.ok) return w;
   s.G = (int)(g_tiles < sms ? g_tiles : sms);
+  s.partition(kBoundaryTiles);
   int cmax = 1;
   for (int b = 0; b < B; ++b) {
     int g, lo, hi;
@@ -185,7 +192,6 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
     if (hi - lo + 1 > cmax) cmax = hi - lo + 1;
   }
   s.cmax = cmax;
-  w.ok = (unsigned long long)g_tiles * (unsigned long long)s.G < (1ull << 32);
   const size_t n_slots = (size_t)B * cmax;
   const int ncand = N - W > 0 ? N - W : 0;
   Carve c{(uint8_t*)ws, 0};
