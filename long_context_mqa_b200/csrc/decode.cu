@@ -6,7 +6,7 @@
 // estimates it from a sample of the tiles, phase 2 streams K and V once against that reference,
 // and the selection is made exact with bounds and a re-score of the few keys near the threshold:
 //
-//   phase 1  every sample_stride-th tile of each sequence (about 128 tiles), K only.
+//   phase 1  every sample_stride-th tile of each sequence (about 64 tiles), K only.
 //            S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads); the two
 //            softmax warpgroups split the heads (32 each); every thread owns one key lane and
 //            keeps, per head, a reference r and a sum l of exp2(s*c - r) (r moves only when a

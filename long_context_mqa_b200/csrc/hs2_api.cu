@@ -205,8 +205,8 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   p.lse2x = c.take<float>((size_t)B * H);
   p.ovf = c.take<int>((size_t)B + 1);
   p.fallback = 0;
-  // phase 1 estimates each head's logsumexp from about 128 tiles (16k keys) per sequence
-  p.sample_stride = s.tps / 128 > 1 ? s.tps / 128 : 1;
+  // phase 1 estimates each head's logsumexp from about 64 tiles (8k keys) per sequence
+  p.sample_stride = s.tps / 64 > 1 ? s.tps / 64 : 1;
   p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
   p.seq_done = c.take<int>((size_t)B);
