@@ -10,14 +10,13 @@
 //   O += P V_sel             tcgen05, M = 64 heads, N = d, P (bf16) K-major in shared memory
 // TMEM rows of an M = 64 accumulator sit in lanes 0..15 of each 32-lane quarter, so thread
 // (warp q, lane l < 16) owns head row 16 q + l; lane l + 16 takes over the upper half of that
-// row's keys for the softmax. Two CTAs share an SM, so one CTA's gathers overlap the other's
-// math. With one split the CTA writes the final bf16 output (and lse). With few query rows
+// row's keys for the softmax. Without splits two CTAs share an SM, so one CTA's gathers overlap
+// the other's math. With one split the CTA writes the final bf16 output (and lse). With few query rows
 // (decode) a row's index list is split over a cluster of CTAs; head h of the row is merged by
 // cluster rank h % n: as soon as its own tiles are done (and every CTA of the cluster has
 // started: a cluster barrier arrived at the start, waited on here) each CTA stores its
-// unnormalised O rows into their owners' exchange buffers and its per-head (max, sum) into
-// every CTA's, and after a second cluster barrier each CTA merges its heads from local shared
-// memory. Launched as a programmatic dependent: the prologue overlaps the previous kernel's
+// unnormalised O rows and per-head (max, sum) into their owners' exchange buffers, and after a
+// second cluster barrier each CTA merges its heads from local shared memory. Launched as a programmatic dependent: the prologue overlaps the previous kernel's
 // tail and every global read waits for it.
 #include "decode.h"
 #include "host_util.h"
@@ -325,11 +324,10 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     }
     if (owns) {
       const float mv = l_run > 0.f && have ? m_run : -INFINITY, lv = have ? l_run : 0.f;
+      // only the owner reads head `head`'s (max, sum)
       const uint32_t m_loc = smem_u32(xm + split * MH + head), l_loc = smem_u32(xl + split * MH + head);
-      for (int s2 = 0; s2 < n; ++s2) {
-        st_dsmem_f32(dsmem_addr(m_loc, s2), mv);
-        st_dsmem_f32(dsmem_addr(l_loc, s2), lv);
-      }
+      st_dsmem_f32(dsmem_addr(m_loc, (uint32_t)owner), mv);
+      st_dsmem_f32(dsmem_addr(l_loc, (uint32_t)owner), lv);
     }
   }
   tc_fence_before();
