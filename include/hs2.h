@@ -97,12 +97,31 @@ HS2_API const char* hs2_status_string(hs2_status s);
  * idx  [B, Lq, window+topk] int32  selected token indices of each query, ascending;
  *                           exactly min(t+1, window+topk) valid entries, then -1 padding
  * Supported: (H, d) in {(64, 128), (16, 64)}; Lq == 1 or Lq == Lk (bf16, fp32 accumulate).
- * Decode (Lq == 1) supports (H, d) = (64, 128); prefill (Lq == Lk) supports topk <= 1024.
+ * Decode (Lq == 1) supports (H, d) = (64, 128) and B <= 256; prefill (Lq == Lk) supports
+ * topk <= 1024.
  */
 HS2_API size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk);
 HS2_API hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,
                                 int H, int d, float scale, int window, int topk, hs2_bf16* out, float* lse,
                                 int32_t* idx, void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* Ragged decode: one query per sequence, sequence b with its own cache length lens[b] (the
+ * per-sequence N of multi-turn agent serving, whose short actions and long, accumulating
+ * observations the pages take as the setting: arex-research.com, the lead and section
+ * "短动作、长观测：prefill、KV cache 与检索同时成为瓶颈").
+ * lens is a HOST array of B lengths, 1 <= lens[b] <= Lk, read before the call returns (the
+ * work split across SMs is computed from it on the host). K, V are [B, Lk, d]: sequence b's
+ * cache is its first lens[b] rows, the rest is never read. Q, out [B, 1, H, d]; lse [B, 1, H];
+ * idx [B, 1, window+topk] as above, sequence b's query sitting at t = lens[b] - 1. Every
+ * sequence's result equals hs2_full_attn_select on that sequence alone. Supported: (H, d) =
+ * (64, 128), 1 <= B <= 256. The workspace size depends on lens (query it with the same lens).
+ */
+HS2_API size_t hs2_full_attn_select_ragged_workspace_bytes(int B, const int32_t* lens, int Lk, int H, int d,
+                                                           int window, int topk);
+HS2_API hs2_status hs2_full_attn_select_ragged(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B,
+                                               const int32_t* lens, int Lk, int H, int d, float scale, int window,
+                                               int topk, hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                               size_t workspace_bytes, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * Sparse attention over selected tokens (one sparse layer)

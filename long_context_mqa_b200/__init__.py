@@ -53,6 +53,10 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_full_attn_select_workspace_bytes.restype = sz
     lib.hs2_full_attn_select.argtypes = [P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, P, P, P, P, sz, P]
     lib.hs2_full_attn_select.restype = i32
+    lib.hs2_full_attn_select_ragged_workspace_bytes.argtypes = [i32, P, i32, i32, i32, i32, i32]
+    lib.hs2_full_attn_select_ragged_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select_ragged.argtypes = [P, P, P, i32, P, i32, i32, i32, f32, i32, i32, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_ragged.restype = i32
     lib.hs2_sparse_attn_workspace_bytes.argtypes = [i32] * 6
     lib.hs2_sparse_attn_workspace_bytes.restype = sz
     lib.hs2_sparse_attn.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, sz, P]
@@ -158,6 +162,50 @@ def full_attn_select(q, k, v, *, scale=None, window=WINDOW, topk=TOPK, out=None,
                                     out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
                                     ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(code, "hs2_full_attn_select")
+    return out, lse, idx
+
+
+def _lens_array(lens, B, Lk):
+    arr = (ctypes.c_int32 * B)(*[int(x) for x in lens])
+    if len(lens) != B or any(not (1 <= int(x) <= Lk) for x in lens):
+        raise ValueError(f"lens must hold B={B} lengths in [1, {Lk}]")
+    return arr
+
+
+def full_attn_select_ragged_workspace_bytes(lens, Lk, H, d, window=WINDOW, topk=TOPK) -> int:
+    B = len(lens)
+    return int(lib.hs2_full_attn_select_ragged_workspace_bytes(B, _lens_array(lens, B, Lk), Lk, H, d, window, topk))
+
+
+def full_attn_select_ragged(q, k, v, lens, *, scale=None, window=WINDOW, topk=TOPK, out=None, lse=None, idx=None,
+                            workspace=None, stream=None):
+    """Decode over sequences of different cache lengths (hs2_full_attn_select_ragged).
+
+    q [B,1,H,d]; k, v [B,Lk,d] with sequence b's cache in its first lens[b] rows; lens: B host
+    integers. Returns (out [B,1,H,d] bf16, lse [B,1,H] fp32, idx [B,1,window+topk] int32).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    if Lq != 1 or tuple(k.shape) != (B, Lk, d) or tuple(v.shape) != (B, Lk, d):
+        raise ValueError("q must be [B,1,H,d] and k, v [B,Lk,d]")
+    lens_c = _lens_array(list(lens), B, Lk)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = window + topk
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, 1, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, 1, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    nbytes = int(lib.hs2_full_attn_select_ragged_workspace_bytes(B, lens_c, Lk, H, d, window, topk))
+    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    code = lib.hs2_full_attn_select_ragged(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, lens_c, Lk, H, d, scale, window,
+                                           topk, out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                           ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select_ragged")
     return out, lse, idx
 
 

@@ -1,12 +1,13 @@
 // Decode step of the full-attention + selection layer (one query token per sequence, the
-// query at position t = N-1 of an N-token K/V cache), as one persistent kernel.
+// query at position t = N_b - 1 of sequence b's N_b-token K/V cache; the N_b may differ), as one
+// persistent kernel.
 //
 // The score of a key is sum_h p_h = sum_h exp(s_h - lse_h): each head's logsumexp over the whole
 // row is needed before any score is final. Instead of a full first pass over K for it, phase 1
 // estimates it from a sample of the tiles, phase 2 streams K and V once against that reference,
 // and the selection is made exact with bounds and a re-score of the few keys near the threshold:
 //
-//   phase 1  every sample_stride-th tile of each sequence (about 64 tiles), K only.
+//   phase 1  every st-th tile of each sequence (about 64 tiles), K only.
 //            S^T = K_tile Q^T on tcgen05 (M = 128 keys in TMEM lanes, N = 64 heads); the two
 //            softmax warpgroups split the heads (32 each); every thread owns one key lane and
 //            keeps, per head, a reference r and a sum l of exp2(s*c - r) (r moves only when a
@@ -26,7 +27,7 @@
 //            not. select.cu collects the band between them, re-scores it exactly and selects.
 //
 // A sequence whose p' reaches 2^64 (a key far more probable than everything sampled) is flagged
-// and redone with every tile (sample_stride 1: the reference is then the exact lse) by a second
+// and redone with every tile (the reference is then the exact lse) by a second
 // launch of this kernel, which leaves at once when nothing is flagged.
 //
 // The grid is one CTA per SM, launched cooperatively (all CTAs co-resident). Warp roles
@@ -87,6 +88,11 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
 
 // the first phase-1 (sampled) tile at or after local tile lt
 __device__ __forceinline__ int first_sample(int lt, int st) { return (lt + st - 1) / st * st; }
+// phase 1 of sequence b takes every st-th tile: about `target` tiles (every tile when target is 0)
+__device__ __forceinline__ int sample_stride(const Sched& S, int b, int target) {
+  const int tiles = (int)(S.seq_start[b + 1] - S.seq_start[b]);
+  return target > 0 && tiles / target > 1 ? tiles / target : 1;
+}
 
 template <int H, int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -175,29 +181,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         long long t0, t1;
         S.range(g, cta, t0, t1);
         for (long long t = t0; t < t1 && ok;) {  // phase 1: K, ascending
-          const int b = (int)(t / S.tps);
-          const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          const int b = S.seq_of(t);
+          const long long seg_end = t1 < (long long)S.seq_start[b + 1] ? t1 : (long long)S.seq_start[b + 1];
           if (skip_seq(b)) { t = seg_end; continue; }
           if (!load_q(b)) { ok = false; break; }
-          const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
-          for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi && ok; lt += st)
+          const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
+          for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi && ok; lt += st)
             if (!load_tile(&tmK, lt, b, keep)) ok = false;
           t = seg_end;
         }
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: descending
-          const int b = (int)(t / S.tps);
-          const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          const int b = S.seq_of(t);
+          const long long seg_lo = t0 > (long long)S.seq_start[b] ? t0 : (long long)S.seq_start[b];
           if (skip_seq(b)) { t = seg_lo - 1; continue; }
           if (!load_q(b)) { ok = false; break; }
           // in the order the tensor core consumes them: S of a tile needs its K, then the PV of
           // the tile before it (the next higher one) needs that tile's V
           const long long seg_hi = t;
           for (; t >= seg_lo; --t) {
-            const int lt = (int)(t - (long long)b * S.tps);
+            const int lt = (int)(t - (long long)S.seq_start[b]);
             if (!load_tile(&tmK, lt, b, once)) { ok = false; break; }
             if (t < seg_hi && !load_tile(&tmV, lt + 1, b, once)) { ok = false; break; }
           }
-          if (ok && !load_tile(&tmV, (int)(seg_lo - (long long)b * S.tps), b, once)) { ok = false; break; }
+          if (ok && !load_tile(&tmV, (int)(seg_lo - (long long)S.seq_start[b]), b, once)) { ok = false; break; }
         }
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
@@ -254,12 +260,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         long long t0, t1;
         S.range(g, cta, t0, t1);
         for (long long t = t0; t < t1 && ok;) {  // phase 1
-          const int b = (int)(t / S.tps);
-          const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+          const int b = S.seq_of(t);
+          const long long seg_end = t1 < (long long)S.seq_start[b + 1] ? t1 : (long long)S.seq_start[b + 1];
           if (skip_seq(b)) { t = seg_end; continue; }
           if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
-          const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
-          for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi && ok; lt += st)
+          const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
+          for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi && ok; lt += st)
             if (!issue_s(ri++)) ok = false;
           t = seg_end;
           if (!ok) break;
@@ -267,8 +273,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ++nq;
         }
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2
-          const int b = (int)(t / S.tps);
-          const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+          const int b = S.seq_of(t);
+          const long long seg_lo = t0 > (long long)S.seq_start[b] ? t0 : (long long)S.seq_start[b];
           if (skip_seq(b)) { t = seg_lo - 1; continue; }
           const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
           // S of a tile, then PV of the tile before it
@@ -298,7 +304,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int swarp = all_tid >> 5;                 // 0..7
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float c = p.c;
-    const int ncand = p.N - p.W > 0 ? p.N - p.W : 0;
     float(*red1)[4][HW][2] = reinterpret_cast<float(*)[4][HW][2]>(&red[0][0][0]);
     // state the selection accumulates into, cleared before this CTA's first grid-barrier arrival
     if (cta == 0) {
@@ -325,15 +330,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------------------------------- phase 1 (sampled tiles)
       uint32_t n1 = 0;  // K tiles phase 1 took through the ring
       for (long long t = t0; t < t1;) {
-        const int b = (int)(t / S.tps);
-        const long long seg_end = t1 < (long long)(b + 1) * S.tps ? t1 : (long long)(b + 1) * S.tps;
+        const int b = S.seq_of(t);
+        const long long seg_end = t1 < (long long)S.seq_start[b + 1] ? t1 : (long long)S.seq_start[b + 1];
         if (skip_seq(b)) { t = seg_end; continue; }  // uniform: every softmax warp skips it
         bool first = true;
         float r[HW], l[HW];
 #pragma unroll
         for (int h = 0; h < HW; ++h) { r[h] = -INFINITY; l[h] = 0.f; }
-        const int st = p.sample_stride, lt_hi = (int)(seg_end - (long long)b * S.tps);
-        for (int lt = first_sample((int)(t - (long long)b * S.tps), st); lt < lt_hi; lt += st) {
+        const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
+        for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi; lt += st) {
           const uint32_t jt = js++;
           ++n1;
           if (!ok) continue;
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[buf]);
-          const bool valid = lt * TILE + row < p.N;
+          const bool valid = lt * TILE + row < S.seq_len[b];
           if (first) {
             // a lane's first key of the segment sets its references (invalid lanes only occur in
             // a sequence's partial last tile, which then is the segment's last sampled tile)
@@ -405,7 +410,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int hg = all_tid / HW, hh = all_tid % HW;
           float mm = red1[hg][0][hh][0], ll = red1[hg][0][hh][1];
           for (int w = 1; w < 4; ++w) merge_ml(mm, ll, red1[hg][w][hh][0], red1[hg][w][hh][1]);
-          const size_t sl = (size_t)S.slot(b, cta, S.cta_of(g, (long long)b * S.tps));
+          const size_t sl = (size_t)S.slot(b, cta, S.cta_of(g, (long long)S.seq_start[b]));
           p.ml[sl * 2 * H + all_tid] = mm;
           p.ml[sl * 2 * H + H + all_tid] = ll;
         }
@@ -440,11 +445,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (abort_flag) ok = false;
       // ---------------------------------------------------------------- phase 2
       for (long long t = t1 - 1; t >= t0;) {
-        const int b = (int)(t / S.tps);
-        const long long seg_lo = t0 > (long long)b * S.tps ? t0 : (long long)b * S.tps;
+        const int b = S.seq_of(t);
+        const long long seg_lo = t0 > (long long)S.seq_start[b] ? t0 : (long long)S.seq_start[b];
         if (skip_seq(b)) { t = seg_lo - 1; continue; }  // uniform: every softmax warp skips it
         int sg, c_lo, c_hi;
         S.covering(b, sg, c_lo, c_hi);
+        const int n_b = S.seq_len[b], ncand = n_b - p.W > 0 ? n_b - p.W : 0;  // this sequence's
         {  // the sequence's lse from every phase-1 partial of it: 16 threads per partial record
            // (4 heads each), 16 records per round, then a shuffle and a shared-memory merge
           const int q4 = all_tid & 15;
@@ -479,7 +485,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float la = 0.f, lb = 0.f;  // sums of p' over this warp's keys for heads 2*lane, 2*lane + 1
         for (uint32_t x = 0; x < n; ++x, --t, ++jp, ++js) {
           if ((int)(jp & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
-          const int lt = (int)(t - (long long)b * S.tps);
+          const int lt = (int)(t - (long long)S.seq_start[b]);
           const int buf = jp & 1;   // == wg: this warpgroup's P buffer
           const int sbi = js & 1;   // the TMEM S buffer of this tile
           if (!warp_wait_bar(&s_full[sbi], (js >> 1) & 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
@@ -497,7 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cnt(&s_empty[sbi], 2);
           const int key = lt * TILE + row;
-          const bool valid = key < p.N;
+          const bool valid = key < n_b;
           float sa = 0.f, sb = 0.f;
           uint32_t pk[H / 2];
 #pragma unroll
@@ -521,6 +527,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (atomicExch(&p.ovf[b], 1) == 0) atomicAdd(&p.ovf[p.B], 1);
           }
           if (!warp_wait_bar(&p_empty[buf], (npu & 1) ^ 1, limit, &abort_flag, p.st, 223)) { ok = false; continue; }
+          if ((lt + 1) * TILE > n_b) {
+            // the sequence's last tile, partial: its V rows past the sequence hold whatever the
+            // caller's buffer holds there (rows of a longer sequence's slot in a ragged batch).
+            // P is 0 for them, but 0 * inf is NaN in the PV product: zero those rows first. The
+            // tile's V item cannot be overwritten before this warpgroup's P releases its PV.
+            const uint32_t vi = x == n - 1 ? base + 2 * n - 1 : base + 2 * x + 2;
+            const int vs = (int)(vi % RING);
+            if (!warp_wait_bar(&r_full[vs], (vi / RING) & 1, limit, &abort_flag, p.st, 225)) { ok = false; continue; }
+            if (!valid) {
+              const uint32_t vrow = smem_u32(sR + vs * KT_BYTES);
+#pragma unroll
+              for (int ch = 0; ch < D / 8; ++ch)
+                st_shared_v4(vrow + (ch / 8) * (TILE * 128) + sw128_off(row, ch % 8), 0u, 0u, 0u, 0u);
+            }
+            fence_async_smem();  // the zeros are read by the tensor core
+          }
           const uint32_t prow = smem_u32(sP + buf * P_BYTES);
 #pragma unroll
           for (int ch = 0; ch < H / 8; ++ch)
@@ -546,7 +568,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           la += v[0];
           lb += v[1];
           const bool is_cand = valid && key < ncand;
-          if (is_cand) p.sc[(size_t)b * ncand + key] = score;
+          if (is_cand) p.sc[(size_t)b * p.sc_stride + key] = score;
           const unsigned bin = (__float_as_uint(score) >> 20) & (NBINS - 1);
           const unsigned act = __ballot_sync(0xffffffffu, is_cand);
           if (is_cand) {
@@ -741,7 +763,7 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
     DecParams q = p;
     if (pass == 1) {
       q.fallback = 1;
-      q.sample_stride = 1;
+      q.sample_tiles = 0;  // every tile: the reference is the exact lse
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.sch.G);

@@ -14,23 +14,24 @@ struct DevStatus;
 namespace dec {
 // Parameters of the fused decode (one query per sequence) full-attention + selection kernel.
 struct DecParams {
-  int B, N, W, K;          // sequences, cache length, window, top-k
-  Sched sch;               // groups of sequences x contiguous tile ranges per CTA
+  int B, N, W, K;          // sequences, cache rows per sequence in K/V (the longest length), window, top-k
+  Sched sch;               // per-sequence lengths and tiles, contiguous tile ranges per CTA
   float c;                 // scale * log2(e)
   long long wait_ns;       // bound of every device-side wait
-  float* ml;               // [n_groups*G*segmax][2][H] phase-1 partial (max, sum), log2 domain
+  float* ml;               // [B*cmax][2][H] phase-1 partial (max, sum), log2 domain
   float* lse_out;          // [B][H] natural log (caller's lse)
-  float* opart;            // [n_groups*G*segmax][H][D] phase-2 partial outputs
-  float* sc;               // [B][N-W] head-summed scores of the older tokens
+  float* opart;            // [B*cmax][H][D] phase-2 partial outputs
+  float* sc;               // [B][sc_stride] head-summed scores of the older tokens
+  int sc_stride;           // max(N - W, 1): room for the longest sequence's older tokens
   unsigned* hist;          // [B][2048] histogram of score bits 30..20
   int* seq_done;           // [B] CTAs done with each sequence's histogram
   unsigned* bitmap;        // [B][words] selection bitmap of the older tokens (cleared here)
-  int words;               // ceil((N - W) / 32) rounded up to a multiple of 8 (32-byte rows)
+  int words;               // ceil(sc_stride / 32) rounded up to a multiple of 8 (32-byte rows)
   int* meta;               // [B][8] selection metadata (threshold bin, above, need, counters)
   int K_sel;               // top-k of the selection (== K)
   unsigned* gbar;          // grid-barrier arrivals: zero when a step starts; the sampled launch
                            // counts to G per group, the redo on from there (the collect kernel re-arms it)
-  int sample_stride;       // phase 1 takes every sample_stride-th tile of each sequence
+  int sample_tiles;        // phase 1 samples about this many tiles per sequence (0: every tile)
   float* lp;               // [B*cmax][H] per-(sequence, CTA) sums of p' = exp2(s*c - lse2')
   float* lsum;             // [B][H] their totals L'_h (the output is sum(O') / L')
   float* lse2x;            // [B][H] exact lse, log2 units (for the exact re-score of the band)
@@ -49,8 +50,9 @@ constexpr int META = 8;  // ints per sequence: bin above which all are in, their
                          // bin, band keys collected, band size expected
 // Top-k selection over a materialised score vector per sequence (decode path).
 struct SelParams {
-  int B, N, W, K, S;
-  int ncand;                     // max(N - W, 0) older tokens per sequence
+  int B, N, W, K, S;              // N: cache rows per sequence in K (the longest length)
+  int ncand;                     // max(N - W, 1): the stride of the per-sequence score and band
+                                 // arrays; sequence b's own count is max(sch.seq_len[b] - W, 0)
   const float* sc;               // [B][ncand]
   const unsigned* hist;          // [B][NBINS]
   int* meta;                     // [B][META]
@@ -67,7 +69,7 @@ struct SelParams {
   dec::Sched sch;
   // exact re-score of the band keys
   const __nv_bfloat16* qry;      // [B][H][D] the decode queries
-  const __nv_bfloat16* kc;       // [B][N][D] the K cache
+  const __nv_bfloat16* kc;       // [B][N][D] the K cache (sequence b's first seq_len[b] rows)
   const float* lse2x;            // [B][H] exact lse, log2 units
   float c;                       // scale * log2(e)
   int sms;

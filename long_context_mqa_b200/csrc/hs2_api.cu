@@ -167,23 +167,23 @@ struct DecodeWs {
 // record and logsumexp cost about this many tiles of streaming; measured on B200: ~6 us).
 constexpr int kBoundaryTiles = 4;
 
-static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K, int sms) {
+static DecodeWs carve_decode(void* ws, int B, const int* lens, int N, int H, int D, int W, int K, int sms) {
   DecodeWs w{};
   dec::DecParams& p = w.p;
   p.B = B; p.N = N; p.W = W; p.K = K;
-  // One group of all sequences. (The schedule can split them into groups small enough for a
-  // group's K to stay in L2 between the phases; measured on B200 the per-group grid barrier,
+  w.ok = B <= dec::kMaxSeqs;  // the schedule's per-sequence tables
+  if (!w.ok) return w;
+  // One flattened range of all sequences' tiles. (Sequences can be taken in groups small enough
+  // for a group's K to stay in L2 between the phases; measured on B200 the per-group grid barrier,
   // pipeline drain and refill cost more than the HBM re-reads they save.)
   dec::Sched& s = p.sch;
-  s.B = B;
-  s.tps = (N + 127) / 128;
-  s.gs = B;
-  s.n_groups = (B + s.gs - 1) / s.gs;
-  if (sms > dec::kMaxCtas) sms = dec::kMaxCtas;  // the schedule's start table
-  const long long g_tiles = (long long)s.gs * s.tps;
-  w.ok = g_tiles < (1ll << 31);  // 32-bit tile arithmetic inside the group
+  long long tiles = 0;
+  for (int b = 0; b < B; ++b) tiles += (lens[b] + 127) / 128;
+  w.ok = tiles < (1ll << 31);  // 32-bit tile arithmetic
   if (!w.ok) return w;
-  s.G = (int)(g_tiles < sms ? g_tiles : sms);
+  s.set_lengths(B, lens);
+  if (sms > dec::kMaxCtas) sms = dec::kMaxCtas;  // the schedule's start table
+  s.G = (int)(tiles < sms ? tiles : sms);
   s.partition(kBoundaryTiles);
   int cmax = 1;
   for (int b = 0; b < B; ++b) {
@@ -193,7 +193,7 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   }
   s.cmax = cmax;
   const size_t n_slots = (size_t)B * cmax;
-  const int ncand = N - W > 0 ? N - W : 0;
+  const int stride = N - W > 1 ? N - W : 1;  // room for the longest sequence's older tokens
   Carve c{(uint8_t*)ws, 0};
   p.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
   // the grid-barrier counter lives in the status block, so clearing the status re-arms it
@@ -206,16 +206,17 @@ static DecodeWs carve_decode(void* ws, int B, int N, int H, int D, int W, int K,
   p.ovf = c.take<int>((size_t)B + 1);
   p.fallback = 0;
   // phase 1 estimates each head's logsumexp from about 64 tiles (8k keys) per sequence
-  p.sample_stride = s.tps / 64 > 1 ? s.tps / 64 : 1;
-  p.sc = c.take<float>((size_t)B * (ncand > 0 ? ncand : 1));
+  p.sample_tiles = 64;
+  p.sc_stride = stride;
+  p.sc = c.take<float>((size_t)B * stride);
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
   p.seq_done = c.take<int>((size_t)B);
   w.meta = c.take<int>((size_t)B * sel::META);
   p.meta = w.meta;
   p.K_sel = K;
-  p.words = ((ncand + 31) / 32 + 7) / 8 * 8;  // rows of 32-byte multiples (vector loads)
-  p.bitmap = c.take<unsigned>((size_t)B * (p.words > 0 ? p.words : 1));
-  w.bnd = c.take<unsigned long long>((size_t)B * (ncand > 0 ? ncand : 1));
+  p.words = ((stride + 31) / 32 + 7) / 8 * 8;  // rows of 32-byte multiples (vector loads)
+  p.bitmap = c.take<unsigned>((size_t)B * p.words);
+  w.bnd = c.take<unsigned long long>((size_t)B * stride);
   w.bytes = c.off;
   return w;
 }
@@ -283,8 +284,50 @@ void hs2_set_wait_limit_ns(long long limit_ns) { g_wait_ns = limit_ns > 0 ? limi
 size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk) {
   if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || d <= 0 || window < 1 || topk < 0) return 0;
   const int sms = num_sms() > 0 ? num_sms() : 148;
-  if (Lq == 1) return carve_decode(nullptr, B, Lk, H, d, window, topk, sms).bytes;
+  if (Lq == 1) {
+    if (B > dec::kMaxSeqs) return 0;
+    std::vector<int> lens((size_t)B, Lk);
+    return carve_decode(nullptr, B, lens.data(), Lk, H, d, window, topk, sms).bytes;
+  }
   return prefill::workspace_bytes(B, Lq, Lk, H, d, window, topk, sms, kStatusBytes);
+}
+
+// The decode path (one query per sequence at the end of its lens[b]-token cache).
+static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, const int* lens, int Lk,
+                             int H, int d, float c, int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
+                             void* workspace, size_t workspace_bytes, int sms, cudaStream_t st) {
+  if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
+  DecodeWs w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
+  if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
+  w.p.c = c;
+  w.p.wait_ns = wait_limit_ns();
+  w.p.lse_out = lse;
+  CUtensorMap tmK, tmV, tmQ;
+  if (!make_tmap_3d(&tmK, K, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+      !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+      !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
+    return HS2_ERR_CUDA;
+  if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, st) != cudaSuccess) return HS2_ERR_CUDA;
+  sel::SelParams sp;
+  sp.opart = w.p.opart;
+  sp.out = reinterpret_cast<__nv_bfloat16*>(out);
+  sp.H = H; sp.D = d; sp.sch = w.p.sch;
+  sp.lsum = w.p.lsum;
+  sp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
+  sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
+  sp.lse2x = w.p.lse2x;
+  sp.gbar = w.p.gbar;
+  sp.c = c;
+  sp.sms = sms;
+  sp.wait_ns = w.p.wait_ns;
+  sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
+  sp.ncand = w.p.sc_stride;
+  sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.bnd = w.bnd;
+  sp.bitmap = w.p.bitmap; sp.words = w.p.words;
+  sp.idx = idx; sp.st = w.p.st;
+  if (sel::launch_select(sp, st) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
 }
 
 hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,
@@ -302,42 +345,47 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float c = scale * 1.4426950408889634f;
   if (Lq == 1) {
-    if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
-    DecodeWs w = carve_decode(workspace, B, Lk, H, d, window, topk, sms);
-    if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
-    if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
-    w.p.c = c;
-    w.p.wait_ns = wait_limit_ns();
-    w.p.lse_out = lse;
-    CUtensorMap tmK, tmV, tmQ;
-    if (!make_tmap_3d(&tmK, K, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
-        !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
-        !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
-      return HS2_ERR_CUDA;
-    if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, st) != cudaSuccess) return HS2_ERR_CUDA;
-    sel::SelParams sp;
-    sp.opart = w.p.opart;
-    sp.out = reinterpret_cast<__nv_bfloat16*>(out);
-    sp.H = H; sp.D = d; sp.sch = w.p.sch;
-    sp.lsum = w.p.lsum;
-    sp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
-    sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
-    sp.lse2x = w.p.lse2x;
-    sp.gbar = w.p.gbar;
-    sp.c = c;
-    sp.sms = sms;
-    sp.wait_ns = w.p.wait_ns;
-    sp.B = B; sp.N = Lk; sp.W = window; sp.K = topk; sp.S = window + topk;
-    sp.ncand = Lk - window > 0 ? Lk - window : 0;
-    sp.sc = w.p.sc; sp.hist = w.p.hist; sp.meta = w.meta; sp.bnd = w.bnd;
-    sp.bitmap = w.p.bitmap; sp.words = w.p.words;
-    sp.idx = idx; sp.st = w.p.st;
-    if (sel::launch_select(sp, st) != cudaSuccess) return HS2_ERR_CUDA;
-    return HS2_OK;
+    if (B > dec::kMaxSeqs) return HS2_ERR_UNSUPPORTED_SHAPE;
+    std::vector<int> lens((size_t)B, Lk);
+    return run_decode(Q, K, V, B, lens.data(), Lk, H, d, c, window, topk, out, lse, idx, workspace, workspace_bytes,
+                      sms, st);
   }
   if (Lq != Lk) return HS2_ERR_UNSUPPORTED_SHAPE;
   return prefill::run(Q, K, V, B, Lq, Lk, H, d, c, window, topk, out, lse, idx, workspace, workspace_bytes, sms,
                       kStatusBytes, st);
+}
+
+static bool ragged_lens_ok(int B, const int32_t* lens, int Lk) {
+  if (!lens || B <= 0 || B > dec::kMaxSeqs) return false;
+  for (int b = 0; b < B; ++b)
+    if (lens[b] < 1 || lens[b] > Lk) return false;
+  return true;
+}
+
+size_t hs2_full_attn_select_ragged_workspace_bytes(int B, const int32_t* lens, int Lk, int H, int d, int window,
+                                                   int topk) {
+  if (Lk <= 0 || H <= 0 || d <= 0 || window < 1 || topk < 0 || !ragged_lens_ok(B, lens, Lk)) return 0;
+  const int sms = num_sms() > 0 ? num_sms() : 148;
+  return carve_decode(nullptr, B, reinterpret_cast<const int*>(lens), Lk, H, d, window, topk, sms).bytes;
+}
+
+hs2_status hs2_full_attn_select_ragged(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B,
+                                       const int32_t* lens, int Lk, int H, int d, float scale, int window, int topk,
+                                       hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                       size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K || !V || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(lse) || !aligned16(idx))
+    return HS2_ERR_INVALID_ARG;
+  if (Lk <= 0 || window < 1 || topk < 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (!lens || B <= 0) return HS2_ERR_INVALID_ARG;
+  if (B > dec::kMaxSeqs) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!ragged_lens_ok(B, lens, Lk)) return HS2_ERR_INVALID_ARG;
+  if (window + topk > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!shape_ok(H, d)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  return run_decode(Q, K, V, B, reinterpret_cast<const int*>(lens), Lk, H, d, scale * 1.4426950408889634f, window,
+                    topk, out, lse, idx, workspace, workspace_bytes, num_sms(), reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int d, int S) {

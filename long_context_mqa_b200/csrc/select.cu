@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p) {
   const int beta = meta[0], beta_lo = meta[3];
   const float* sc = p.sc + (size_t)b * p.ncand;
   unsigned* bm = p.bitmap + (size_t)b * p.words;
+  const int nc = p.sch.seq_len[b] - p.W > 0 ? p.sch.seq_len[b] - p.W : 0;  // this sequence's older tokens
   const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
   const int c0 = blockIdx.x * COLLECT_CHUNK + threadIdx.x * 4;
   // four consecutive scores per thread per step (one bitmap word, one 16-byte load); the loads
@@ -80,12 +81,12 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int j0 = c0 + (half * 4 + k) * 1024;
-      if (vec && j0 + 3 < p.ncand) {
+      if (vec && j0 + 3 < nc) {
         const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + j0));
         v[k][0] = f.x; v[k][1] = f.y; v[k][2] = f.z; v[k][3] = f.w;
       } else {
 #pragma unroll
-        for (int x = 0; x < 4; ++x) v[k][x] = j0 + x < p.ncand ? __ldcg(sc + j0 + x) : 0.f;
+        for (int x = 0; x < 4; ++x) v[k][x] = j0 + x < nc ? __ldcg(sc + j0 + x) : 0.f;
       }
     }
 #pragma unroll
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256) sel_collect_kernel(SelParams p) {
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
         const int j = j0 + x;
-        const bool in_range = j < p.ncand;
+        const bool in_range = j < nc;
         const uint32_t bits = __float_as_uint(v[k][x]);
         const int bin = in_range ? (int)((bits >> 20) & (NBINS - 1)) : -2;
         if (in_range && bin > beta) upmask |= 1u << (j & 31);
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
     const int slot = tile * TILE + tid;
     const bool in = slot < n_band;
     const int j = in ? (int)(uint32_t)p.bnd[(size_t)b * p.ncand + slot] : 0;
-    const bool valid = in && j >= 0 && j < p.ncand;
+    const bool valid = in && j >= 0 && j < p.sch.seq_len[b] - p.W;
     {
       const __nv_bfloat16* kb = p.kc + (size_t)b * p.N * D;
       const int jv = valid ? j : -1, sub = lane >> 4, ch = lane & 15;
@@ -390,11 +391,12 @@ __global__ void __launch_bounds__(NT) sel_final_kernel(SelParams p) {
     __syncthreads();  // wsum is rewritten by the next round
   }
   const unsigned total_top = done;
-  const int wlen = p.N < p.W ? p.N : p.W;
-  const int expect_top = p.ncand < p.K ? p.ncand : p.K;
+  const int n_b = p.sch.seq_len[b], nc = n_b - p.W > 0 ? n_b - p.W : 0;  // this sequence's
+  const int wlen = n_b < p.W ? n_b : p.W;
+  const int expect_top = nc < p.K ? nc : p.K;
   if (tid == 0 && (int)total_top != expect_top) report_status(p.st, kStatusBounds, 302);
   for (int i = tid; i < p.S; i += NT) {
-    if (i >= (int)total_top && i < (int)total_top + wlen) out[i] = p.N - wlen + (i - (int)total_top);
+    if (i >= (int)total_top && i < (int)total_top + wlen) out[i] = n_b - wlen + (i - (int)total_top);
     else if (i >= (int)total_top + wlen) out[i] = -1;
   }
 }

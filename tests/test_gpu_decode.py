@@ -91,11 +91,11 @@ def test_decode_full_size(hs2, name):
 
 
 def test_decode_dominant_key_outside_the_phase1_sample_is_redone_exactly(hs2):
-    """Phase 1 estimates each head's logsumexp from a sample of the tiles (every 2nd tile here).
+    """Phase 1 estimates each head's logsumexp from a sample of the tiles (every 4th tile here).
     A key that head 0 prefers over all sampled keys by about 2^74 sits in an unsampled tile: its
     unnormalised probability overflows the sampled reference, the sequence is flagged, and the
     exact redo (every tile) must give the oracle's output, lse and selection."""
-    B, N, j = 2, 40000, 200  # 313 tiles per sequence: phase 1 takes tiles 0, 2, 4, ...; key 200 is in tile 1
+    B, N, j = 2, 40000, 200  # 313 tiles per sequence: phase 1 takes tiles 0, 4, 8, ...; key 200 is in tile 1
     g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=N))
     q0 = bf16_to_f64(to_torch_bf16(g.q[1, 0, 0]))
     k_dom = 60.0 * q0 / np.linalg.norm(q0)
@@ -103,3 +103,61 @@ def test_decode_dominant_key_outside_the_phase1_sample_is_redone_exactly(hs2):
     q, k, v, out, lse, idx = _run_full(hs2, g)
     ora, st = _check_full(g, out, lse, idx)
     assert j in set(idx.cpu().numpy()[1, 0].tolist())
+
+
+def _check_seq(g, b, n, out, lse, idx):
+    """Sequence b of a ragged batch against the oracle run on that sequence alone (n tokens)."""
+    wl = g.wl
+    ora = oracle.full_attn_select(g.q[b:b + 1], g.k[b:b + 1, :n], g.v[b:b + 1, :n], wl.scale, wl.window, wl.topk,
+                                  want_score=True)
+    assert_out_close(bf16_to_f64(out[b:b + 1]).reshape(ora["out"].shape), ora["out"], f"sequence {b} (N={n})")
+    assert np.abs(lse[b].double().cpu().numpy().reshape(ora["lse"].shape) - ora["lse"]).max() < 2e-3
+    st = check_selection(idx[b].cpu().numpy().reshape(1, -1), ora["idx"], ora["score"], np.array([n - 1]),
+                         wl.window, wl.topk)
+    assert st.ok(), (b, n, st.failures)
+
+
+@pytest.mark.parametrize("lens", [[40000, 777, 129, 12345, 1, 128, 1153], [300, 70000], [5000, 5000, 5000]])
+def test_decode_ragged_matches_each_sequence_alone(hs2, lens):
+    """Sequences of different cache lengths in one call: each equals the oracle on that sequence
+    alone; rows past a sequence's length are garbage the kernels must never read (NaN here)."""
+    B, Lk = len(lens), max(lens)
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=Lk))
+    q, k, v = to_torch_bf16(g.q), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    for b, n in enumerate(lens):
+        k[b, n:] = float("nan")
+        v[b, n:] = float("nan")
+    out, lse, idx = hs2.full_attn_select_ragged(q, k, v, lens, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    assert hs2.read_device_status(hs2.cached_workspace("full")) == 0
+    for b, n in enumerate(lens):
+        _check_seq(g, b, n, out, lse, idx)
+    # a sparse layer over the ragged selection reuses K, V and the GPU indices
+    qs = g.q_sparse(0)
+    o2 = hs2.sparse_attn(to_torch_bf16(qs), k, v, idx, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    ref = oracle.sparse_attn(qs, g.k, g.v, idx.cpu().numpy(), g.wl.scale)
+    assert_out_close(bf16_to_f64(o2).reshape(ref["out"].shape), ref["out"], "sparse layer over ragged selection")
+
+
+def test_decode_ragged_with_equal_lengths_is_the_batched_call(hs2):
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=3, Lk=20000))
+    q, k, v = to_torch_bf16(g.q), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    out1, lse1, idx1 = [t.clone() for t in hs2.full_attn_select(q, k, v, scale=g.wl.scale)]
+    out2, lse2, idx2 = hs2.full_attn_select_ragged(q, k, v, [20000] * 3, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2) and torch.equal(idx1, idx2)
+
+
+def test_decode_ragged_long_and_short_at_full_scale(hs2):
+    """One 262,144-token sequence next to short ones: the long sequence's work spreads over most
+    SMs while the short ones finish in one tile or a few."""
+    lens = [262144, 3000, 131072, 200]
+    B, Lk = len(lens), max(lens)
+    g = synth.SyntheticInputs(synth.small("decode_256k", B=B, Lk=Lk))
+    q, k, v = to_torch_bf16(g.q), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    out, lse, idx = hs2.full_attn_select_ragged(q, k, v, lens, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    assert hs2.read_device_status(hs2.cached_workspace("full")) == 0
+    for b, n in enumerate(lens):
+        _check_seq(g, b, n, out, lse, idx)
