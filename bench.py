@@ -288,6 +288,7 @@ def main():
     ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-ragged", action="store_true", help="skip the ragged-batch decode clause")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph of the steps")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (small profiling cases)")
@@ -476,6 +477,11 @@ def run_gpu(args):
     e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = _throughput(world, e2e_steps, e2e_ms)
 
+    # ---------------- ragged decode (a batch of different cache lengths in the same buffers)
+    ragged = None
+    if not args.no_ragged:
+        ragged = bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks)
+
     # ---------------- prefill (secondary clause of the metric)
     prefill = None
     if not args.no_prefill:
@@ -501,13 +507,73 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "note": "public Python API, pinned host inputs, result read every step"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
-            "device_status": [status, status_sp], "cpu_baseline": cpu, "prefill": prefill,
+            "device_status": [status, status_sp], "cpu_baseline": cpu, "ragged": ragged, "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+RAGGED_FRACTIONS = (1.0, 0.75, 0.5, 0.375, 0.25, 0.125, 0.0625, 0.015625)
+
+
+def bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks, steps=200, warmup=5):
+    """Decode steps over a ragged batch: sequence b keeps the first lens[b] rows of the bench's
+    cache (lengths from the full cache down to 1/64 of it), one hs2_full_attn_select_ragged plus
+    the sparse layers per step, as one CUDA graph; device-timed like the main line."""
+    import torch
+    lens = [max(1, int(wl.Lk * RAGGED_FRACTIONS[b % len(RAGGED_FRACTIONS)])) for b in range(wl.B)]
+    S = wl.window + wl.topk
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, 1, wl.H), dtype=torch.float32, device=q.device)
+    idx = torch.empty((wl.B, 1, S), dtype=torch.int32, device=q.device)
+    outs = [torch.empty_like(q) for _ in range(wl.n_sparse)]
+    ws = torch.zeros(hs2.full_attn_select_ragged_workspace_bytes(lens, wl.Lk, wl.H, wl.d), dtype=torch.uint8,
+                     device=q.device)
+    ws_sp = [torch.zeros(hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S), dtype=torch.uint8,
+                         device=q.device) for _ in range(wl.n_sparse)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hs2.full_attn_select_ragged(q, k, v, lens, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws)
+        for i in range(wl.n_sparse):
+            hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(steps):
+            hs2.profile_enable("dec_fused" if i % 8 == 0 else None)
+            step()
+        hs2.profile_enable(None)
+    graph.replay()            # upload and warm (the timing events of the replay below overwrite its own)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    _barrier(world)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    dec_ms, dec_n = hs2.profile_read("dec_fused")
+    status = hs2.read_device_status(ws)
+    del graph
+    dec_bytes = sum(n * wl.d * 2 * 2 + max(n - wl.window, 0) * 4 for n in lens)
+    dec_s = dec_ms / max(dec_n, 1) / 1e3
+    return {"workload": f"decode_ragged: B={wl.B} sequences of {lens} tokens in the {wl.Lk}-row cache buffers, "
+                        f"H={wl.H}, d={wl.d}, window {wl.window} + top-{wl.topk}, {wl.n_sparse} sparse layers",
+            "value": _throughput(world, steps, ms), "unit": "steps/s", "ms_per_step": ms / steps,
+            "tokens_per_step": sum(lens),
+            "roofline": {"kernel": "dec_fused", "bound": "hbm", "achieved": dec_bytes / dec_s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_bytes / dec_s / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": dec_s * 1e3,
+                         "launches_timed": dec_n},
+            "device_status": status}
 
 
 def bench_prefill(args, world, dev, peaks, reps=5, warmup=2):

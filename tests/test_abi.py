@@ -59,3 +59,25 @@ def test_workspace_queries_are_sane(B, Lk):
     assert n >= B * max(Lk - 128, 0) * 12
     assert hs2.full_attn_select_workspace_bytes(0, 1, Lk, 64, 128) == 0
     assert hs2.sparse_attn_workspace_bytes(B, 1, Lk, 64, 128, 1152) >= 256
+
+
+def test_ragged_workspace_query_and_argument_checks():
+    import long_context_mqa_b200 as hs2
+    lens = [262144, 3000, 1, 128, 129]
+    n = hs2.full_attn_select_ragged_workspace_bytes(lens, 262144, 64, 128)
+    # room for the longest sequence's older tokens in every row, at least
+    assert n >= len(lens) * (262144 - 128) * 12
+    # equal lengths: the batched call's workspace
+    assert hs2.full_attn_select_ragged_workspace_bytes([5000] * 3, 5000, 64, 128) == \
+        hs2.full_attn_select_workspace_bytes(3, 1, 5000, 64, 128)
+    L = hs2.lib
+    bad = (ctypes.c_int32 * 2)(10, 0)      # a length of 0
+    assert L.hs2_full_attn_select_ragged_workspace_bytes(2, bad, 100, 64, 128, 128, 1024) == 0
+    over = (ctypes.c_int32 * 2)(10, 101)   # longer than Lk
+    assert L.hs2_full_attn_select_ragged_workspace_bytes(2, over, 100, 64, 128, 128, 1024) == 0
+    many = (ctypes.c_int32 * 257)(*([10] * 257))  # more sequences than the schedule's tables hold
+    assert L.hs2_full_attn_select_ragged_workspace_bytes(257, many, 100, 64, 128, 128, 1024) == 0
+    assert L.hs2_full_attn_select_ragged(None, None, None, 2, bad, 100, 64, 128, 0.1, 128, 1024, None, None, None,
+                                         None, 0, None) == hs2.ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        hs2.full_attn_select_ragged_workspace_bytes([10, 0], 100, 64, 128)
