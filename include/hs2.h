@@ -86,8 +86,9 @@ HS2_API const char* hs2_status_string(hs2_status s);
  * Full attention + token selection
  * ---------------------------------------------------------------------------------
  * Q    [B, Lq, H, d] bf16  queries; query i sits at position t = Lk - Lq + i
- *                           (Lq == Lk: prefill over the whole sequence; Lq == 1: one decode
- *                           step whose own K/V row is already the last cache row)
+ *                           (Lq == Lk: prefill over the whole sequence; 1 < Lq < Lk: a chunk of
+ *                           Lq new tokens appended to an Lk - Lq token cache, whose K/V rows are
+ *                           already the last Lq cache rows; Lq == 1: one decode step)
  * K, V [B, Lk, d]    bf16  the single K/V head
  * scale                     softmax scale applied to q.k (e.g. 1/sqrt(d))
  * window, topk              forced recent tokens and number of older tokens chosen by score
@@ -96,9 +97,9 @@ HS2_API const char* hs2_status_string(hs2_status s);
  * lse  [B, Lq, H]    fp32  natural-log logsumexp of the scaled logits of the causal row
  * idx  [B, Lq, window+topk] int32  selected token indices of each query, ascending;
  *                           exactly min(t+1, window+topk) valid entries, then -1 padding
- * Supported: (H, d) in {(64, 128), (16, 64)}; Lq == 1 or Lq == Lk (bf16, fp32 accumulate).
- * Decode (Lq == 1) supports (H, d) = (64, 128) and B <= 256; prefill (Lq == Lk) supports
- * topk <= 1024.
+ * Supported: (H, d) in {(64, 128), (16, 64)}, 1 <= Lq <= Lk (bf16, fp32 accumulate). Lq == 1
+ * with (H, d) = (64, 128) runs the decode kernels (B <= 256); every other shape runs the prefill
+ * kernels, which support topk <= 1024.
  */
 HS2_API size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk);
 HS2_API hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk,

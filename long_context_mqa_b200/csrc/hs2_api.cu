@@ -284,7 +284,7 @@ void hs2_set_wait_limit_ns(long long limit_ns) { g_wait_ns = limit_ns > 0 ? limi
 size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk) {
   if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || d <= 0 || window < 1 || topk < 0) return 0;
   const int sms = num_sms() > 0 ? num_sms() : 148;
-  if (Lq == 1) {
+  if (Lq == 1 && H == 64 && d == 128) {  // the decode kernels
     if (B > dec::kMaxSeqs) return 0;
     std::vector<int> lens((size_t)B, Lk);
     return carve_decode(nullptr, B, lens.data(), Lk, H, d, window, topk, sms).bytes;
@@ -344,13 +344,13 @@ hs2_status hs2_full_attn_select(const hs2_bf16* Q, const hs2_bf16* K, const hs2_
   const int sms = num_sms();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float c = scale * 1.4426950408889634f;
-  if (Lq == 1) {
+  if (Lq == 1 && H == 64 && d == 128) {  // decode: one query per sequence
     if (B > dec::kMaxSeqs) return HS2_ERR_UNSUPPORTED_SHAPE;
     std::vector<int> lens((size_t)B, Lk);
     return run_decode(Q, K, V, B, lens.data(), Lk, H, d, c, window, topk, out, lse, idx, workspace, workspace_bytes,
                       sms, st);
   }
-  if (Lq != Lk) return HS2_ERR_UNSUPPORTED_SHAPE;
+  // a whole prompt (Lq == Lk) or a chunk of Lq queries appended to a cache (Lq < Lk)
   return prefill::run(Q, K, V, B, Lq, Lk, H, d, c, window, topk, out, lse, idx, workspace, workspace_bytes, sms,
                       kStatusBytes, st);
 }

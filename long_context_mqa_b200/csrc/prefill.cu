@@ -1,4 +1,5 @@
-// Prefill (Lq == Lk) full attention + token selection.
+// Prefill full attention + token selection: Lq queries at positions off + 0 .. off + Lq - 1
+// (off = Lk - Lq: Lq == Lk is a whole prompt, Lq < Lk a chunk appended to a cache).
 //
 // Pass 1, fa_fwd: causal MQA flash attention producing out and the per-(query, head) logsumexp.
 //   Rows of a 128-row tile are (query, head) pairs -- all heads of 128/H consecutive queries --
@@ -40,9 +41,10 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr int SOFT_EXP2 = 0;
 
 struct PfParams {
-  int B, L, H;
-  int rows_per_batch;   // L * H
-  int items_per_batch;  // ceil(L * H / 256)
+  int B, Lq, Lk, H;
+  int off;              // Lk - Lq: query i sits at position off + i
+  int rows_per_batch;   // Lq * H
+  int items_per_batch;  // ceil(Lq * H / 256)
   int n_items;
   float c;              // scale * log2(e)
   int W, K, S;
@@ -97,8 +99,8 @@ struct FaCfg {
 // key tiles an item covers: 0 .. last_tile
 __device__ __forceinline__ int fa_last_tile(const PfParams& p, int item_in_batch) {
   int t_hi = (item_in_batch * 256 + 255) / p.H;
-  if (t_hi > p.L - 1) t_hi = p.L - 1;
-  return t_hi / 128;
+  if (t_hi > p.Lq - 1) t_hi = p.Lq - 1;
+  return (p.off + t_hi) / 128;
 }
 
 template <int H, int D>
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(NT, 1)
       const int jt = fa_last_tile(p, ib);
       const int rloc = ib * 256 + w * 128 + row;      // row within the batch
       const bool valid_row = rloc < p.rows_per_batch;
-      const int t = rloc / H;
+      const int t = p.off + rloc / H;  // the row's query position
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j <= jt; ++j) {
         if (!warp_wait(&s_full[w], n_s & 1, limit, &abort_flag, p.st, 621)) { ok = false; break; }
@@ -381,8 +383,8 @@ __device__ __forceinline__ ScItem sc_item(const PfParams& p, int item, int nq) {
   s.b = item / p.items_per_batch;
   s.ib = item % p.items_per_batch;
   s.tq0 = s.ib * nq;
-  s.t_hi = s.tq0 + nq - 1 < p.L - 1 ? s.tq0 + nq - 1 : p.L - 1;
-  const int last_cand = s.t_hi - p.W;
+  s.t_hi = s.tq0 + nq - 1 < p.Lq - 1 ? s.tq0 + nq - 1 : p.Lq - 1;
+  const int last_cand = p.off + s.t_hi - p.W;  // the newest older key of the item's last query
   s.n_tiles = last_cand >= 0 ? last_cand / 128 + 1 : 0;
   return s;
 }
@@ -590,7 +592,7 @@ __global__ void __launch_bounds__(NT, 1)
       for (int x = wt; x < C::QW * H; x += 128) {
         const int q = wg * C::QW + x / H, h = x % H;
         const int t = si.tq0 + q;
-        const float l = t < p.L ? p.lse[((size_t)si.b * p.L + t) * H + h] : 0.f;
+        const float l = t < p.Lq ? p.lse[((size_t)si.b * p.Lq + t) * H + h] : 0.f;
         slse2[q * H + h] = -l * LOG2E;  // stored negated: one FFMA gives s*c - lse2
       }
       wg_bar(wg);
@@ -616,7 +618,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int qq = 0; qq < C::QW; ++qq) {
           const int q = wg * C::QW + qq;
           const int t = si.tq0 + q;
-          const bool cand = t < p.L && key <= t - p.W;
+          const bool cand = t < p.Lq && key <= p.off + t - p.W;
           if (!__any_sync(0xffffffffu, cand)) continue;  // warp-uniform: no lane has a candidate here
           // the exponentials can be shared between the MUFU (ex2) and the FMA pipes (exp2_fma2);
           // four independent pairs of partial sums keep the additions off one dependency chain
@@ -670,7 +672,8 @@ __global__ void __launch_bounds__(NT, 1)
       for (int qq = 0; qq < C::QW; ++qq) {
         const int q = wg * C::QW + qq;
         const int t = si.tq0 + q;
-        if (t >= p.L) continue;  // uniform across the warpgroup
+        if (t >= p.Lq) continue;  // uniform across the warpgroup
+        const int pos = p.off + t;  // the query's position
         const int n = cnt[q];
         const int keep = n < p.K ? n : p.K;
         unsigned long long* qb = cbuf + (size_t)q * C::CAP;
@@ -685,8 +688,8 @@ __global__ void __launch_bounds__(NT, 1)
         }
         wg_bar(wg);
         int* ib32 = reinterpret_cast<int*>(qb);
-        const int wlo = t - p.W + 1 > 0 ? t - p.W + 1 : 0;
-        const int wlen = t - wlo + 1;
+        const int wlo = pos - p.W + 1 > 0 ? pos - p.W + 1 : 0;
+        const int wlen = pos - wlo + 1;
         // the picks (<= topk <= 1024) are sorted; the window t-W+1..t follows them, all larger
 #pragma unroll
         for (int m2 = 0; m2 < 1024 / 128; ++m2) {
@@ -707,7 +710,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
         const int total = keep + wlen;
-        int32_t* dst = p.idx + ((size_t)si.b * p.L + t) * p.S;
+        int32_t* dst = p.idx + ((size_t)si.b * p.Lq + t) * p.S;
         for (int i = wt; i < p.S; i += 128) dst[i] = i < keep ? ib32[i] : (i < total ? wlo + (i - keep) : -1);
         wg_bar(wg);
       }
@@ -724,23 +727,24 @@ __global__ void __launch_bounds__(NT, 1)
 size_t workspace_bytes(int, int, int, int, int, int, int, int, size_t status_bytes) { return status_bytes; }
 
 template <int H, int D>
-static hs2_status run_t(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int L, float c, int window,
-                        int topk, hs2_bf16* out, float* lse, int32_t* idx, DevStatus* st, int sms,
+static hs2_status run_t(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk, float c,
+                        int window, int topk, hs2_bf16* out, float* lse, int32_t* idx, DevStatus* st, int sms,
                         cudaStream_t stream) {
   using FC = FaCfg<H, D>;
   using SC = ScCfg<H, D>;
   if (topk > SC::CAP - 128 || topk > 1024) return HS2_ERR_UNSUPPORTED_SHAPE;  // picks are sorted in 1024 slots
-  const long long rows_total = (long long)B * L * H;
+  const long long rows_total = (long long)B * Lq * H;
   if (rows_total >= (1LL << 31)) return HS2_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tmQ1, tmQ2, tmK, tmV;
   if (!make_tmap_2d(&tmQ1, Q, D, rows_total, D, 64, 128) || !make_tmap_2d(&tmQ2, Q, D, rows_total, D, 64, 256) ||
-      !make_tmap_3d(&tmK, K, D, L, B, D, (uint64_t)L * D, 64, 128) ||
-      !make_tmap_3d(&tmV, V, D, L, B, D, (uint64_t)L * D, 64, 128))
+      !make_tmap_3d(&tmK, K, D, Lk, B, D, (uint64_t)Lk * D, 64, 128) ||
+      !make_tmap_3d(&tmV, V, D, Lk, B, D, (uint64_t)Lk * D, 64, 128))
     return HS2_ERR_CUDA;
   PfParams p;
-  p.B = B; p.L = L; p.H = H;
-  p.rows_per_batch = L * H;
-  p.items_per_batch = (L * H + 255) / 256;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = H;
+  p.off = Lk - Lq;
+  p.rows_per_batch = Lq * H;
+  p.items_per_batch = (Lq * H + 255) / 256;
   p.n_items = B * p.items_per_batch;
   p.c = c;
   p.W = window; p.K = topk; p.S = window + topk;
@@ -770,11 +774,11 @@ static hs2_status run_t(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
 hs2_status run(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lq, int Lk, int H, int d, float c,
                int window, int topk, hs2_bf16* out, float* lse, int32_t* idx, void* ws, size_t ws_bytes, int sms,
                size_t status_bytes, cudaStream_t stream) {
-  if (Lq != Lk) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (Lq < 1 || Lq > Lk) return HS2_ERR_UNSUPPORTED_SHAPE;
   if (ws_bytes < status_bytes) return HS2_ERR_WORKSPACE;
   DevStatus* st = reinterpret_cast<DevStatus*>(ws);
-  if (H == 64 && d == 128) return run_t<64, 128>(Q, K, V, B, Lq, c, window, topk, out, lse, idx, st, sms, stream);
-  if (H == 16 && d == 64) return run_t<16, 64>(Q, K, V, B, Lq, c, window, topk, out, lse, idx, st, sms, stream);
+  if (H == 64 && d == 128) return run_t<64, 128>(Q, K, V, B, Lq, Lk, c, window, topk, out, lse, idx, st, sms, stream);
+  if (H == 16 && d == 64) return run_t<16, 64>(Q, K, V, B, Lq, Lk, c, window, topk, out, lse, idx, st, sms, stream);
   return HS2_ERR_UNSUPPORTED_SHAPE;
 }
 

@@ -1,4 +1,5 @@
-"""GPU parity of the prefill path (Lq == Lk) and of the KV Bridging GEMM against the fp64 oracle."""
+"""GPU parity of the prefill path (Lq == Lk, and chunks Lq < Lk appended to a cache) and of the KV
+Bridging GEMM against the fp64 oracle."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +36,7 @@ def _check(g, out, lse, idx, rows):
     glse = lse.double().cpu().numpy().reshape(wl.B * wl.Lq, wl.H)[rows]
     assert np.abs(glse - ora["lse"]).max() < 2e-3
     gidx = idx.cpu().numpy().reshape(wl.B * wl.Lq, -1)[rows]
-    st = check_selection(gidx, ora["idx"], ora["score"], rows % wl.Lq, wl.window, wl.topk)
+    st = check_selection(gidx, ora["idx"], ora["score"], wl.Lk - wl.Lq + rows % wl.Lq, wl.window, wl.topk)
     assert st.ok(), st.failures
     return st
 
@@ -119,3 +120,28 @@ def test_bridge_full_size_sampled(hs2):
                                      [wl.bridge_T - 1]]))
     ref = oracle.bridge_kv_proj(g.bridge_h, g.bridge_w, rows=rows)
     _bridge_check(bf16_to_f64(kv)[:, :, rows], ref)
+
+
+@pytest.mark.parametrize("B,Lq,Lk", [(1, 700, 3000), (2, 256, 1500), (1, 2, 5000), (1, 1299, 1300), (2, 129, 1152)])
+def test_chunked_prefill_h64_all_rows(hs2, B, Lq, Lk):
+    """A chunk of Lq queries appended to a cache of Lk - Lq tokens: query i at position Lk - Lq + i,
+    every row against the oracle, and a sparse layer over the chunk's selection."""
+    wl = synth.small("prefill_32k", B=B, Lq=Lq, Lk=Lk)
+    g = synth.SyntheticInputs(wl)
+    q, k, v, out, lse, idx = _prefill(hs2, g)
+    _check(g, out, lse, idx, np.arange(B * Lq))
+    qs = g.q_sparse(0)
+    o2 = hs2.sparse_attn(to_torch_bf16(qs), k, v, idx, scale=wl.scale)
+    torch.cuda.synchronize()
+    ref = oracle.sparse_attn(qs, g.k, g.v, idx.cpu().numpy(), wl.scale)
+    assert_out_close(bf16_to_f64(o2).reshape(ref["out"].shape), ref["out"], "sparse layer over a chunk")
+
+
+@pytest.mark.parametrize("Lq", [300, 1])
+def test_chunked_prefill_tiny_config(hs2, Lq):
+    """16 heads, head_dim 64: a chunk (and a single query, which these shapes run on the prefill
+    kernels) against a 2048-token cache."""
+    wl = synth.small("tiny_prefill", Lq=Lq, Lk=2048)
+    g = synth.SyntheticInputs(wl)
+    _, _, _, out, lse, idx = _prefill(hs2, g)
+    _check(g, out, lse, idx, np.arange(Lq))
