@@ -639,6 +639,31 @@ def bench_prefill(args, world, dev, peaks, reps=5, warmup=2):
         sp_tf = sp_flops / (kern["sparse_attn_per_layer"] / 1e3) / 1e12
         res["sparse_roofline"] = {"bound": "tensor", "achieved": sp_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": sp_tf / peaks["bf16_tflops"], "flops": "4*H*d*S*L per layer"}
+    if not args.prefill_len:
+        # chunked prefill: the last CHUNK queries of the same prompt appended to the cache of the
+        # first L - CHUNK tokens (query i at position L - CHUNK + i), same K/V buffers
+        CHUNK = 4096
+        qc = q[:, -CHUNK:]
+        oc = torch.empty_like(qc)
+        lc = torch.empty((1, CHUNK, wl.H), dtype=torch.float32, device=dev)
+        ic = torch.empty((1, CHUNK, wl.window + wl.topk), dtype=torch.int32, device=dev)
+        for _ in range(warmup):
+            hs2.full_attn_select(qc, k, v, scale=wl.scale, out=oc, lse=lc, idx=ic)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(s)
+        for _ in range(reps):
+            hs2.full_attn_select(qc, k, v, scale=wl.scale, out=oc, lse=lc, idx=ic)
+        c1.record(s)
+        c1.synchronize()
+        cms = _max_over_ranks(c0.elapsed_time(c1), world) / reps
+        off = wl.Lk - CHUNK
+        cP = CHUNK * off + CHUNK * (CHUNK + 1) / 2   # (query, key) pairs of the chunk
+        ctf = 6 * wl.H * wl.d * cP / (cms / 1e3) / 1e12
+        res["chunk"] = {"workload": f"{CHUNK} queries appended to a {off}-token cache (H={wl.H}, d={wl.d})",
+                        "tok_per_s": world * CHUNK / (cms / 1e3), "ms": cms,
+                        "roofline": {"bound": "tensor", "achieved": ctf, "peak": peaks["bf16_tflops_sustained"],
+                                     "unit": "TFLOP/s", "frac": ctf / peaks["bf16_tflops_sustained"],
+                                     "flops": "executed 6*H*d*(pairs of the chunk's causal rows)"}}
     if wl.bridge_T and not args.prefill_len:
         # KV Bridging: one batched GEMM H[T x hidden] . [W_k^l | W_v^l ...]
         hb = _bf16(g.bridge_h, dev)
