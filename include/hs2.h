@@ -124,6 +124,24 @@ HS2_API hs2_status hs2_full_attn_select_ragged(const hs2_bf16* Q, const hs2_bf16
                                                int topk, hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
                                                size_t workspace_bytes, hs2_stream stream);
 
+/* Paged decode: as the ragged call, with each sequence's cache in pages of 128 tokens of shared
+ * pools (a serving system's block-allocated KV cache).
+ * K_pages, V_pages [n_pages, 128, d] bf16  the page pools
+ * page_table [B, max_pages] int32 (DEVICE)  page of sequence b's tokens 128 i .. 128 i + 127; only
+ *                           the first ceil(lens[b] / 128) entries of a row are read; an id outside
+ *                           [0, n_pages) is recorded as HS2_ERR_DEVICE_BOUNDS (its rows read as 0)
+ * lens [B] int32 (HOST)     1 <= lens[b] <= 128 * max_pages
+ * Rows of a sequence's last page past lens[b] are never used. The results equal the ragged call
+ * on the same tokens laid out contiguously. Supported: (H, d) = (64, 128), 1 <= B <= 256.
+ */
+HS2_API size_t hs2_full_attn_select_paged_workspace_bytes(int B, const int32_t* lens, int max_pages, int H, int d,
+                                                          int window, int topk);
+HS2_API hs2_status hs2_full_attn_select_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, const hs2_bf16* V_pages,
+                                              int n_pages, const int32_t* page_table, int max_pages, int B,
+                                              const int32_t* lens, int H, int d, float scale, int window, int topk,
+                                              hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                              size_t workspace_bytes, hs2_stream stream);
+
 /* ---------------------------------------------------------------------------------
  * Sparse attention over selected tokens (one sparse layer)
  * ---------------------------------------------------------------------------------
@@ -141,6 +159,16 @@ HS2_API size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int
 HS2_API hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
                            int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
                            void* workspace, size_t workspace_bytes, hs2_stream stream);
+/* Sparse attention over a paged cache: K_pages, V_pages, page_table, max_pages and n_pages as for
+ * hs2_full_attn_select_paged; idx [B, Lq, S] holds token positions (< 128 * max_pages) of each
+ * sequence, mapped through its page-table row. Workspace: hs2_sparse_attn_workspace_bytes with
+ * Lk = 128 * max_pages. An out-of-pool page id is recorded as HS2_ERR_DEVICE_BOUNDS and its token
+ * skipped.
+ */
+HS2_API hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, const hs2_bf16* V_pages,
+                                         int n_pages, const int32_t* page_table, int max_pages, const int32_t* idx,
+                                         int B, int Lq, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * Sparse attention without a caller workspace

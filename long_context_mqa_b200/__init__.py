@@ -57,6 +57,12 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_full_attn_select_ragged_workspace_bytes.restype = sz
     lib.hs2_full_attn_select_ragged.argtypes = [P, P, P, i32, P, i32, i32, i32, f32, i32, i32, P, P, P, P, sz, P]
     lib.hs2_full_attn_select_ragged.restype = i32
+    lib.hs2_full_attn_select_paged_workspace_bytes.argtypes = [i32, P, i32, i32, i32, i32, i32]
+    lib.hs2_full_attn_select_paged_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select_paged.argtypes = [P, P, P, i32, P, i32, i32, P, i32, i32, f32, i32, i32, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_paged.restype = i32
+    lib.hs2_sparse_attn_paged.argtypes = [P, P, P, i32, P, i32, P, i32, i32, i32, i32, i32, f32, P, P, P, sz, P]
+    lib.hs2_sparse_attn_paged.restype = i32
     lib.hs2_sparse_attn_workspace_bytes.argtypes = [i32] * 6
     lib.hs2_sparse_attn_workspace_bytes.restype = sz
     lib.hs2_sparse_attn.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, sz, P]
@@ -207,6 +213,66 @@ def full_attn_select_ragged(q, k, v, lens, *, scale=None, window=WINDOW, topk=TO
                                            ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(code, "hs2_full_attn_select_ragged")
     return out, lse, idx
+
+
+def full_attn_select_paged_workspace_bytes(lens, max_pages, H, d, window=WINDOW, topk=TOPK) -> int:
+    B = len(lens)
+    return int(lib.hs2_full_attn_select_paged_workspace_bytes(B, _lens_array(lens, B, max_pages * 128), max_pages, H, d,
+                                                              window, topk))
+
+
+def full_attn_select_paged(q, k_pages, v_pages, page_table, lens, *, scale=None, window=WINDOW, topk=TOPK, out=None,
+                           lse=None, idx=None, workspace=None, stream=None):
+    """Decode over a paged cache (hs2_full_attn_select_paged).
+
+    q [B,1,H,d]; k_pages, v_pages [n_pages,128,d]; page_table [B,max_pages] int32 on the device;
+    lens: B host integers. Returns (out, lse, idx) as full_attn_select_ragged.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_pages, "k_pages", torch.bfloat16, 3)
+    _need(v_pages, "v_pages", torch.bfloat16, 3)
+    _need(page_table, "page_table", torch.int32, 2)
+    B, Lq, H, d = q.shape
+    n_pages = k_pages.shape[0]
+    max_pages = page_table.shape[1]
+    if Lq != 1 or tuple(k_pages.shape) != (n_pages, 128, d) or v_pages.shape != k_pages.shape or page_table.shape[0] != B:
+        raise ValueError("q [B,1,H,d], k_pages/v_pages [n_pages,128,d], page_table [B,max_pages]")
+    lens_c = _lens_array(list(lens), B, max_pages * 128)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = window + topk
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, 1, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, 1, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    nbytes = int(lib.hs2_full_attn_select_paged_workspace_bytes(B, lens_c, max_pages, H, d, window, topk))
+    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    code = lib.hs2_full_attn_select_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), n_pages,
+                                          page_table.data_ptr(), max_pages, B, lens_c, H, d, scale, window, topk,
+                                          out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                          ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select_paged")
+    return out, lse, idx
+
+
+def sparse_attn_paged(q, k_pages, v_pages, page_table, idx, *, scale=None, out=None, workspace=None, stream=None):
+    """Sparse attention over a paged cache (hs2_sparse_attn_paged); idx [B,Lq,S] token positions."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_pages, "k_pages", torch.bfloat16, 3)
+    _need(v_pages, "v_pages", torch.bfloat16, 3)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(idx, "idx", torch.int32, 3)
+    B, Lq, H, d = q.shape
+    S = idx.shape[2]
+    n_pages, max_pages = k_pages.shape[0], page_table.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    nbytes = sparse_attn_workspace_bytes(B, Lq, max_pages * 128, H, d, S)
+    ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
+    code = lib.hs2_sparse_attn_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), n_pages,
+                                     page_table.data_ptr(), max_pages, idx.data_ptr(), B, Lq, H, d, S, scale,
+                                     out.data_ptr(), None, ws.data_ptr(), ws.numel() * ws.element_size(),
+                                     _stream_ptr(stream))
+    _check(code, "hs2_sparse_attn_paged")
+    return out
 
 
 def sparse_attn(q, k, v, idx, *, scale=None, out=None, lse=None, want_lse=False, workspace=None, stream=None):

@@ -86,6 +86,30 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
   m = mx;
 }
 
+// Page ids of a run of n tiles lt0, lt0 + step, ... of sequence b from a page table
+// [B][max_pages] (a contiguous cache: no table, every id -1). Each id is read 4 tiles before the
+// producer needs it, so the table's latency hides behind the ring's waits.
+struct PageRun {
+  const int32_t* row;
+  int lt, step, left, v0, v1, v2, v3;
+  __device__ __forceinline__ int load(int k) const {
+    return row && k < left ? __ldg(row + lt + k * step) : -1;
+  }
+  __device__ __forceinline__ void start(const int32_t* ptab, int max_pages, int b, int lt0, int st, int n) {
+    row = ptab ? ptab + (size_t)b * max_pages : nullptr;
+    lt = lt0; step = st; left = n;
+    v0 = load(0); v1 = load(1); v2 = load(2); v3 = load(3);
+  }
+  __device__ __forceinline__ int next() {
+    const int r = v0;
+    v0 = v1; v1 = v2; v2 = v3;
+    v3 = load(4);
+    lt += step;
+    --left;
+    return r;
+  }
+};
+
 // the first phase-1 (sampled) tile at or after local tile lt
 __device__ __forceinline__ int first_sample(int lt, int st) { return (lt + st - 1) / st * st; }
 // phase 1 of sequence b takes every st-th tile: about `target` tiles (every tile when target is 0)
@@ -168,15 +192,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++nq;
         return true;
       };
-      auto load_tile = [&](const CUtensorMap* m, int lt, int b, uint64_t pol) -> bool {
+      // tile lt of sequence b: rows lt*128.. of its cache, or (paged cache) page `pg`, whose 128
+      // rows are the third tensor-map coordinate's slice (an id outside the pool reads zeros)
+      auto load_tile = [&](const CUtensorMap* m, int lt, int b, uint64_t pol, int pg) -> bool {
         const int s = ri % RING;
         if (!wait_bar(&r_empty[s], ((ri / RING) & 1) ^ 1, limit, &abort_flag, p.st, 202)) return false;
         mbar_expect_tx(&r_full[s], KT_BYTES);
+        if (p.ptab && (pg < 0 || pg >= p.n_pages)) report_status(p.st, kStatusBounds, 203);  // reads zeros
+        const int c1 = p.ptab ? 0 : lt * TILE, c2 = p.ptab ? pg : b;
         for (int kb = 0; kb < NKB; ++kb)
-          tma_load_3d_hint(sR + s * KT_BYTES + kb * (TILE * 128), m, &r_full[s], kb * 64, lt * TILE, b, pol);
+          tma_load_3d_hint(sR + s * KT_BYTES + kb * (TILE * 128), m, &r_full[s], kb * 64, c1, c2, pol);
         ++ri;
         return true;
       };
+      // page ids of a run of tiles lt0, lt0 + step, ... (count n), read 4 ahead of their use
+      PageRun pr;
       for (int g = 0; g < S.n_groups && ok; ++g) {
         long long t0, t1;
         S.range(g, cta, t0, t1);
@@ -186,8 +216,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (skip_seq(b)) { t = seg_end; continue; }
           if (!load_q(b)) { ok = false; break; }
           const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
-          for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi && ok; lt += st)
-            if (!load_tile(&tmK, lt, b, keep)) ok = false;
+          const int lt0 = first_sample((int)(t - (long long)S.seq_start[b]), st);
+          pr.start(p.ptab, p.max_pages, b, lt0, st, lt0 < lt_hi ? (lt_hi - 1 - lt0) / st + 1 : 0);
+          for (int lt = lt0; lt < lt_hi && ok; lt += st)
+            if (!load_tile(&tmK, lt, b, keep, pr.next())) ok = false;
           t = seg_end;
         }
         for (long long t = t1 - 1; t >= t0 && ok;) {  // phase 2: descending
@@ -198,12 +230,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // in the order the tensor core consumes them: S of a tile needs its K, then the PV of
           // the tile before it (the next higher one) needs that tile's V
           const long long seg_hi = t;
+          pr.start(p.ptab, p.max_pages, b, (int)(seg_hi - (long long)S.seq_start[b]), -1, (int)(seg_hi - seg_lo + 1));
+          int pg_prev = -1;  // the page of tile lt + 1 (its V follows this tile's K)
           for (; t >= seg_lo; --t) {
             const int lt = (int)(t - (long long)S.seq_start[b]);
-            if (!load_tile(&tmK, lt, b, once)) { ok = false; break; }
-            if (t < seg_hi && !load_tile(&tmV, lt + 1, b, once)) { ok = false; break; }
+            const int pg = pr.next();
+            if (!load_tile(&tmK, lt, b, once, pg)) { ok = false; break; }
+            if (t < seg_hi && !load_tile(&tmV, lt + 1, b, once, pg_prev)) { ok = false; break; }
+            pg_prev = pg;
           }
-          if (ok && !load_tile(&tmV, (int)(seg_lo - (long long)S.seq_start[b]), b, once)) { ok = false; break; }
+          if (ok && !load_tile(&tmV, (int)(seg_lo - (long long)S.seq_start[b]), b, once, pg_prev)) { ok = false; break; }
         }
       }
       if (!ok) {  // let the copies already issued land before the CTA exits

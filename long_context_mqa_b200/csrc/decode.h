@@ -37,6 +37,8 @@ struct DecParams {
   float* lse2x;            // [B][H] exact lse, log2 units (for the exact re-score of the band)
   int* ovf;                // [B + 1] sequences whose p' overflowed the sampled reference (and a count)
   int fallback;            // 0: the sampled schedule; 1: redo the flagged sequences with every tile
+  const int32_t* ptab;     // paged cache: [B][max_pages] page of each 128-token tile (NULL: contiguous)
+  int max_pages, n_pages;  // table width, pages in the K/V pools
   DevStatus* st;
 };
 size_t fused_smem_bytes(int H, int D);
@@ -74,6 +76,8 @@ struct SelParams {
   float c;                       // scale * log2(e)
   int sms;
   unsigned* gbar;                // the decode kernel's grid-barrier counters, re-armed here
+  const int32_t* ptab;           // paged cache: [B][max_pages] page ids, kc is the page pool (NULL: contiguous)
+  int max_pages, n_pages;
   long long wait_ns;             // bound of the re-score kernel's wait for its MMA
 };
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
@@ -90,6 +94,8 @@ struct SpParams {
   __nv_bfloat16* out;
   float* lse;                 // may be null
   long long wait_ns;
+  const int32_t* ptab;        // paged cache: [B][max_pages] page ids, K/V are the page pools of
+  int max_pages, n_pages;     // n_pages x 128 rows (NULL: K/V are [B][Lk] rows)
   DevStatus* st;
 };
 size_t sparse_smem_bytes(int H, int D, int nsplit);

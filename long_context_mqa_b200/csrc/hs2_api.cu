@@ -292,10 +292,12 @@ size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d,
   return prefill::workspace_bytes(B, Lq, Lk, H, d, window, topk, sms, kStatusBytes);
 }
 
-// The decode path (one query per sequence at the end of its lens[b]-token cache).
+// The decode path (one query per sequence at the end of its lens[b]-token cache). K, V are
+// [B][Lk] rows, or (ptab != NULL) pools of n_pages pages of 128 rows with Lk = max_pages * 128.
 static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, const int* lens, int Lk,
                              int H, int d, float c, int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
-                             void* workspace, size_t workspace_bytes, int sms, cudaStream_t st) {
+                             void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
+                             const int32_t* ptab = nullptr, int max_pages = 0, int n_pages = 0) {
   if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
   DecodeWs w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
   if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
@@ -303,9 +305,14 @@ static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf1
   w.p.c = c;
   w.p.wait_ns = wait_limit_ns();
   w.p.lse_out = lse;
+  w.p.ptab = ptab;
+  w.p.max_pages = max_pages;
+  w.p.n_pages = n_pages;
+  // contiguous: (d, Lk rows, B sequences); paged: (d, 128 rows, n_pages pages)
+  const uint64_t rows = ptab ? 128 : (uint64_t)Lk, planes = ptab ? (uint64_t)n_pages : (uint64_t)B;
   CUtensorMap tmK, tmV, tmQ;
-  if (!make_tmap_3d(&tmK, K, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
-      !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+  if (!make_tmap_3d(&tmK, K, d, rows, planes, d, rows * d, 64, 128) ||
+      !make_tmap_3d(&tmV, V, d, rows, planes, d, rows * d, 64, 128) ||
       !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
     return HS2_ERR_CUDA;
   if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, st) != cudaSuccess) return HS2_ERR_CUDA;
@@ -318,6 +325,9 @@ static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf1
   sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
   sp.lse2x = w.p.lse2x;
   sp.gbar = w.p.gbar;
+  sp.ptab = ptab;
+  sp.max_pages = max_pages;
+  sp.n_pages = n_pages;
   sp.c = c;
   sp.sms = sms;
   sp.wait_ns = w.p.wait_ns;
@@ -388,15 +398,46 @@ hs2_status hs2_full_attn_select_ragged(const hs2_bf16* Q, const hs2_bf16* K, con
                     topk, out, lse, idx, workspace, workspace_bytes, num_sms(), reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t hs2_full_attn_select_paged_workspace_bytes(int B, const int32_t* lens, int max_pages, int H, int d,
+                                                  int window, int topk) {
+  if (max_pages <= 0 || max_pages > (1 << 23)) return 0;
+  return hs2_full_attn_select_ragged_workspace_bytes(B, lens, max_pages * 128, H, d, window, topk);
+}
+
+hs2_status hs2_full_attn_select_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, const hs2_bf16* V_pages,
+                                      int n_pages, const int32_t* page_table, int max_pages, int B,
+                                      const int32_t* lens, int H, int d, float scale, int window, int topk,
+                                      hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                      size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K_pages || !V_pages || !page_table || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(idx) || (reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
+    return HS2_ERR_INVALID_ARG;
+  if (n_pages <= 0 || max_pages <= 0 || max_pages > (1 << 23) || window < 1 || topk < 0 || !(scale > 0.f))
+    return HS2_ERR_INVALID_ARG;
+  const int Lk = max_pages * 128;
+  if (!lens || B <= 0) return HS2_ERR_INVALID_ARG;
+  if (B > dec::kMaxSeqs) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!ragged_lens_ok(B, lens, Lk)) return HS2_ERR_INVALID_ARG;
+  if (window + topk > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  return run_decode(Q, K_pages, V_pages, B, reinterpret_cast<const int*>(lens), Lk, H, d,
+                    scale * 1.4426950408889634f, window, topk, out, lse, idx, workspace, workspace_bytes, num_sms(),
+                    reinterpret_cast<cudaStream_t>(stream), page_table, max_pages, n_pages);
+}
+
 size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int d, int S) {
   if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || d <= 0 || S <= 0) return 0;
   const int sms = num_sms() > 0 ? num_sms() : 148;
   return carve_sparse(nullptr, B, Lq, H, d, S, sms, nullptr);
 }
 
-hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
-                           int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
-                           void* workspace, size_t workspace_bytes, hs2_stream stream) {
+static hs2_status run_sparse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
+                             int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
+                             void* workspace, size_t workspace_bytes, hs2_stream stream, const int32_t* ptab,
+                             int max_pages, int n_pages) {
   if (!Q || !K || !V || !idx || !out) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (lse && !aligned16(lse)))
     return HS2_ERR_INVALID_ARG;
@@ -420,8 +461,28 @@ hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16*
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.wait_ns = wait_limit_ns();
+  p.ptab = ptab;
+  p.max_pages = max_pages;
+  p.n_pages = n_pages;
   if (sparse::launch_sparse(p, H, d, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HS2_ERR_CUDA;
   return HS2_OK;
+}
+
+hs2_status hs2_sparse_attn(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
+                           int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
+                           void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  return run_sparse(Q, K, V, idx, B, Lq, Lk, H, d, S, scale, out, lse, workspace, workspace_bytes, stream, nullptr,
+                    0, 0);
+}
+
+hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, const hs2_bf16* V_pages, int n_pages,
+                                 const int32_t* page_table, int max_pages, const int32_t* idx, int B, int Lq, int H,
+                                 int d, int S, float scale, hs2_bf16* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, hs2_stream stream) {
+  if (!page_table || (reinterpret_cast<uintptr_t>(page_table) & 3u) != 0) return HS2_ERR_INVALID_ARG;
+  if (n_pages <= 0 || max_pages <= 0 || max_pages > (1 << 23)) return HS2_ERR_INVALID_ARG;
+  return run_sparse(Q, K_pages, V_pages, idx, B, Lq, max_pages * 128, H, d, S, scale, out, lse, workspace,
+                    workspace_bytes, stream, page_table, max_pages, n_pages);
 }
 
 size_t hs2_bridge_kv_proj_workspace_bytes(int T, int hidden, int n_layers, int d) {

@@ -176,16 +176,26 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
     const int slot = tile * TILE + tid;
     const bool in = slot < n_band;
     const int j = in ? (int)(uint32_t)p.bnd[(size_t)b * p.ncand + slot] : 0;
-    const bool valid = in && j >= 0 && j < p.sch.seq_len[b] - p.W;
+    bool valid = in && j >= 0 && j < p.sch.seq_len[b] - p.W;
+    // the K row of key j: row j of sequence b's cache, or (paged) row j % 128 of its page
+    long long krow = -1;
+    if (valid) {
+      if (p.ptab) {
+        const int pg = __ldg(p.ptab + (size_t)b * p.max_pages + (j >> 7));
+        if (pg >= 0 && pg < p.n_pages) krow = (long long)pg * 128 + (j & 127);
+        else { valid = false; report_status(p.st, kStatusBounds, 313); }
+      } else {
+        krow = (long long)b * p.N + j;
+      }
+    }
     {
-      const __nv_bfloat16* kb = p.kc + (size_t)b * p.N * D;
-      const int jv = valid ? j : -1, sub = lane >> 4, ch = lane & 15;
+      const int sub = lane >> 4, ch = lane & 15;
 #pragma unroll
       for (int it = 0; it < 16; ++it) {
         const int rr = 2 * it + sub;  // row within this warp's 32
-        const int jr = __shfl_sync(0xffffffffu, jv, rr);
+        const long long kr = __shfl_sync(0xffffffffu, krow, rr);
         cp_async_16(smem_u32(sK) + (ch / 8) * (TILE * 128) + sw128_off(warp * 32 + rr, ch % 8),
-                    kb + (size_t)(jr >= 0 ? jr : 0) * D + ch * 8, jr >= 0);
+                    p.kc + (size_t)(kr >= 0 ? kr : 0) * D + ch * 8, kr >= 0);
       }
     }
     cp_async_commit();

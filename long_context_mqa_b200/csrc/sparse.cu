@@ -73,8 +73,9 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   if (slot1 > p.S) slot1 = p.S;
   const int ntiles = (slot1 - slot0 + TILE - 1) / TILE;
   const int32_t* idx_row = p.idx + (size_t)r * p.S;
-  const __nv_bfloat16* Kb = p.K + (size_t)b * p.Lk * D;
-  const __nv_bfloat16* Vb = p.V + (size_t)b * p.Lk * D;
+  // the rows of this row's sequence (contiguous cache) or the page pools (paged cache)
+  const __nv_bfloat16* Kb = p.ptab ? p.K : p.K + (size_t)b * p.Lk * D;
+  const __nv_bfloat16* Vb = p.ptab ? p.V : p.V + (size_t)b * p.Lk * D;
   const uint32_t tS = 0, tO = 128;
   const int prow = warp * 16 + (lane & 15);  // the row this lane's pair works on
   const int head = warp * 16 + lane;         // the head row this thread owns (lanes 0..15)
@@ -110,9 +111,19 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     const int slot = slot0 + t * TILE + tid;
     int j = -1;
     if (slot < slot1) j = idx_row[slot];
-    const bool valid = j >= 0 && j < p.Lk;
+    bool valid = j >= 0 && j < p.Lk;
+    // the row of token j: row j of the sequence's cache, or (paged) row j % 128 of its page
+    long long krow = -1;
+    if (valid) {
+      if (p.ptab) {
+        const int pg = __ldg(p.ptab + (size_t)b * p.max_pages + (j >> 7));
+        valid = pg >= 0 && pg < p.n_pages;
+        krow = valid ? (long long)pg * 128 + (j & 127) : -1;
+      } else {
+        krow = j;
+      }
+    }
     if (j != -1 && !valid) bad = true;
-    const int jv = valid ? j : -1;
     const unsigned m = __ballot_sync(0xffffffffu, valid);
     if (lane == 0) vmask[warp] = m;
     const uint32_t kd = smem_u32(sK), vd = smem_u32(sV);
@@ -120,11 +131,11 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
 #pragma unroll
     for (int it = 0; it < 32 / RPS; ++it) {
       const int rr = it * RPS + sub;  // row within this warp's 32
-      const int jr = __shfl_sync(0xffffffffu, jv, rr);
+      const long long kr = __shfl_sync(0xffffffffu, krow, rr);
       const uint32_t off = (ch / 8) * (TILE * 128) + sw128_off(warp * 32 + rr, ch % 8);
-      const size_t src = (size_t)(jr >= 0 ? jr : 0) * D + ch * 8;
-      cp_async_16(kd + off, Kb + src, jr >= 0);
-      cp_async_16(vd + off, Vb + src, jr >= 0);
+      const size_t src = (size_t)(kr >= 0 ? kr : 0) * D + ch * 8;
+      cp_async_16(kd + off, Kb + src, kr >= 0);
+      cp_async_16(vd + off, Vb + src, kr >= 0);
     }
     cp_async_commit();
   };

@@ -161,3 +161,66 @@ def test_decode_ragged_long_and_short_at_full_scale(hs2):
     assert hs2.read_device_status(hs2.cached_workspace("full")) == 0
     for b, n in enumerate(lens):
         _check_seq(g, b, n, out, lse, idx)
+
+
+def _paged_layout(g, lens, seed=7, spare=5):
+    """The synthetic cache of each sequence copied into randomly placed 128-token pages of shared
+    pools; page tails past a sequence and spare pages hold NaN, unused table entries an id far
+    outside the pool (neither may ever be read)."""
+    rng = np.random.default_rng(seed)
+    B, d = len(lens), g.wl.d
+    tiles = [(n + 127) // 128 for n in lens]
+    max_pages = max(tiles) + 2
+    n_pages = sum(tiles) + spare
+    perm = rng.permutation(n_pages)
+    table = np.full((B, max_pages), 1 << 30, np.int32)
+    k = torch.full((n_pages, 128, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    v = torch.full((n_pages, 128, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kc, vc = to_torch_bf16(g.k), to_torch_bf16(g.v)
+    nxt = 0
+    for b, n in enumerate(lens):
+        for i in range(tiles[b]):
+            pg = int(perm[nxt]); nxt += 1
+            table[b, i] = pg
+            r = min(128, n - 128 * i)
+            k[pg, :r] = kc[b, 128 * i:128 * i + r]
+            v[pg, :r] = vc[b, 128 * i:128 * i + r]
+    return k, v, torch.from_numpy(table).cuda(), max_pages
+
+
+@pytest.mark.parametrize("lens", [[40000, 777, 129, 12345, 1, 128], [262144, 3000]])
+def test_decode_paged_equals_ragged_contiguous(hs2, lens):
+    """A paged cache gives bit-for-bit the ragged call's results on the same tokens laid out
+    contiguously (same tiles, same order, same arithmetic), and so does a sparse layer."""
+    B, Lk = len(lens), max(lens)
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=B, Lk=Lk))
+    q, k, v = to_torch_bf16(g.q), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    ref = [t.clone() for t in hs2.full_attn_select_ragged(q, k, v, lens, scale=g.wl.scale)]
+    kp, vp, table, max_pages = _paged_layout(g, lens)
+    out, lse, idx = hs2.full_attn_select_paged(q, kp, vp, table, lens, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    assert hs2.read_device_status(hs2.cached_workspace("full")) == 0
+    assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]) and torch.equal(idx, ref[2])
+    qs = to_torch_bf16(g.q_sparse(0))
+    o_c = hs2.sparse_attn(qs, k, v, idx, scale=g.wl.scale).clone()
+    o_p = hs2.sparse_attn_paged(qs, kp, vp, table, idx, scale=g.wl.scale)
+    torch.cuda.synchronize()
+    assert hs2.read_device_status(hs2.cached_workspace("sparse")) == 0
+    assert torch.equal(o_c, o_p)
+    if B <= 6:  # and against the oracle, per sequence
+        for b, n in enumerate(lens):
+            _check_seq(g, b, n, out, lse, idx)
+
+
+def test_decode_paged_bad_page_id_is_reported(hs2):
+    lens = [3000, 700]
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=2, Lk=3000))
+    q = to_torch_bf16(g.q)
+    kp, vp, table, _ = _paged_layout(g, lens)
+    table[1, 2] = kp.shape[0] + 5   # a used entry outside the pool
+    ws = torch.zeros(hs2.full_attn_select_paged_workspace_bytes(lens, table.shape[1], 64, 128), dtype=torch.uint8,
+                     device="cuda")
+    hs2.full_attn_select_paged(q, kp, vp, table, lens, scale=g.wl.scale, workspace=ws)
+    assert hs2.read_device_status(ws) == hs2.ERR_DEVICE_BOUNDS
+    hs2.clear_device_status(ws)
+    assert hs2.read_device_status(ws) == 0
