@@ -563,6 +563,51 @@ def bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks, steps=200, warmup=5):
     dec_ms, dec_n = hs2.profile_read("dec_fused")
     status = hs2.read_device_status(ws)
     del graph
+
+    # the same tokens in 128-token pages scattered over shared pools (a page table per sequence)
+    rng = np.random.default_rng(1)
+    tiles = [(n + 127) // 128 for n in lens]
+    n_pages, max_pages = sum(tiles), max(tiles)
+    perm = rng.permutation(n_pages)
+    kp = torch.empty((n_pages, 128, wl.d), dtype=torch.bfloat16, device=q.device)
+    vp = torch.empty_like(kp)
+    table = np.zeros((wl.B, max_pages), np.int32)
+    nxt = 0
+    for b, n in enumerate(lens):
+        for i in range(tiles[b]):
+            pg = int(perm[nxt]); nxt += 1
+            table[b, i] = pg
+            r = min(128, n - 128 * i)
+            kp[pg, :r] = k[b, 128 * i:128 * i + r]
+            vp[pg, :r] = v[b, 128 * i:128 * i + r]
+    table = torch.from_numpy(table).to(q.device)
+    ws_p = torch.zeros(hs2.full_attn_select_paged_workspace_bytes(lens, max_pages, wl.H, wl.d), dtype=torch.uint8,
+                       device=q.device)
+
+    def step_paged():
+        hs2.full_attn_select_paged(q, kp, vp, table, lens, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws_p)
+        for i in range(wl.n_sparse):
+            hs2.sparse_attn_paged(qs[i], kp, vp, table, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i])
+
+    for _ in range(warmup):
+        step_paged()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            step_paged()
+    graph.replay()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    _barrier(world)
+    ms_p = _max_over_ranks(e0.elapsed_time(e1), world)
+    status_p = hs2.read_device_status(ws_p)
+    del graph, kp, vp
+
     dec_bytes = sum(n * wl.d * 2 * 2 + max(n - wl.window, 0) * 4 for n in lens)
     dec_s = dec_ms / max(dec_n, 1) / 1e3
     return {"workload": f"decode_ragged: B={wl.B} sequences of {lens} tokens in the {wl.Lk}-row cache buffers, "
@@ -573,6 +618,9 @@ def bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks, steps=200, warmup=5):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_bytes / dec_s / 1e9 / peaks["hbm_gbs"],
                          "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": dec_s * 1e3,
                          "launches_timed": dec_n},
+            "paged": {"value": _throughput(world, steps, ms_p), "unit": "steps/s", "ms_per_step": ms_p / steps,
+                      "layout": f"the same tokens in {n_pages} pages of 128 tokens, randomly placed in shared pools, "
+                                f"one page-table row per sequence", "device_status": status_p},
             "device_status": status}
 
 
