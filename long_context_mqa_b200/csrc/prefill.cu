@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(NT, 1)
   __shared__ unsigned hist[2][256];
   __shared__ unsigned long long s_prefix[2];
   __shared__ int s_need[2], s_cnt[2];
+  __shared__ unsigned s_wsum[2][4];  // per-warp totals of the final ordered write
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const long long limit = p.wait_ns;
 
@@ -690,7 +691,50 @@ __global__ void __launch_bounds__(NT, 1)
         int* ib32 = reinterpret_cast<int*>(qb);
         const int wlo = pos - p.W + 1 > 0 ? pos - p.W + 1 : 0;
         const int wlen = pos - wlo + 1;
-        // the picks (<= topk <= 1024) are sorted; the window t-W+1..t follows them, all larger
+        int32_t* dst = p.idx + ((size_t)si.b * p.Lq + t) * p.S;
+        const int ncp = pos - p.W + 1;  // candidate positions 0 .. pos - W
+        const int nwords = ncp > 0 ? (ncp + 31) / 32 : 0;
+        if (nwords <= 2 * C::CAP) {
+          // the picks in ascending order through a bitmap of the candidate positions (in the
+          // query's buffer): set their bits, then one prefix count over the words writes them;
+          // the window t-W+1..t follows, all larger
+          unsigned* bm = reinterpret_cast<unsigned*>(qb);
+          for (int i = wt; i < nwords; i += 128) bm[i] = 0u;
+          wg_bar(wg);
+#pragma unroll
+          for (int m2 = 0; m2 < PER; ++m2)
+            if (mine[m2] != 0x7FFFFFFF) atomicOr(&bm[mine[m2] >> 5], 1u << (mine[m2] & 31));
+          wg_bar(wg);
+          const int per = (nwords + 127) / 128;
+          const int w0 = wt * per, w1 = w0 + per < nwords ? w0 + per : nwords;
+          unsigned cw = 0;
+          for (int i = w0; i < w1; ++i) cw += __popc(bm[i]);
+          unsigned incl = cw;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned nb = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nb;
+          }
+          const int wq = (warp - 2) & 3;
+          if (lane == 31) s_wsum[wg][wq] = incl;
+          wg_bar(wg);
+          unsigned o_pos = incl - cw;
+          for (int x = 0; x < wq; ++x) o_pos += s_wsum[wg][x];
+          for (int i = w0; i < w1; ++i) {
+            unsigned word = bm[i];
+            while (word) {
+              const int bit = __ffs(word) - 1;
+              word &= word - 1;
+              if (o_pos < (unsigned)keep) dst[o_pos] = i * 32 + bit;
+              ++o_pos;
+            }
+          }
+          for (int i = wt; i < p.S; i += 128)
+            if (i >= keep) dst[i] = i < keep + wlen ? wlo + (i - keep) : -1;
+          wg_bar(wg);
+          continue;
+        }
+        // (positions beyond the buffer's bitmap capacity) a bitonic sort of the picks
 #pragma unroll
         for (int m2 = 0; m2 < 1024 / 128; ++m2) {
           const int i = wt + 128 * m2;
@@ -710,7 +754,6 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
         const int total = keep + wlen;
-        int32_t* dst = p.idx + ((size_t)si.b * p.Lq + t) * p.S;
         for (int i = wt; i < p.S; i += 128) dst[i] = i < keep ? ib32[i] : (i < total ? wlo + (i - keep) : -1);
         wg_bar(wg);
       }
