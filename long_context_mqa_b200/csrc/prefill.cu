@@ -259,18 +259,24 @@ __global__ void __launch_bounds__(NT, 1)
         // causal masking only where the tile reaches past some row's query (warp-uniform)
         const bool masked = __any_sync(0xffffffffu, j * 128 + 127 > t);
         const int kvis = t - j * 128;  // keys 0..kvis of this tile are visible to this row
-        // pass over S: max of the raw logits (c > 0, so scaling commutes with the max)
+        // pass over S: max of the raw logits (c > 0, so scaling commutes with the max), 64 columns
+        // per TMEM wait
         float rmax = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          tmem_ld32(sS + cc * 32, v);
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[2][32];
+          tmem_ld32(sS + hh * 64, v[0]);
+          tmem_ld32(sS + hh * 64 + 32, v[1]);
           tmem_ld_wait();
-          if (masked) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = cc * 32 + x <= kvis ? v[x] : -INFINITY;
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int cc = 2 * hh + c2;
+            if (masked) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) v[c2][x] = cc * 32 + x <= kvis ? v[c2][x] : -INFINITY;
+            }
+            rmax = fmaxf(rmax, max32(v[c2]));
           }
-          rmax = fmaxf(rmax, max32(v));
         }
         const float mx = rmax * c;
         const bool raise = mx > -INFINITY && (m_used == -INFINITY || mx > m_used + 8.f);
@@ -300,10 +306,15 @@ __global__ void __launch_bounds__(NT, 1)
         // probabilities -> P (K-major: row = this thread's (query, head), K = the 128 keys)
         float la = 0.f, lb = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          tmem_ld32(sS + cc * 32, v);
+        for (int hh = 0; hh < 2; ++hh) {
+          float vv[2][32];
+          tmem_ld32(sS + hh * 64, vv[0]);
+          tmem_ld32(sS + hh * 64 + 32, vv[1]);
           tmem_ld_wait();
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+          const int cc = 2 * hh + c2;
+          const float* v = vv[c2];
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
@@ -321,6 +332,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             st_shared_v4(blk + sw128_off(row, (cc % 2) * 4 + q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
         }
         l += la + lb;
         tc_fence_before();
