@@ -420,6 +420,16 @@ def run_gpu(args):
     status_sp = max(hs2.read_device_status(w) for w in ws_sp)
     ms_per_step = ms_total / args.steps
     value = _throughput(world, args.steps, ms_total)
+    # the decode sparse layers' gathers: B rows x S selected K and V rows per layer
+    sparse_gather = None
+    if "sparse_attn" in breakdown:
+        per_layer_ms = breakdown["sparse_attn"] / wl.n_sparse
+        gb = wl.B * (wl.window + wl.topk) * wl.d * 2 * 2
+        sparse_gather = {"achieved": gb / (per_layer_ms / 1e3) / 1e9, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                         "frac": gb / (per_layer_ms / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_layer": gb,
+                         "ms_per_layer": per_layer_ms,
+                         "note": "4.7 MB per layer: latency-bound (a dependent chain of gather, S, softmax, PV "
+                                 "and cluster merge); at the HBM peak the bytes would take 0.7 us"}
 
     # ---------------- roofline of the dominant kernel (the fused decode kernel)
     ncand = wl.Lk - wl.window
@@ -515,6 +525,7 @@ def run_gpu(args):
                        "launch": (f"the {args.steps} timed steps replayed as one CUDA graph" if graph is not None
                                   else (graph_note or "eager launches"))},
             "roofline": roofline, "step_roofline": step_roof, "kernel_ms_per_step": breakdown,
+            "sparse_gather": sparse_gather,
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "note": "public Python API; per step one H2D copy of the five layers' queries from pinned memory, the new token's K/V rows, one D2H copy of the outputs and indices, a stream synchronize"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
@@ -698,6 +709,14 @@ def bench_prefill(args, world, dev, peaks, reps=5, warmup=2):
         sp_tf = sp_flops / (kern["sparse_attn_per_layer"] / 1e3) / 1e12
         res["sparse_roofline"] = {"bound": "tensor", "achieved": sp_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": sp_tf / peaks["bf16_tflops"], "flops": "4*H*d*S*L per layer"}
+        # the gather side of the same layer: every query row gathers its S selected K and V rows
+        # (2*d bf16 each) once for all heads; the cache is L2-resident, so this is the rate at which
+        # the kernel moves gathered rows, set against the HBM copy bandwidth
+        g_bytes = wl.Lq * (wl.window + wl.topk) * wl.d * 2 * 2
+        g_gbs = g_bytes / (kern["sparse_attn_per_layer"] / 1e3) / 1e9
+        res["sparse_gather"] = {"achieved": g_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                                "frac": g_gbs / peaks["hbm_gbs"], "bytes_per_layer": g_bytes,
+                                "note": "gathered K+V rows per layer (L2-resident cache) against the HBM copy peak"}
     if not args.prefill_len:
         # chunked prefill: the last CHUNK queries of the same prompt appended to the cache of the
         # first L - CHUNK tokens (query i at position L - CHUNK + i), same K/V buffers
