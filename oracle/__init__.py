@@ -9,6 +9,11 @@ compiled on first use with gcc into ``liboracle.so`` next to it. See that file's
 for what is computed and which passages of the pages each function follows.
 
 Arrays: bf16 tensors are passed as numpy ``uint16`` bit patterns.
+
+An FP8 (e4m3) K/V cache is read through ``e4m3_to_bf16``: the codes are decoded from the OCP
+8-bit floating-point definition (numpy, below) and multiplied by the tensor's power-of-two
+scale; every such value is exactly a bf16 value, so the functions above then run unchanged on
+the cache the kernels read.
 """
 from __future__ import annotations
 
@@ -79,6 +84,35 @@ def _rows(rows, total):
 def _check(rc, what):
     if rc != 0:
         raise RuntimeError(f"oracle {what}: {ERRORS.get(rc, rc)}")
+
+
+def e4m3_values() -> np.ndarray:
+    """The value of each of the 256 e4m3 codes (float64; NaN for 0x7F and 0xFF).
+
+    Code bits s eeee mmm: exponent field e with bias 7; e == 0 encodes the subnormals
+    m/8 * 2^-6, otherwise (1 + m/8) * 2^(e - 7); no infinities, and s 1111 111 is NaN.
+    """
+    c = np.arange(256)
+    s, e, m = c >> 7, (c >> 3) & 15, c & 7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.power(2.0, e - 7.0))
+    val = np.where(s == 1, -mag, mag)
+    val[(c & 0x7F) == 0x7F] = np.nan
+    return val
+
+
+def e4m3_to_bf16(codes, scale: float) -> np.ndarray:
+    """bf16 bit patterns of code value * scale (scale a power of two; exact, else ValueError)."""
+    m, _ = np.frexp(scale)
+    if not (scale > 0 and m == 0.5):
+        raise ValueError("the e4m3 scale must be a positive power of two")
+    x = e4m3_values()[np.asarray(codes, dtype=np.uint8)] * scale
+    if np.isnan(x).any():
+        raise ValueError("NaN code in the e4m3 cache")
+    f = x.astype(np.float32)
+    u = f.view(np.uint32)
+    if np.any(f.astype(np.float64) != x) or np.any(u & np.uint32(0xFFFF)):
+        raise ValueError("dequantised value is not a bf16 value")
+    return (u >> np.uint32(16)).astype(np.uint16)
 
 
 def full_attn_select(q, k, v, scale, window, topk, rows=None, want_score=False, threads=0):

@@ -20,6 +20,11 @@ u (a normalised N(0, I_d) draw) is added with gain 3 to exactly floor(0.02 * Lk)
 positions per sequence (drawn without replacement) and to every query vector (all heads,
 all layers), so that the top-k selection is not trivial. V is not planted. The bridge
 hidden state is N(0, 1) and the projection weights are N(0, 0.02^2).
+
+FP8 cache: the same float32 K and V samples stored as OCP e4m3 codes (1 sign, 4 exponent bits
+with bias 7, 3 mantissa bits, subnormals, no infinities) times one power-of-two scale per
+tensor, the smallest for which the largest magnitude fits under 448; each value rounds to the
+nearest code, ties to the even code.
 """
 from __future__ import annotations
 
@@ -85,6 +90,42 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+E4M3_MAX = 448.0
+
+
+def e4m3_scale(x: np.ndarray) -> float:
+    """The power-of-two scale 2^e with max|x| / 2^e <= 448 for the smallest such e."""
+    amax = float(np.max(np.abs(x))) if x.size else 0.0
+    if amax == 0.0:
+        return 1.0
+    e = math.ceil(math.log2(amax / E4M3_MAX))
+    if amax / 2.0 ** e > E4M3_MAX:  # log2 rounding at an exact power of two
+        e += 1
+    return float(2.0 ** e)
+
+
+def f32_to_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
+    """Codes of x / scale rounded to e4m3 (nearest, ties to even); |x / scale| must be <= 448."""
+    a = np.asarray(x, dtype=np.float64).reshape(-1) / scale
+    if not np.all(np.isfinite(a)) or np.max(np.abs(a), initial=0.0) > E4M3_MAX:
+        raise ValueError("value outside the e4m3 range")
+    sign = np.signbit(a).astype(np.int64)
+    m = np.abs(a)
+    code = np.empty(m.shape, np.int64)
+    sub = m < 2.0 ** -6
+    # subnormal range: steps of 2^-9 (code = steps; 8 steps is the smallest normal, code 8)
+    code[sub] = np.rint(m[sub] * 2.0 ** 9).astype(np.int64)
+    nrm = ~sub
+    if np.any(nrm):
+        _, ex = np.frexp(m[nrm])           # m = f * 2^ex, f in [0.5, 1)
+        e = ex.astype(np.int64) - 1        # m in [2^e, 2^(e+1))
+        steps = np.rint(np.ldexp(m[nrm], (3 - e).astype(np.int32))).astype(np.int64)  # 8..16
+        code[nrm] = (e + 6) * 8 + steps    # (e + 7) * 8 + (steps - 8); 16 steps carries into e + 1
+    if np.any(code > 0x7E):
+        raise ValueError("value rounds above 448")
+    return (code | (sign << 7)).astype(np.uint8).reshape(np.shape(x))
+
+
 _CHUNK = 1 << 24  # elements per independent sub-stream for large tensors
 
 
@@ -139,17 +180,35 @@ class SyntheticInputs:
     @cached_property
     def k(self) -> np.ndarray:
         """[B, Lk, d] keys (one KV head)."""
-        wl = self.wl
-        k = _normal_f32(self._s[3], (wl.B, wl.Lk, wl.d))
-        for b in range(wl.B):
-            k[b, self.planted[b]] += PLANT_GAIN * self.u
-        return f32_to_bf16_bits(k)
+        return f32_to_bf16_bits(self._k_f32)
 
     @cached_property
     def v(self) -> np.ndarray:
         """[B, Lk, d] values (one KV head)."""
         wl = self.wl
         return f32_to_bf16_bits(_normal_f32(self._s[4], (wl.B, wl.Lk, wl.d)))
+
+    @cached_property
+    def _k_f32(self) -> np.ndarray:
+        wl = self.wl
+        k = _normal_f32(self._s[3], (wl.B, wl.Lk, wl.d))
+        for b in range(wl.B):
+            k[b, self.planted[b]] += PLANT_GAIN * self.u
+        return k
+
+    @cached_property
+    def k8(self) -> tuple[np.ndarray, float]:
+        """([B, Lk, d] e4m3 codes, power-of-two scale) of the same key samples as ``k``."""
+        k = self._k_f32
+        sc = e4m3_scale(k)
+        return f32_to_e4m3(k, sc), sc
+
+    @cached_property
+    def v8(self) -> tuple[np.ndarray, float]:
+        """([B, Lk, d] e4m3 codes, power-of-two scale) of the same value samples as ``v``."""
+        v = _normal_f32(self._s[4], (self.wl.B, self.wl.Lk, self.wl.d))
+        sc = e4m3_scale(v)
+        return f32_to_e4m3(v, sc), sc
 
     def q_sparse(self, layer: int) -> np.ndarray:
         """[B, Lq, H, d] query of sparse layer `layer` (same distribution as q)."""

@@ -272,3 +272,76 @@ def test_row_sampling_matches_full_run():
     part = oracle.full_attn_select(g.q, g.k, g.v, wl.scale, 16, 32, rows=[2, 0], want_score=True)
     for key in ("out", "lse", "idx", "score"):
         np.testing.assert_array_equal(part[key], full[key][[2, 0]])
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (e4m3) cache: the oracle's decoder and the input generator's encoder
+# ---------------------------------------------------------------------------------------------
+def test_e4m3_decoder_matches_torch_for_every_code():
+    """The oracle's decoder of the 8-bit format against torch's float8_e4m3fn conversion."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    val = oracle.e4m3_values()
+    assert np.array_equal(np.isnan(val), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(val[ok], ref[ok])
+
+
+def test_e4m3_closed_forms():
+    val = oracle.e4m3_values()
+    assert val[0x38] == 1.0 and val[0xB8] == -1.0          # 0 0111 000: 2^(7-7)
+    assert val[0x7E] == 448.0                              # largest finite: 2^8 * 1.75
+    assert val[0x01] == 2.0 ** -9 and val[0x07] == 7 * 2.0 ** -9   # subnormals m/8 * 2^-6
+    assert val[0x08] == 2.0 ** -6                          # smallest normal
+    assert val[0x00] == 0.0 and val[0x80] == 0.0 and np.signbit(val[0x80])
+    assert np.isnan(val[0x7F]) and np.isnan(val[0xFF])
+    assert np.all(np.diff(val[:0x7F]) > 0)                 # codes 0..126 increase strictly
+
+
+def test_e4m3_encoder_matches_torch():
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(100000) * 40.0, rng.standard_normal(1000) * 0.01,
+                        # ties between neighbouring codes go to the even code
+                        [2.0 ** -10, 3 * 2.0 ** -10, 1.0625, 1.1875, 448.0, -448.0, 0.0, 2.0 ** -6 * (1 - 1 / 16)]])
+    x = x.astype(np.float32)
+    for sc in (1.0, 2.0 ** -6):
+        got = synth.f32_to_e4m3(x * np.float32(sc), sc)
+        ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(got, ref)
+    with pytest.raises(ValueError):
+        synth.f32_to_e4m3(np.array([449.0], np.float32), 1.0)
+
+
+def test_e4m3_scale_and_dequantisation():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((3, 50, 8)) * 3).astype(np.float32)
+    sc = synth.e4m3_scale(x)
+    assert np.max(np.abs(x)) / sc <= 448.0 < 2 * np.max(np.abs(x)) / sc
+    codes = synth.f32_to_e4m3(x, sc)
+    deq = bf16_bits_to_f32(oracle.e4m3_to_bf16(codes, sc)).astype(np.float64)
+    ref = torch.from_numpy(codes.reshape(-1)).view(torch.float8_e4m3fn).double().numpy().reshape(x.shape) * sc
+    assert np.array_equal(deq, ref)
+    # nearest code: the error is at most half a step (relative 2^-4 for normals, 2^-10 * sc below)
+    err = np.abs(deq - x)
+    assert np.all(err <= np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * sc) + 1e-12)
+    with pytest.raises(ValueError):
+        oracle.e4m3_to_bf16(codes, 0.3)
+
+
+def test_attention_on_e4m3_cache_matches_torch_sdpa():
+    """Attention over a dequantised e4m3 cache (through the bf16 view) against torch SDPA on
+    torch's own decoding of the same codes."""
+    rng = np.random.default_rng(13)
+    B, Lq, Lk, H, d = 2, 1, 45, 4, 16
+    q = _rand_bf16(rng, (B, Lq, H, d))
+    kf = (rng.standard_normal((B, Lk, d)) * 2).astype(np.float32)
+    vf = rng.standard_normal((B, Lk, d)).astype(np.float32)
+    ks, vs = synth.e4m3_scale(kf), synth.e4m3_scale(vf)
+    k8, v8 = synth.f32_to_e4m3(kf, ks), synth.f32_to_e4m3(vf, vs)
+    kb, vb = oracle.e4m3_to_bf16(k8, ks), oracle.e4m3_to_bf16(v8, vs)
+    r = oracle.full_attn_select(q, kb, vb, 0.25, 4, 8)
+    dec = lambda c, s: torch.from_numpy(c.reshape(-1)).view(torch.float8_e4m3fn).double().reshape(c.shape) * s
+    Q = _t64(q).permute(0, 2, 1, 3)
+    K = dec(k8, ks)[:, None].expand(-1, H, -1, -1)
+    V = dec(v8, vs)[:, None].expand(-1, H, -1, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=0.25).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(r["out"], o.reshape(B * Lq, H, d), rtol=0, atol=1e-12)
