@@ -289,6 +289,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-ragged", action="store_true", help="skip the ragged-batch decode clause")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 (e4m3) K/V cache decode clause")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph of the steps")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (small profiling cases)")
@@ -503,6 +504,11 @@ def run_gpu(args):
     if not args.no_ragged:
         ragged = bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks)
 
+    # ---------------- the same decode step over an FP8 (e4m3) K/V cache
+    fp8 = None
+    if not args.no_fp8:
+        fp8 = bench_fp8(args, world, wl, hs2, q, k, v, qs, peaks)
+
     # ---------------- prefill (secondary clause of the metric)
     prefill = None
     if not args.no_prefill:
@@ -529,7 +535,7 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "note": "public Python API; per step one H2D copy of the five layers' queries from pinned memory, the new token's K/V rows, one D2H copy of the outputs and indices, a stream synchronize"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
-            "device_status": [status, status_sp], "cpu_baseline": cpu, "ragged": ragged, "prefill": prefill,
+            "device_status": [status, status_sp], "cpu_baseline": cpu, "ragged": ragged, "fp8_kv": fp8, "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -643,6 +649,71 @@ def bench_ragged(args, world, wl, hs2, q, k, v, qs, peaks, steps=200, warmup=5):
             "paged": {"value": _throughput(world, steps, ms_p), "unit": "steps/s", "ms_per_step": ms_p / steps,
                       "layout": f"the same tokens in {n_pages} pages of 128 tokens, randomly placed in shared pools, "
                                 f"one page-table row per sequence", "device_status": status_p},
+            "device_status": status}
+
+
+def bench_fp8(args, world, wl, hs2, q, k, v, qs, peaks, steps=200, warmup=5):
+    """The decode step over the bench's cache stored as e4m3 codes (one power-of-two scale per
+    tensor: the bf16 cache divided by 2^ceil(log2(max|x| / 448)) and rounded by torch's float8
+    conversion on the device), one hs2_full_attn_select_fp8kv plus the sparse layers over the same
+    codes per step, as one CUDA graph; device-timed like the main line."""
+    import torch
+
+    def quant(x):
+        amax = float(x.abs().max())
+        sc = 2.0 ** math.ceil(math.log2(amax / 448.0)) if amax > 0 else 1.0
+        return (x.float() / sc).to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), sc
+
+    k8, ks = quant(k)
+    v8, vs = quant(v)
+    S = wl.window + wl.topk
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, 1, wl.H), dtype=torch.float32, device=q.device)
+    idx = torch.empty((wl.B, 1, S), dtype=torch.int32, device=q.device)
+    outs = [torch.empty_like(q) for _ in range(wl.n_sparse)]
+    ws = torch.zeros(hs2.full_attn_select_fp8kv_workspace_bytes(wl.B, None, wl.Lk, wl.H, wl.d), dtype=torch.uint8,
+                     device=q.device)
+    ws_sp = [torch.zeros(hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S), dtype=torch.uint8,
+                         device=q.device) for _ in range(wl.n_sparse)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hs2.full_attn_select_fp8kv(q, k8, v8, ks, vs, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws)
+        for i in range(wl.n_sparse):
+            hs2.sparse_attn_fp8kv(qs[i], k8, v8, ks, vs, idx, scale=wl.scale, out=outs[i], workspace=ws_sp[i])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(steps):
+            hs2.profile_enable("dec_fused" if i % 8 == 0 else None)
+            step()
+        hs2.profile_enable(None)
+    graph.replay()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    _barrier(world)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    dec_ms, dec_n = hs2.profile_read("dec_fused")
+    status = hs2.read_device_status(ws)
+    del graph, k8, v8
+    # one byte per cached K and V element, plus the 4-byte score of each older token
+    dec_bytes = wl.B * (wl.Lk * wl.d * 2 + max(wl.Lk - wl.window, 0) * 4)
+    dec_s = dec_ms / max(dec_n, 1) / 1e3
+    return {"workload": f"{wl.name} with the K/V cache as e4m3 codes ({wl.B * wl.Lk * wl.d * 2 / 1e6:.0f} MB, half "
+                        f"the bf16 bytes), per-tensor power-of-two scales",
+            "value": _throughput(world, steps, ms), "unit": "steps/s", "ms_per_step": ms / steps,
+            "roofline": {"kernel": "dec_fused (e4m3)", "bound": "hbm", "achieved": dec_bytes / dec_s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_bytes / dec_s / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": dec_s * 1e3,
+                         "launches_timed": dec_n, "traffic": _traffic("dec_fused_e4m3")},
             "device_status": status}
 
 

@@ -142,6 +142,30 @@ HS2_API hs2_status hs2_full_attn_select_paged(const hs2_bf16* Q, const hs2_bf16*
                                               hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
                                               size_t workspace_bytes, hs2_stream stream);
 
+/* FP8 cache: the decode step over a K/V cache stored as 8-bit floats (the pages' KV-cache cost
+ * figures at 1M tokens are quoted for FP8 storage: arex-research.com, section "三套 80B-A3B
+ * 对照模型里算出的数字", the cost paragraph).
+ * K8, V8     e4m3 codes (OCP FP8: sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ *            subnormals; 0x7F / 0xFF are NaN), [B, Lk, d] rows, or with a page table the pools
+ *            [n_pages, 128, d] as for hs2_full_attn_select_paged (then Lk == 128 * max_pages)
+ * k_scale, v_scale  per-tensor factors, positive and finite: the cache holds K = k_scale * K8,
+ *            V = v_scale * V8 (a power of two keeps every value exact in bf16)
+ * lens       HOST array of B lengths (1 <= lens[b] <= Lk), or NULL: every sequence Lk tokens
+ * Q, out, lse, idx as for the ragged call; results equal that call on the dequantised bf16 cache
+ * (every e4m3 value times a power of two is a bf16 value). The kernels read the codes (half the
+ * bytes of bf16) and widen them exactly on chip. Supported: (H, d) = (64, 128), one query per
+ * sequence, 1 <= B <= 256. Workspace: hs2_full_attn_select_fp8kv_workspace_bytes with the same
+ * B, lens (or NULL) and Lk.
+ */
+HS2_API size_t hs2_full_attn_select_fp8kv_workspace_bytes(int B, const int32_t* lens, int Lk, int H, int d,
+                                                          int window, int topk);
+HS2_API hs2_status hs2_full_attn_select_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8, float k_scale,
+                                              float v_scale, int B, const int32_t* lens, int Lk,
+                                              const int32_t* page_table, int max_pages, int n_pages, int H, int d,
+                                              float scale, int window, int topk, hs2_bf16* out, float* lse,
+                                              int32_t* idx, void* workspace, size_t workspace_bytes,
+                                              hs2_stream stream);
+
 /* ---------------------------------------------------------------------------------
  * Sparse attention over selected tokens (one sparse layer)
  * ---------------------------------------------------------------------------------
@@ -169,6 +193,17 @@ HS2_API hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pa
                                          int n_pages, const int32_t* page_table, int max_pages, const int32_t* idx,
                                          int B, int Lq, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
                                          void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* Sparse attention over an FP8 cache: K8, V8, k_scale, v_scale (and the optional page table,
+ * with Lk == 128 * max_pages) as for hs2_full_attn_select_fp8kv; every other argument as for
+ * hs2_sparse_attn, whose workspace size applies. Results equal hs2_sparse_attn on the
+ * dequantised bf16 cache. Supported: (H, d) in {(64, 128), (16, 64)}, 1 <= S <= 4096.
+ */
+HS2_API hs2_status hs2_sparse_attn_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8, float k_scale,
+                                         float v_scale, const int32_t* idx, int B, int Lq, int Lk,
+                                         const int32_t* page_table, int max_pages, int n_pages, int H, int d, int S,
+                                         float scale, hs2_bf16* out, float* lse, void* workspace,
+                                         size_t workspace_bytes, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * Sparse attention without a caller workspace
@@ -225,6 +260,10 @@ HS2_API hs2_status hs2_selftest_wait_timeout(void* workspace, size_t workspace_b
  * flushing subnormals) it is mixed with (into y_mufu), so a test can bound their error. No
  * counterpart in the paper: a check of an arithmetic building block. */
 HS2_API hs2_status hs2_selftest_exp2(const float* x, float* y_soft, float* y_mufu, int n, hs2_stream stream);
+/* hs2_selftest_e4m3: widens the n device e4m3 codes x (n even) with the conversions the FP8-cache
+ * kernels use, to f16 bit patterns (y_f16) and bf16 bit patterns (y_bf16), so a test can check
+ * them against the format's definition. */
+HS2_API hs2_status hs2_selftest_e4m3(const uint8_t* x, uint16_t* y_f16, uint16_t* y_bf16, int n, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * Diagnostics (never needed on the compute path)

@@ -67,6 +67,16 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_sparse_attn_workspace_bytes.restype = sz
     lib.hs2_sparse_attn.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, sz, P]
     lib.hs2_sparse_attn.restype = i32
+    lib.hs2_full_attn_select_fp8kv_workspace_bytes.argtypes = [i32, P, i32, i32, i32, i32, i32]
+    lib.hs2_full_attn_select_fp8kv_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select_fp8kv.argtypes = [P, P, P, f32, f32, i32, P, i32, P, i32, i32, i32, i32, f32, i32, i32,
+                                               P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_fp8kv.restype = i32
+    lib.hs2_sparse_attn_fp8kv.argtypes = [P, P, P, f32, f32, P, i32, i32, i32, P, i32, i32, i32, i32, i32, f32, P, P,
+                                          P, sz, P]
+    lib.hs2_sparse_attn_fp8kv.restype = i32
+    lib.hs2_selftest_e4m3.argtypes = [P, P, P, i32, P]
+    lib.hs2_selftest_e4m3.restype = i32
     lib.hs2_bridge_kv_proj_workspace_bytes.argtypes = [i32] * 4
     lib.hs2_bridge_kv_proj_workspace_bytes.restype = sz
     lib.hs2_bridge_kv_proj.argtypes = [P, i32, i32, P, i32, i32, P, P, sz, P]
@@ -275,6 +285,90 @@ def sparse_attn_paged(q, k_pages, v_pages, page_table, idx, *, scale=None, out=N
     return out
 
 
+def _fp8_cache(k8, v8, page_table, B, d):
+    """(Lk, max_pages, n_pages) of an e4m3 cache: [B,Lk,d] rows, or pools [n_pages,128,d] + table."""
+    _need(k8, "k8", torch.uint8, 3)
+    _need(v8, "v8", torch.uint8, 3)
+    if v8.shape != k8.shape or k8.shape[2] != d:
+        raise ValueError("k8 and v8 must have the same shape [.., .., d]")
+    if page_table is None:
+        if k8.shape[0] != B:
+            raise ValueError("k8, v8 must be [B, Lk, d]")
+        return k8.shape[1], 0, 0
+    _need(page_table, "page_table", torch.int32, 2)
+    if k8.shape[1] != 128 or page_table.shape[0] != B:
+        raise ValueError("paged: k8, v8 [n_pages, 128, d], page_table [B, max_pages]")
+    return page_table.shape[1] * 128, page_table.shape[1], k8.shape[0]
+
+
+def full_attn_select_fp8kv_workspace_bytes(B, lens, Lk, H, d, window=WINDOW, topk=TOPK) -> int:
+    lens_c = _lens_array(list(lens), B, Lk) if lens is not None else None
+    return int(lib.hs2_full_attn_select_fp8kv_workspace_bytes(B, lens_c, Lk, H, d, window, topk))
+
+
+def full_attn_select_fp8kv(q, k8, v8, k_scale, v_scale, *, lens=None, page_table=None, scale=None, window=WINDOW,
+                           topk=TOPK, out=None, lse=None, idx=None, workspace=None, stream=None):
+    """Decode step over an e4m3 K/V cache (hs2_full_attn_select_fp8kv).
+
+    q [B,1,H,d] bf16; k8, v8 uint8 e4m3 codes [B,Lk,d] (or page pools [n_pages,128,d] with
+    page_table [B,max_pages] int32 on the device); the cache is k_scale * k8, v_scale * v8;
+    lens: B host integers or None (every sequence full). Returns (out, lse, idx) as
+    full_attn_select_ragged.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    B, Lq, H, d = q.shape
+    if Lq != 1:
+        raise ValueError("q must be [B, 1, H, d]")
+    Lk, max_pages, n_pages = _fp8_cache(k8, v8, page_table, B, d)
+    lens_c = _lens_array(list(lens), B, Lk) if lens is not None else None
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = window + topk
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, 1, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, 1, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    nbytes = int(lib.hs2_full_attn_select_fp8kv_workspace_bytes(B, lens_c, Lk, H, d, window, topk))
+    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    code = lib.hs2_full_attn_select_fp8kv(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(k_scale), float(v_scale), B,
+                                          lens_c, Lk, page_table.data_ptr() if page_table is not None else None,
+                                          max_pages, n_pages, H, d, scale, window, topk, out.data_ptr(),
+                                          lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                          ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select_fp8kv")
+    return out, lse, idx
+
+
+def sparse_attn_fp8kv(q, k8, v8, k_scale, v_scale, idx, *, page_table=None, scale=None, out=None, lse=None,
+                      want_lse=False, workspace=None, stream=None):
+    """Sparse attention over an e4m3 K/V cache (hs2_sparse_attn_fp8kv); arguments as
+    full_attn_select_fp8kv and sparse_attn. Returns out, or (out, lse) when want_lse or lse is given."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(idx, "idx", torch.int32, 3)
+    B, Lq, H, d = q.shape
+    Lk, max_pages, n_pages = _fp8_cache(k8, v8, page_table, B, d)
+    S = idx.shape[2]
+    if tuple(idx.shape[:2]) != (B, Lq):
+        raise ValueError("idx must be [B, Lq, S]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", torch.bfloat16, 4)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    nbytes = sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S)
+    ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
+    code = lib.hs2_sparse_attn_fp8kv(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(k_scale), float(v_scale),
+                                     idx.data_ptr(), B, Lq, Lk, page_table.data_ptr() if page_table is not None else None,
+                                     max_pages, n_pages, H, d, S, scale, out.data_ptr(),
+                                     lse.data_ptr() if lse is not None else None, ws.data_ptr(),
+                                     ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_sparse_attn_fp8kv")
+    return (out, lse) if lse is not None else out
+
+
 def sparse_attn(q, k, v, idx, *, scale=None, out=None, lse=None, want_lse=False, workspace=None, stream=None):
     """Sparse attention of one sparse layer over the reused K/V and indices (hs2_sparse_attn).
 
@@ -356,6 +450,17 @@ def selftest_exp2(x: torch.Tensor, stream=None):
     _check(lib.hs2_selftest_exp2(x.data_ptr(), ys.data_ptr(), ym.data_ptr(), x.numel(), _stream_ptr(stream)),
            "hs2_selftest_exp2")
     return ys, ym
+
+
+def selftest_e4m3(x: torch.Tensor, stream=None):
+    """(f16 bits, bf16 bits) as int16 tensors: the device widening of the e4m3 codes x (uint8,
+    even length) that the FP8-cache kernels use, see hs2.h."""
+    _need(x, "x", torch.uint8, 1)
+    yh = torch.empty(x.numel(), dtype=torch.int16, device=x.device)
+    yb = torch.empty_like(yh)
+    _check(lib.hs2_selftest_e4m3(x.data_ptr(), yh.data_ptr(), yb.data_ptr(), x.numel(), _stream_ptr(stream)),
+           "hs2_selftest_e4m3")
+    return yh, yb
 
 
 def kernel_launches() -> int:

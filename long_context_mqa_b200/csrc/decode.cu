@@ -36,6 +36,15 @@
 // warps 2..5 and 6..9 = softmax warpgroups 0 and 1 (warp w reads TMEM lanes 32*(w%4)..+31).
 // Every wait is bounded; on timeout the kernel records it in the status word and unwinds with
 // its barrier sequence intact.
+//
+// FP8 cache (F8): K and V arrive as e4m3 tiles (16 KB, half the bytes) through a 6-slot ring and
+// the softmax warps widen them exactly to f16: a K row into TMEM, where the S MMA reads its A
+// operand (each thread writes its own key's row: lane = key), a V row into an f16 tile in shared
+// memory for the PV MMA; the query is rewritten in place as f16 when it lands and P is packed
+// as f16, so every MMA is f16 x f16 with fp32 accumulation. The cache's scales are folded into
+// the logit factor c and the output combine. f16 P holds values below 65504: the references are
+// offset (p' = 4 p'' in the sampled pass, 2^12 p in the exact redo, both cancelling in O / L')
+// and a key whose head sum passes 65504 is flagged for the redo.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -44,9 +53,15 @@ namespace hs2 {
 namespace dec {
 
 constexpr int TILE = 128;
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 320;     // bf16 cache
+constexpr int NTHREADS_F8 = 448;  // FP8 cache: + a warpgroup that widens the e4m3 tiles
+constexpr int CONV_WARP0 = 10;    // its first warp
 constexpr int SM_WG0 = 2;  // first warp of softmax warpgroup 0
 constexpr int RING = 5;    // K/V tile slots
+constexpr int RING8 = 8;   // e4m3 K/V tile slots (FP8 cache)
+constexpr float F8_MAX_SCORE = 65504.f;  // largest f16: a bound on each p' of a key
+constexpr float F8_OFF_SAMPLED = 2.f;    // log2 offsets of the p' reference (FP8 cache)
+constexpr float F8_OFF_EXACT = 12.f;
 constexpr int NBINS = 2048;
 constexpr float REF_SLACK = 64.f;
 
@@ -118,8 +133,8 @@ __device__ __forceinline__ int sample_stride(const Sched& S, int b, int target) 
   return target > 0 && tiles / target > 1 ? tiles / target : 1;
 }
 
-template <int H, int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
+template <int H, int D, bool F8>
+__global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
     dec_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, DecParams p) {
   static_assert(H == 64 && D == 128, "the decode kernel is instantiated for 64 heads x 128");
@@ -128,14 +143,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int P_BYTES = TILE * H * 2;
   constexpr int NKB = D / 64;
   constexpr int HW = H / 2;  // heads per warpgroup in phase 1
+  constexpr int NR = F8 ? RING8 : RING;                // ring slots
+  constexpr int SLOT_BYTES = F8 ? TILE * D : KT_BYTES;  // one K or V tile as it arrives
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                  // Q of the current segment
-  uint8_t* sR = sQ + Q_BYTES;          // RING tiles (K or V)
-  uint8_t* sP = sR + RING * KT_BYTES;  // P^T of warpgroup 0 / 1
+  uint8_t* sQ = smem;                     // Q of the current segment
+  uint8_t* sR = sQ + Q_BYTES;             // NR tiles (K or V)
+  uint8_t* sV = sR + NR * SLOT_BYTES;     // FP8 cache: the f16 V tile of the next PV
+  uint8_t* sP = sV + (F8 ? KT_BYTES : 0);  // P^T of warpgroup 0 / 1
   uint32_t* shist = (uint32_t*)(sP + 2 * P_BYTES);
-  __shared__ __align__(8) uint64_t r_full[RING], r_empty[RING], s_full[2], s_empty[2], p_full[2], p_empty[2], q_full,
+  __shared__ __align__(8) uint64_t r_full[NR], r_empty[NR], s_full[2], s_empty[2], p_full[2], p_empty[2], q_full,
       q_empty, o_full, o_empty;
+  // FP8 cache: the f16 K rows in TMEM and the f16 V tiles (filled by the widening warps,
+  // emptied by the S and PV MMAs) and the query rewritten as f16
+  __shared__ __align__(8) uint64_t ka_full[2], ka_empty[2], v16_full, v16_empty, q16_full;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ __align__(16) float slse[H];
@@ -151,6 +172,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const Sched& S = p.sch;  // in parameter space (its start table is indexed at run time)
   const long long limit = p.wait_ns;
   const uint32_t tS = 0, tO = 2 * H;  // TMEM columns: S buffers 0..2H-1, O^T 2H..3H-1
+  constexpr uint32_t tKA = 256;       // FP8 cache: f16 K tiles 256..319, 320..383 (D / 2 columns each)
+  constexpr uint32_t tLA = 384;       // FP8 cache: per-row sums of p' of warpgroup 0 / 1 (H columns each)
+  constexpr uint32_t TMEM_COLS = F8 ? 512 : 256;
   // launched as a programmatic dependent: nothing before this point touches global memory
   griddep_wait();
   // the exact redo runs only if the sampled launch before it flagged a sequence (every CTA reads
@@ -159,9 +183,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // in the redo, only flagged sequences are processed (every role skips the same segments)
   auto skip_seq = [&](int b) -> bool { return p.fallback && *(volatile const int*)&p.ovf[b] == 0; };
 
-  for (int i = threadIdx.x; i < NBINS; i += NTHREADS) shist[i] = 0;
+  for (int i = threadIdx.x; i < NBINS; i += (F8 ? NTHREADS_F8 : NTHREADS)) shist[i] = 0;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < RING; ++i) { mbar_init(&r_full[i], 1); mbar_init(&r_empty[i], 1); }
+    // FP8 cache: a slot is released by the 4 widening warps; bf16: by the MMA that read it
+    for (int i = 0; i < NR; ++i) { mbar_init(&r_full[i], 1); mbar_init(&r_empty[i], F8 ? 4 : 1); }
+    if (F8) {
+      for (int i = 0; i < 2; ++i) { mbar_init(&ka_full[i], 4); mbar_init(&ka_empty[i], 1); }
+      mbar_init(&v16_full, 4); mbar_init(&v16_empty, 1);
+      mbar_init(&q16_full, 4);
+    }
     for (int i = 0; i < 2; ++i) {
       // phase 1: all 8 softmax warps release an S buffer; phase 2: the 4 warps of its owner, x2
       mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8);
@@ -172,7 +202,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(&tmem_base, TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -195,13 +225,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // tile lt of sequence b: rows lt*128.. of its cache, or (paged cache) page `pg`, whose 128
       // rows are the third tensor-map coordinate's slice (an id outside the pool reads zeros)
       auto load_tile = [&](const CUtensorMap* m, int lt, int b, uint64_t pol, int pg) -> bool {
-        const int s = ri % RING;
-        if (!wait_bar(&r_empty[s], ((ri / RING) & 1) ^ 1, limit, &abort_flag, p.st, 202)) return false;
-        mbar_expect_tx(&r_full[s], KT_BYTES);
+        const int s = ri % NR;
+        if (!wait_bar(&r_empty[s], ((ri / NR) & 1) ^ 1, limit, &abort_flag, p.st, 202)) return false;
+        mbar_expect_tx(&r_full[s], SLOT_BYTES);
         if (p.ptab && (pg < 0 || pg >= p.n_pages)) report_status(p.st, kStatusBounds, 203);  // reads zeros
         const int c1 = p.ptab ? 0 : lt * TILE, c2 = p.ptab ? pg : b;
-        for (int kb = 0; kb < NKB; ++kb)
-          tma_load_3d_hint(sR + s * KT_BYTES + kb * (TILE * 128), m, &r_full[s], kb * 64, c1, c2, pol);
+        if constexpr (F8) {  // one 128-byte row per key: a single swizzled box
+          tma_load_3d_hint(sR + s * SLOT_BYTES, m, &r_full[s], 0, c1, c2, pol);
+        } else {
+          for (int kb = 0; kb < NKB; ++kb)
+            tma_load_3d_hint(sR + s * KT_BYTES + kb * (TILE * 128), m, &r_full[s], kb * 64, c1, c2, pol);
+        }
         ++ri;
         return true;
       };
@@ -243,43 +277,64 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
-        for (uint32_t x = (ri > RING ? ri - RING : 0); x < ri; ++x) mbar_wait(&r_full[x % RING], (x / RING) & 1, limit);
+        for (uint32_t x = (ri > NR ? ri - NR : 0); x < ri; ++x) mbar_wait(&r_full[x % NR], (x / NR) & 1, limit);
         if (nq > 0) mbar_wait(&q_full, (nq - 1) & 1, limit);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16(128, H, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16(D, H, 1, 1);
+      constexpr uint32_t IDESC_S = F8 ? idesc_f16(128, H, 0, 0) : idesc_bf16(128, H, 0, 0);
+      constexpr uint32_t IDESC_O = F8 ? idesc_f16(D, H, 1, 1) : idesc_bf16(D, H, 1, 1);
+      uint64_t* const qready = F8 ? &q16_full : &q_full;  // the query as the MMAs read it
       // js counts S tiles (the TMEM S buffer is js & 1), jp phase-2 tiles (their P buffer / owner)
       uint32_t ri = 0, js = 0, jp = 0, nq = 0, seg2 = 0;
       uint32_t npu[2] = {0, 0};  // PV uses of each P buffer
+      uint32_t npv = 0;          // PVs issued (FP8 cache: uses of the f16 V buffer)
       bool ok = true;
       auto issue_s = [&](uint32_t kidx) -> bool {
-        const int s = kidx % RING, buf = js & 1;
-        if (!wait_bar(&r_full[s], (kidx / RING) & 1, limit, &abort_flag, p.st, 211)) return false;
+        const int s = kidx % NR, buf = js & 1;
+        if constexpr (F8) {  // the tile's f16 K rows, written to TMEM by the softmax warps
+          if (!wait_bar(&ka_full[buf], (js >> 1) & 1, limit, &abort_flag, p.st, 217)) return false;
+        } else {
+          if (!wait_bar(&r_full[s], (kidx / NR) & 1, limit, &abort_flag, p.st, 211)) return false;
+        }
         if (!wait_bar(&s_empty[buf], ((js >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 212)) return false;
         tc_fence_after();
-        const uint64_t ka = sdesc(smem_u32(sR + s * KT_BYTES), 16, 1024), qa = sdesc(smem_u32(sQ), 16, 1024);
+        const uint64_t qa = sdesc(smem_u32(sQ), 16, 1024);
+        if constexpr (F8) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
-          const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
-          umma_bf16(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
+            umma_ts(tmem + tS + buf * H, tmem + tKA + buf * (D / 2) + kk * 8, bq, IDESC_S, kk > 0);
+          }
+          umma_commit(&s_full[buf]);
+          umma_commit(&ka_empty[buf]);
+        } else {
+          const uint64_t ka = sdesc(smem_u32(sR + s * KT_BYTES), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
+            const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
+            umma_bf16(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
+          }
+          umma_commit(&s_full[buf]);
+          umma_commit(&r_empty[s]);
         }
-        umma_commit(&s_full[buf]);
-        umma_commit(&r_empty[s]);
         ++js;
         return true;
       };
       auto issue_pv = [&](uint32_t jj, uint32_t vidx, bool first) -> bool {
-        const int buf = jj & 1, s = vidx % RING;
+        const int buf = jj & 1, s = vidx % NR;
         if (!wait_bar(&p_full[buf], npu[buf] & 1, limit, &abort_flag, p.st, 214)) return false;
-        if (!wait_bar(&r_full[s], (vidx / RING) & 1, limit, &abort_flag, p.st, 215)) return false;
+        if constexpr (F8) {  // the tile's f16 V (one buffer: one use per PV)
+          if (!wait_bar(&v16_full, npv & 1, limit, &abort_flag, p.st, 218)) return false;
+        } else {
+          if (!wait_bar(&r_full[s], (vidx / NR) & 1, limit, &abort_flag, p.st, 215)) return false;
+        }
         if (first && !wait_bar(&o_empty, (seg2 & 1) ^ 1, limit, &abort_flag, p.st, 216)) return false;
         tc_fence_after();
-        const uint64_t va = sdesc(smem_u32(sR + s * KT_BYTES), TILE * 128, 1024);
+        const uint64_t va = sdesc(smem_u32(F8 ? sV : sR + s * KT_BYTES), TILE * 128, 1024);
         const uint64_t pa = sdesc(smem_u32(sP + buf * P_BYTES), TILE * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) {
@@ -288,8 +343,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           umma_bf16(tmem + tO, a, bb, IDESC_O, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&p_empty[buf]);
-        umma_commit(&r_empty[s]);
+        umma_commit(F8 ? &v16_empty : &r_empty[s]);
         npu[buf]++;
+        ++npv;
         return true;
       };
       for (int g = 0; g < S.n_groups && ok; ++g) {
@@ -299,7 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int b = S.seq_of(t);
           const long long seg_end = t1 < (long long)S.seq_start[b + 1] ? t1 : (long long)S.seq_start[b + 1];
           if (skip_seq(b)) { t = seg_end; continue; }
-          if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
+          if (!wait_bar(qready, nq & 1, limit, &abort_flag, p.st, 210)) { ok = false; break; }
           const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
           for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi && ok; lt += st)
             if (!issue_s(ri++)) ok = false;
@@ -314,7 +370,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (skip_seq(b)) { t = seg_lo - 1; continue; }
           const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
           // S of a tile, then PV of the tile before it
-          if (!wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
+          if (!wait_bar(qready, nq & 1, limit, &abort_flag, p.st, 213)) { ok = false; break; }
           for (uint32_t x = 0; x < n; ++x, ++jp) {
             if (!issue_s(base + (x == 0 ? 0u : 2 * x - 1))) { ok = false; break; }
             if (x > 0 && !issue_pv(jp - 1, base + 2 * x, x == 1)) { ok = false; break; }
@@ -328,6 +384,122 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ri = base + 2 * n;
           t = seg_lo - 1;
         }
+      }
+    }
+  } else if (F8 && warp >= CONV_WARP0) {
+    // ------------------------------------------------------------------ e4m3 widening (FP8 cache)
+    // Takes every ring item in order: the query of a segment (rewritten in place as f16), a K
+    // tile (each thread its key row, f16, into the TMEM buffer of the tile's S MMA), a V tile
+    // (each thread its key row into the f16 V buffer of the tile's PV MMA, zeros past the
+    // sequence). It runs up to two tiles ahead of the MMAs, bounded by those buffers.
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;                 // key within the tile == TMEM lane
+    const int ctid = (warp - CONV_WARP0) * 32 + lane;    // 0..127
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    uint32_t ri = 0, js = 0, jp = 0, nq = 0;
+    uint32_t nv = 0;  // V tiles widened into the f16 buffer
+    bool ok = true;
+    auto widen_q = [&]() -> bool {
+      if (!warp_wait_bar(&q_full, nq & 1, limit, &abort_flag, p.st, 226)) return false;
+      for (int i = ctid; i < Q_BYTES / 16; i += 128) {
+        const uint32_t a = smem_u32(sQ) + i * 16;
+        const uint4 w = ld_shared_v4(a);
+        st_shared_v4(a, bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q16_full);
+      return true;
+    };
+    auto widen_k = [&](uint32_t item, uint32_t jsx) -> bool {
+      const int slot = (int)(item % NR), kb = (int)(jsx & 1);
+      if (!warp_wait_bar(&r_full[slot], (item / NR) & 1, limit, &abort_flag, p.st, 227)) return false;
+      if (!warp_wait_bar(&ka_empty[kb], ((jsx >> 1) & 1) ^ 1, limit, &abort_flag, p.st, 228)) return false;
+      tc_fence_after();
+      const uint32_t src = smem_u32(sR + slot * SLOT_BYTES);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t w[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint4 x = ld_shared_v4(src + sw128_off(row, hh * 4 + c4));
+          e4m3x4_to_f16x4(x.x, w[c4 * 8 + 0], w[c4 * 8 + 1]);
+          e4m3x4_to_f16x4(x.y, w[c4 * 8 + 2], w[c4 * 8 + 3]);
+          e4m3x4_to_f16x4(x.z, w[c4 * 8 + 4], w[c4 * 8 + 5]);
+          e4m3x4_to_f16x4(x.w, w[c4 * 8 + 6], w[c4 * 8 + 7]);
+        }
+        tmem_st32(tmem + lane_base + tKA + kb * (D / 2) + hh * 32, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(&ka_full[kb]); mbar_arrive(&r_empty[slot]); }
+      return true;
+    };
+    auto widen_v = [&](uint32_t item, bool valid_row) -> bool {
+      const int slot = (int)(item % NR);
+      if (!warp_wait_bar(&r_full[slot], (item / NR) & 1, limit, &abort_flag, p.st, 229)) return false;
+      // the row's 8 chunks in registers first (the e4m3 slot is then free), then the f16 buffer
+      // once the previous PV has read it
+      const uint32_t src = smem_u32(sR + slot * SLOT_BYTES), dst = smem_u32(sV);
+      uint4 x[D / 16];
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c)
+        x[c] = valid_row ? ld_shared_v4(src + sw128_off(row, c)) : make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&r_empty[slot]);
+      if (!warp_wait_bar(&v16_empty, (nv & 1) ^ 1, limit, &abort_flag, p.st, 232)) return false;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t h[8];
+        e4m3x4_to_f16x4(x[c].x, h[0], h[1]);
+        e4m3x4_to_f16x4(x[c].y, h[2], h[3]);
+        e4m3x4_to_f16x4(x[c].z, h[4], h[5]);
+        e4m3x4_to_f16x4(x[c].w, h[6], h[7]);
+        const uint32_t o = dst + (c / 4) * (TILE * 128);
+        st_shared_v4(o + sw128_off(row, (2 * c) % 8), h[0], h[1], h[2], h[3]);
+        st_shared_v4(o + sw128_off(row, (2 * c + 1) % 8), h[4], h[5], h[6], h[7]);
+      }
+      fence_async_smem();  // read by the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v16_full);
+      ++nv;
+      return true;
+    };
+    for (int g = 0; g < S.n_groups; ++g) {
+      long long t0, t1;
+      S.range(g, cta, t0, t1);
+      for (long long t = t0; t < t1;) {  // phase 1: the query, then the sampled K tiles
+        const int b = S.seq_of(t);
+        const long long seg_end = t1 < (long long)S.seq_start[b + 1] ? t1 : (long long)S.seq_start[b + 1];
+        if (skip_seq(b)) { t = seg_end; continue; }
+        if (ok && !widen_q()) ok = false;
+        ++nq;
+        const int st = sample_stride(S, b, p.sample_tiles), lt_hi = (int)(seg_end - (long long)S.seq_start[b]);
+        for (int lt = first_sample((int)(t - (long long)S.seq_start[b]), st); lt < lt_hi; lt += st, ++ri, ++js)
+          if (ok && !widen_k(ri, js)) ok = false;
+        t = seg_end;
+      }
+      for (long long t = t1 - 1; t >= t0;) {  // phase 2: the query, then K(0) K(1) V(0) K(2) V(1) ...
+        const int b = S.seq_of(t);
+        const long long seg_lo = t0 > (long long)S.seq_start[b] ? t0 : (long long)S.seq_start[b];
+        if (skip_seq(b)) { t = seg_lo - 1; continue; }
+        if (ok && !widen_q()) ok = false;
+        ++nq;
+        const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
+        const int n_b = S.seq_len[b];
+        auto v_valid = [&](uint32_t x) {  // row of tile x (descending from t) inside the sequence
+          return (t - (long long)x - (long long)S.seq_start[b]) * TILE + row < (long long)n_b;
+        };
+        for (uint32_t x = 0; x < n && ok; ++x) {
+          if (!widen_k(base + (x == 0 ? 0u : 2 * x - 1), js + x)) { ok = false; break; }
+          if (x > 0 && !widen_v(base + 2 * x, v_valid(x - 1))) { ok = false; break; }
+        }
+        if (ok && !widen_v(base + 2 * n - 1, v_valid(n - 1))) ok = false;
+        ri = base + 2 * n;
+        js += n;
+        jp += n;
+        t = seg_lo - 1;
       }
     }
   } else {
@@ -513,17 +685,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float mm = red[0][h][0], ll = red[0][h][1];
             for (int w = 1; w < 8; ++w) merge_ml(mm, ll, red[w][h][0], red[w][h][1]);
             const float lse2 = mm + log2f(ll);
-            slse[h] = lse2;  // of the sampled tiles only: the reference of p' = exp2(s*c - lse2)
+            // of the sampled tiles only: the reference of p' = exp2(s*c - lse2); FP8 cache: less
+            // an offset that keeps p' well inside the f16 range of P
+            slse[h] = F8 ? lse2 - (p.fallback ? F8_OFF_EXACT : F8_OFF_SAMPLED) : lse2;
           }
           named_bar(3, 256);
         }
         const uint32_t n = (uint32_t)(t - seg_lo + 1), base = ri;
         float la = 0.f, lb = 0.f;  // sums of p' over this warp's keys for heads 2*lane, 2*lane + 1
+        bool lsum_started = false;  // FP8 cache: this warpgroup's TMEM sums hold a tile of the segment
         for (uint32_t x = 0; x < n; ++x, --t, ++jp, ++js) {
           if ((int)(jp & 1) != wg || !ok) continue;  // the other warpgroup's tile, or unwinding
           const int lt = (int)(t - (long long)S.seq_start[b]);
           const int buf = jp & 1;   // == wg: this warpgroup's P buffer
           const int sbi = js & 1;   // the TMEM S buffer of this tile
+          const int key = lt * TILE + row;
+          const bool valid = key < n_b;
           if (!warp_wait_bar(&s_full[sbi], (js >> 1) & 1, limit, &abort_flag, p.st, 222)) { ok = false; continue; }
           tc_fence_after();
           float v[H];
@@ -538,8 +715,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cnt(&s_empty[sbi], 2);
-          const int key = lt * TILE + row;
-          const bool valid = key < n_b;
           float sa = 0.f, sb = 0.f;
           uint32_t pk[H / 2];
 #pragma unroll
@@ -552,25 +727,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float p2 = valid ? fast_exp2(e2) : 0.f, p3 = valid ? fast_exp2(e3) : 0.f;
             fadd2(sa, sb, sa, sb, p0, p1);
             fadd2(sa, sb, sa, sb, p2, p3);
-            pk[h / 2] = pack_bf16x2(p0, p1);
-            pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+            pk[h / 2] = F8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+            pk[h / 2 + 1] = F8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
             v[h] = p0; v[h + 1] = p1; v[h + 2] = p2; v[h + 3] = p3;
           }
           const float score = sa + sb;
           // p' above 2^64 (or not finite): the sampled reference was far too low for this
-          // sequence; flag it for the exact redo (the sum is above 2^64 iff a term is)
-          if (__any_sync(0xffffffffu, valid && !(score <= 1.8446744e19f)) && lane == 0) {
+          // sequence; flag it for the exact redo (the sum is above 2^64 iff a term is). FP8
+          // cache: the head sum above the f16 range (a sufficient test for every term's fit)
+          if (__any_sync(0xffffffffu, valid && !(score <= (F8 ? F8_MAX_SCORE : 1.8446744e19f))) && lane == 0) {
             if (atomicExch(&p.ovf[b], 1) == 0) atomicAdd(&p.ovf[p.B], 1);
           }
           if (!warp_wait_bar(&p_empty[buf], (npu & 1) ^ 1, limit, &abort_flag, p.st, 223)) { ok = false; continue; }
-          if ((lt + 1) * TILE > n_b) {
+          if (!F8 && (lt + 1) * TILE > n_b) {
             // the sequence's last tile, partial: its V rows past the sequence hold whatever the
             // caller's buffer holds there (rows of a longer sequence's slot in a ragged batch).
             // P is 0 for them, but 0 * inf is NaN in the PV product: zero those rows first. The
             // tile's V item cannot be overwritten before this warpgroup's P releases its PV.
             const uint32_t vi = x == n - 1 ? base + 2 * n - 1 : base + 2 * x + 2;
-            const int vs = (int)(vi % RING);
-            if (!warp_wait_bar(&r_full[vs], (vi / RING) & 1, limit, &abort_flag, p.st, 225)) { ok = false; continue; }
+            const int vs = (int)(vi % NR);
+            if (!warp_wait_bar(&r_full[vs], (vi / NR) & 1, limit, &abort_flag, p.st, 225)) { ok = false; continue; }
             if (!valid) {
               const uint32_t vrow = smem_u32(sR + vs * KT_BYTES);
 #pragma unroll
@@ -587,22 +763,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[buf]);
           ++npu;
-          // per-head sums over the warp's 32 keys by a reduce-scatter: at each step a lane keeps
-          // half of its values and adds its partner's copy of that half; at the end lane L holds
-          // heads 2L and 2L + 1
+          if constexpr (F8) {
+            // this key row's p' per head added into the warpgroup's TMEM sums (lane = row); the
+            // sums over the rows are formed once, at the end of the segment
+            const uint32_t la_addr = tmem + lane_base + tLA + wg * H;
 #pragma unroll
-          for (int stp = 0; stp < 5; ++stp) {
-            const int cnt = 64 >> stp, dist = 16 >> stp;
-            const bool up = (lane & dist) != 0;
+            for (int hb = 0; hb < H / 16; ++hb) {
+              float acc[16];
+              if (lsum_started) {
+                tmem_ld16(la_addr + hb * 16, acc);
+                tmem_ld_wait();
+              } else {
 #pragma unroll
-            for (int i = 0; i < cnt / 2; ++i) {
-              const float send = up ? v[i] : v[i + cnt / 2];
-              const float keep = up ? v[i + cnt / 2] : v[i];
-              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, dist);
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < 16; i += 2)
+                fadd2(acc[i], acc[i + 1], acc[i], acc[i + 1], v[hb * 16 + i], v[hb * 16 + i + 1]);
+              tmem_st16(la_addr + hb * 16, acc);
             }
+            tmem_st_wait();
+            lsum_started = true;
+          } else {
+            // per-head sums over the warp's 32 keys by a reduce-scatter: at each step a lane keeps
+            // half of its values and adds its partner's copy of that half; at the end lane L holds
+            // heads 2L and 2L + 1
+#pragma unroll
+            for (int stp = 0; stp < 5; ++stp) {
+              const int cnt = 64 >> stp, dist = 16 >> stp;
+              const bool up = (lane & dist) != 0;
+#pragma unroll
+              for (int i = 0; i < cnt / 2; ++i) {
+                const float send = up ? v[i] : v[i + cnt / 2];
+                const float keep = up ? v[i + cnt / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, dist);
+              }
+            }
+            la += v[0];
+            lb += v[1];
           }
-          la += v[0];
-          lb += v[1];
           const bool is_cand = valid && key < ncand;
           if (is_cand) p.sc[(size_t)b * p.sc_stride + key] = score;
           const unsigned bin = (__float_as_uint(score) >> 20) & (NBINS - 1);
@@ -613,6 +812,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         ri = base + 2 * n;
+        if constexpr (F8) {
+          // the warpgroup's TMEM sums over its rows: one reduce-scatter per segment (lane L ends
+          // with heads 2L and 2L + 1 of its warp's 32 rows)
+          if (lsum_started && ok) {
+            float v[H];
+#pragma unroll
+            for (int hb = 0; hb < H / 32; ++hb) {
+              float tmp[32];
+              tmem_ld32(tmem + lane_base + tLA + wg * H + hb * 32, tmp);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[hb * 32 + i] = tmp[i];
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int stp = 0; stp < 5; ++stp) {
+              const int cnt = 64 >> stp, dist = 16 >> stp;
+              const bool up = (lane & dist) != 0;
+#pragma unroll
+              for (int i = 0; i < cnt / 2; ++i) {
+                const float send = up ? v[i] : v[i + cnt / 2];
+                const float keep = up ? v[i + cnt / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, dist);
+              }
+            }
+            la = v[0];
+            lb = v[1];
+          }
+        }
         {  // this segment's per-head sums of p' over its keys: one record per (sequence, CTA)
           float* rr = &red[0][0][0];  // [8 warps][64 heads]
           rr[swarp * H + 2 * lane] = la;
@@ -772,24 +999,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, 256); }
+  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem, TMEM_COLS); }
 }
 
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
-size_t fused_smem_bytes(int H, int D) {
-  return 1024 + (size_t)H * D * 2 + RING * (size_t)TILE * D * 2 + 2 * (size_t)TILE * H * 2 + NBINS * 4;
+size_t fused_smem_bytes(int H, int D, bool f8) {
+  const size_t ring = f8 ? RING8 * (size_t)TILE * D + (size_t)TILE * D * 2 : RING * (size_t)TILE * D * 2;
+  return 1024 + (size_t)H * D * 2 + ring + 2 * (size_t)TILE * H * 2 + NBINS * 4;
 }
 
 cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                               const DecParams& p, cudaStream_t stream) {
+                               const DecParams& p, bool f8, cudaStream_t stream) {
   constexpr int H = 64, D = 128;
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(dec_fused_kernel<H, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)fused_smem_bytes(H, D));
-    configured = true;
+  static bool configured[2] = {false, false};
+  auto* kern = f8 ? dec_fused_kernel<H, D, true> : dec_fused_kernel<H, D, false>;
+  if (!configured[f8]) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes(H, D, f8));
+    configured[f8] = true;
   }
   // the sampled launch, then the exact redo of any sequence it flagged (normally none: the redo's
   // CTAs read the flag count and leave at once). Every CTA waits for all others at the grid
@@ -803,8 +1031,8 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.sch.G);
-    cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = fused_smem_bytes(H, D);
+    cfg.blockDim = dim3(f8 ? NTHREADS_F8 : NTHREADS);
+    cfg.dynamicSmemBytes = fused_smem_bytes(H, D, f8);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -816,7 +1044,7 @@ cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, c
     cudaError_t e;
     {
       LaunchScope ls(pass == 0 ? "dec_fused" : "dec_redo", stream);
-      e = cudaLaunchKernelEx(&cfg, dec_fused_kernel<H, D>, tmK, tmV, tmQ, q);
+      e = cudaLaunchKernelEx(&cfg, kern, tmK, tmV, tmQ, q);
     }
     if (e != cudaSuccess) return e;
   }

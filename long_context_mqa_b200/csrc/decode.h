@@ -41,9 +41,10 @@ struct DecParams {
   int max_pages, n_pages;  // table width, pages in the K/V pools
   DevStatus* st;
 };
-size_t fused_smem_bytes(int H, int D);
+size_t fused_smem_bytes(int H, int D, bool f8);
+// f8: K and V are e4m3 caches (tensor maps of bytes, 128-byte rows); c then includes K's scale
 cudaError_t launch_decode_attn(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                               const DecParams& p, cudaStream_t stream);
+                               const DecParams& p, bool f8, cudaStream_t stream);
 }  // namespace dec
 
 namespace sel {
@@ -66,12 +67,14 @@ struct SelParams {
   // output records of the decode kernel, summed into out by the collect kernel's extra CTAs
   const float* opart;            // unnormalised output records, at Sched::slot
   const float* lsum;             // [B][H] totals L' dividing them
+  float oscale;                  // factor of the output (an e4m3 V cache's scale, else 1)
   __nv_bfloat16* out;            // [B][H][D]
   int H, D;
   dec::Sched sch;
   // exact re-score of the band keys
   const __nv_bfloat16* qry;      // [B][H][D] the decode queries
   const __nv_bfloat16* kc;       // [B][N][D] the K cache (sequence b's first seq_len[b] rows)
+  const uint8_t* kc8;            // the same as e4m3 codes (FP8 cache; kc unused), c includes its scale
   const float* lse2x;            // [B][H] exact lse, log2 units
   float c;                       // scale * log2(e)
   int sms;
@@ -86,6 +89,8 @@ cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
 namespace sparse {
 struct SpParams {
   const __nv_bfloat16 *Q, *K, *V;
+  const uint8_t *K8, *V8;     // FP8 cache: e4m3 codes (K, V unused); c includes K's scale
+  float oscale;               // factor of the output (the e4m3 V cache's scale, else 1)
   const int32_t* idx;
   int B, Lq, Lk, S;
   int nsplit, split_slots;    // CTAs per query row (a cluster when > 1, at most 16) and the

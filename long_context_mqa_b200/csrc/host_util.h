@@ -13,11 +13,12 @@
 
 namespace hs2 {
 
-// Encodes a 3D bf16 tensor map: dims (inner, rows, batch) with strides in elements,
-// box (box_inner, box_rows, 1), 128-byte swizzle, out-of-range elements read as zero.
+// Encodes a 3D tensor map of bf16 (elem_bytes 2) or bytes (1): dims (inner, rows, batch) with
+// strides in elements, box (box_inner, box_rows, 1), 128-byte swizzle, out-of-range elements
+// read as zero.
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                   uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner, uint32_t box_rows,
-                  bool swizzle128 = true);
+                  bool swizzle128 = true, int elem_bytes = 2);
 
 // 2D variant: dims (inner, rows), row stride in elements.
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_el,

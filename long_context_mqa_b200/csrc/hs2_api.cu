@@ -34,14 +34,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                   uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner, uint32_t box_rows,
-                  bool swizzle128) {
+                  bool swizzle128, int elem_bytes) {
   auto enc = get_encoder();
-  if (!enc) return false;
+  if (!enc || (elem_bytes != 1 && elem_bytes != 2)) return false;
   cuuint64_t dims[3] = {inner, rows, batch};
-  cuuint64_t strides[2] = {row_stride_el * 2, batch_stride_el * 2};
+  cuuint64_t strides[2] = {row_stride_el * elem_bytes, batch_stride_el * elem_bytes};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return enc(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -258,6 +259,19 @@ __global__ void selftest_wait_kernel(DevStatus* st, long long limit_ns) {
   if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns)) report_status(st, kStatusTimeout, 900);
 }
 
+// the device conversions of e4m3 codes, one pair per thread (checked against the format's
+// definition by the tests)
+__global__ void selftest_e4m3_kernel(const uint8_t* x, uint16_t* y_f16, uint16_t* y_bf16, int n_pairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pairs) return;
+  const uint32_t w = (uint32_t)x[2 * i] | ((uint32_t)x[2 * i + 1] << 8);
+  const uint32_t h = e4m3x2_to_f16x2(w), bf = e4m3_f16x2_to_bf16x2(h);
+  y_f16[2 * i] = (uint16_t)(h & 0xFFFFu);
+  y_f16[2 * i + 1] = (uint16_t)(h >> 16);
+  y_bf16[2 * i] = (uint16_t)(bf & 0xFFFFu);
+  y_bf16[2 * i + 1] = (uint16_t)(bf >> 16);
+}
+
 }  // namespace hs2
 
 using namespace hs2;
@@ -293,11 +307,13 @@ size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d,
 }
 
 // The decode path (one query per sequence at the end of its lens[b]-token cache). K, V are
-// [B][Lk] rows, or (ptab != NULL) pools of n_pages pages of 128 rows with Lk = max_pages * 128.
-static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, const int* lens, int Lk,
+// [B][Lk] rows, or (ptab != NULL) pools of n_pages pages of 128 rows with Lk = max_pages * 128;
+// bf16, or (f8) e4m3 codes with c including K's scale and oscale V's.
+static hs2_status run_decode(const void* Q, const void* K, const void* V, int B, const int* lens, int Lk,
                              int H, int d, float c, int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
                              void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
-                             const int32_t* ptab = nullptr, int max_pages = 0, int n_pages = 0) {
+                             const int32_t* ptab = nullptr, int max_pages = 0, int n_pages = 0, bool f8 = false,
+                             float oscale = 1.f) {
   if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
   DecodeWs w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
   if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
@@ -311,18 +327,23 @@ static hs2_status run_decode(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf1
   // contiguous: (d, Lk rows, B sequences); paged: (d, 128 rows, n_pages pages)
   const uint64_t rows = ptab ? 128 : (uint64_t)Lk, planes = ptab ? (uint64_t)n_pages : (uint64_t)B;
   CUtensorMap tmK, tmV, tmQ;
-  if (!make_tmap_3d(&tmK, K, d, rows, planes, d, rows * d, 64, 128) ||
-      !make_tmap_3d(&tmV, V, d, rows, planes, d, rows * d, 64, 128) ||
+  // bf16: boxes of 64 elements (128 bytes) x 128 rows; e4m3: the whole 128-byte row in one box
+  const uint32_t kbox = f8 ? 128 : 64;
+  const int eb = f8 ? 1 : 2;
+  if (!make_tmap_3d(&tmK, K, d, rows, planes, d, rows * d, kbox, 128, true, eb) ||
+      !make_tmap_3d(&tmV, V, d, rows, planes, d, rows * d, kbox, 128, true, eb) ||
       !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
     return HS2_ERR_CUDA;
-  if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, st) != cudaSuccess) return HS2_ERR_CUDA;
+  if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, f8, st) != cudaSuccess) return HS2_ERR_CUDA;
   sel::SelParams sp;
   sp.opart = w.p.opart;
   sp.out = reinterpret_cast<__nv_bfloat16*>(out);
   sp.H = H; sp.D = d; sp.sch = w.p.sch;
   sp.lsum = w.p.lsum;
+  sp.oscale = oscale;
   sp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
-  sp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
+  sp.kc = f8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(K);
+  sp.kc8 = f8 ? reinterpret_cast<const uint8_t*>(K) : nullptr;
   sp.lse2x = w.p.lse2x;
   sp.gbar = w.p.gbar;
   sp.ptab = ptab;
@@ -434,10 +455,11 @@ size_t hs2_sparse_attn_workspace_bytes(int B, int Lq, int Lk, int H, int d, int 
   return carve_sparse(nullptr, B, Lq, H, d, S, sms, nullptr);
 }
 
-static hs2_status run_sparse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx, int B,
+// K, V: bf16 rows, or (f8) e4m3 codes whose scales multiply the logits (k_scale) and the output
+static hs2_status run_sparse(const hs2_bf16* Q, const void* K, const void* V, const int32_t* idx, int B,
                              int Lq, int Lk, int H, int d, int S, float scale, hs2_bf16* out, float* lse,
                              void* workspace, size_t workspace_bytes, hs2_stream stream, const int32_t* ptab,
-                             int max_pages, int n_pages) {
+                             int max_pages, int n_pages, bool f8 = false, float k_scale = 1.f, float v_scale = 1.f) {
   if (!Q || !K || !V || !idx || !out) return HS2_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (lse && !aligned16(lse)))
     return HS2_ERR_INVALID_ARG;
@@ -453,11 +475,14 @@ static hs2_status run_sparse(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf1
   const size_t need = carve_sparse(workspace, B, Lq, H, d, S, sms, &p);
   if (workspace_bytes < need) return HS2_ERR_WORKSPACE;
   p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
-  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
-  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.K = f8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = f8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(V);
+  p.K8 = f8 ? reinterpret_cast<const uint8_t*>(K) : nullptr;
+  p.V8 = f8 ? reinterpret_cast<const uint8_t*>(V) : nullptr;
+  p.oscale = v_scale;
   p.idx = idx;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.S = S;
-  p.c = scale * 1.4426950408889634f;
+  p.c = scale * k_scale * 1.4426950408889634f;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.wait_ns = wait_limit_ns();
@@ -483,6 +508,71 @@ hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, con
   if (n_pages <= 0 || max_pages <= 0 || max_pages > (1 << 23)) return HS2_ERR_INVALID_ARG;
   return run_sparse(Q, K_pages, V_pages, idx, B, Lq, max_pages * 128, H, d, S, scale, out, lse, workspace,
                     workspace_bytes, stream, page_table, max_pages, n_pages);
+}
+
+static bool kv_scale_ok(float s) { return s > 0.f && s < INFINITY; }
+
+size_t hs2_full_attn_select_fp8kv_workspace_bytes(int B, const int32_t* lens, int Lk, int H, int d, int window,
+                                                  int topk) {
+  if (B <= 0 || B > dec::kMaxSeqs || Lk <= 0 || H != 64 || d != 128 || window < 1 || topk < 0) return 0;
+  if (lens) return hs2_full_attn_select_ragged_workspace_bytes(B, lens, Lk, H, d, window, topk);
+  std::vector<int32_t> all((size_t)B, Lk);
+  return hs2_full_attn_select_ragged_workspace_bytes(B, all.data(), Lk, H, d, window, topk);
+}
+
+hs2_status hs2_full_attn_select_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8, float k_scale,
+                                      float v_scale, int B, const int32_t* lens, int Lk, const int32_t* page_table,
+                                      int max_pages, int n_pages, int H, int d, float scale, int window, int topk,
+                                      hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                      size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K8 || !V8 || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K8) || !aligned16(V8) || !aligned16(out) || !aligned16(lse) || !aligned16(idx))
+    return HS2_ERR_INVALID_ARG;
+  if (!kv_scale_ok(k_scale) || !kv_scale_ok(v_scale)) return HS2_ERR_INVALID_ARG;
+  if (Lk <= 0 || window < 1 || topk < 0 || !(scale > 0.f) || B <= 0) return HS2_ERR_INVALID_ARG;
+  if (page_table) {
+    if ((reinterpret_cast<uintptr_t>(page_table) & 3u) != 0 || n_pages <= 0 || max_pages <= 0 ||
+        max_pages > (1 << 23) || Lk != max_pages * 128)
+      return HS2_ERR_INVALID_ARG;
+  }
+  if (B > dec::kMaxSeqs) return HS2_ERR_UNSUPPORTED_SHAPE;
+  std::vector<int> all;
+  const int* ln = reinterpret_cast<const int*>(lens);
+  if (!lens) {
+    all.assign((size_t)B, Lk);
+    ln = all.data();
+  } else if (!ragged_lens_ok(B, lens, Lk)) {
+    return HS2_ERR_INVALID_ARG;
+  }
+  if (window + topk > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  return run_decode(Q, K8, V8, B, ln, Lk, H, d, scale * k_scale * 1.4426950408889634f, window, topk, out, lse, idx,
+                    workspace, workspace_bytes, num_sms(), reinterpret_cast<cudaStream_t>(stream), page_table,
+                    page_table ? max_pages : 0, page_table ? n_pages : 0, true, v_scale);
+}
+
+hs2_status hs2_sparse_attn_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8, float k_scale,
+                                 float v_scale, const int32_t* idx, int B, int Lq, int Lk, const int32_t* page_table,
+                                 int max_pages, int n_pages, int H, int d, int S, float scale, hs2_bf16* out,
+                                 float* lse, void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (!kv_scale_ok(k_scale) || !kv_scale_ok(v_scale)) return HS2_ERR_INVALID_ARG;
+  if (page_table) {
+    if ((reinterpret_cast<uintptr_t>(page_table) & 3u) != 0 || n_pages <= 0 || max_pages <= 0 ||
+        max_pages > (1 << 23) || Lk != max_pages * 128)
+      return HS2_ERR_INVALID_ARG;
+  }
+  return run_sparse(Q, K8, V8, idx, B, Lq, Lk, H, d, S, scale, out, lse, workspace, workspace_bytes, stream,
+                    page_table, page_table ? max_pages : 0, page_table ? n_pages : 0, true, k_scale, v_scale);
+}
+
+hs2_status hs2_selftest_e4m3(const uint8_t* x, uint16_t* y_f16, uint16_t* y_bf16, int n, hs2_stream stream) {
+  if (!x || !y_f16 || !y_bf16 || n < 0 || (n & 1)) return HS2_ERR_INVALID_ARG;
+  if (n == 0) return HS2_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  selftest_e4m3_kernel<<<(n / 2 + 255) / 256, 256, 0, st>>>(x, y_f16, y_bf16, n / 2);
+  return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
 size_t hs2_bridge_kv_proj_workspace_bytes(int T, int hidden, int n_layers, int d) {

@@ -47,7 +47,7 @@ __device__ __forceinline__ void combine_output(const SelParams& p, int b, int h,
     const float4 v = __ldcg(rec + i * rstride);
     acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
   }
-  const float inv = 1.f / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
+  const float inv = p.oscale / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
   __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * lane;
   reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
   reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
@@ -188,7 +188,29 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
         krow = (long long)b * p.N + j;
       }
     }
-    {
+    if (p.kc8) {
+      // e4m3 cache: 128-byte rows, 8 lanes per row, 16 codes per lane widened exactly to bf16
+      const int sub = lane >> 3, ch = lane & 7;
+      uint4 x[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const long long kr = __shfl_sync(0xffffffffu, krow, 4 * it + sub);
+        x[it] = kr >= 0 ? __ldg(reinterpret_cast<const uint4*>(p.kc8 + (size_t)kr * D) + ch) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const uint32_t row_base = smem_u32(sK) + (ch / 4) * (TILE * 128);
+        const int rr = warp * 32 + 4 * it + sub;
+        st_shared_v4(row_base + sw128_off(rr, (2 * ch) % 8), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].x)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].x >> 16)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].y)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].y >> 16)));
+        st_shared_v4(row_base + sw128_off(rr, (2 * ch + 1) % 8), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].z)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].z >> 16)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].w)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x[it].w >> 16)));
+      }
+    } else {
       const int sub = lane >> 4, ch = lane & 15;
 #pragma unroll
       for (int it = 0; it < 16; ++it) {

@@ -127,6 +127,39 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     const unsigned m = __ballot_sync(0xffffffffu, valid);
     if (lane == 0) vmask[warp] = m;
     const uint32_t kd = smem_u32(sK), vd = smem_u32(sV);
+    if (p.K8) {
+      // e4m3 cache: rows of D bytes, LPR8 lanes per row, 16 codes per lane, widened exactly to
+      // bf16 in registers (all loads issued before the first conversion)
+      constexpr int LPR8 = D / 16, RPS8 = 32 / LPR8;
+      const int sub8 = lane / LPR8, ch8 = lane % LPR8;
+      const uint8_t* K8b = p.ptab ? p.K8 : p.K8 + (size_t)b * p.Lk * D;
+      const uint8_t* V8b = p.ptab ? p.V8 : p.V8 + (size_t)b * p.Lk * D;
+      uint4 xk[32 / RPS8], xv[32 / RPS8];
+#pragma unroll
+      for (int it = 0; it < 32 / RPS8; ++it) {
+        const long long kr = __shfl_sync(0xffffffffu, krow, it * RPS8 + sub8);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        xk[it] = kr >= 0 ? __ldg(reinterpret_cast<const uint4*>(K8b + (size_t)kr * D) + ch8) : z;
+        xv[it] = kr >= 0 ? __ldg(reinterpret_cast<const uint4*>(V8b + (size_t)kr * D) + ch8) : z;
+      }
+      auto put = [&](uint32_t base, int rr, const uint4& x) {
+        const uint32_t o = base + (ch8 / 4) * (TILE * 128);
+        st_shared_v4(o + sw128_off(rr, (2 * ch8) % 8), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.x)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.x >> 16)), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.y)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.y >> 16)));
+        st_shared_v4(o + sw128_off(rr, (2 * ch8 + 1) % 8), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.z)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.z >> 16)), e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.w)),
+                     e4m3_f16x2_to_bf16x2(e4m3x2_to_f16x2(x.w >> 16)));
+      };
+#pragma unroll
+      for (int it = 0; it < 32 / RPS8; ++it) {
+        const int rr = warp * 32 + it * RPS8 + sub8;
+        put(kd, rr, xk[it]);
+        put(vd, rr, xv[it]);
+      }
+      cp_async_commit();  // (an empty group: the wait before the MMAs stays uniform)
+      return;
+    }
     const int sub = lane / LPR, ch = lane % LPR;
 #pragma unroll
     for (int it = 0; it < 32 / RPS; ++it) {
@@ -285,7 +318,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
         tmem_ld32(tmem + lane_base + tO + cc * 32, o);
         tmem_ld_wait();
         if (owns) {
-          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          const float inv = l_run > 0.f ? p.oscale / l_run : 0.f;
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(o[2 * x] * inv, o[2 * x + 1] * inv);
@@ -358,7 +391,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
         wgt[s2 * MH + tid] = w;
         L += l * w;
       }
-      wgt[16 * MH + tid] = L > 0.f ? 1.f / L : 0.f;
+      wgt[16 * MH + tid] = L > 0.f ? p.oscale / L : 0.f;
       if (p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
     }
   }
