@@ -166,6 +166,22 @@ HS2_API hs2_status hs2_full_attn_select_fp8kv(const hs2_bf16* Q, const uint8_t* 
                                               int32_t* idx, void* workspace, size_t workspace_bytes,
                                               hs2_stream stream);
 
+/* Whole prompts and chunks over an FP8 cache: the arguments of hs2_full_attn_select with K8, V8
+ * [B, Lk, d] e4m3 codes and k_scale, v_scale as above. Lq == 1 with (H, d) = (64, 128) runs the
+ * FP8 decode kernels (as hs2_full_attn_select_fp8kv with lens NULL); otherwise the cache is
+ * widened once into the workspace as bf16 (k_scale * K8, v_scale * V8, rounded to bf16: exact for
+ * power-of-two scales) and the prefill kernels run on it (they are tensor-bound and read the cache
+ * from L2 many times). Results equal hs2_full_attn_select on that bf16 cache. Supported: as
+ * hs2_full_attn_select. Workspace: hs2_full_attn_select_prefill_fp8kv_workspace_bytes.
+ */
+HS2_API size_t hs2_full_attn_select_prefill_fp8kv_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window,
+                                                                  int topk);
+HS2_API hs2_status hs2_full_attn_select_prefill_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8,
+                                                      float k_scale, float v_scale, int B, int Lq, int Lk, int H,
+                                                      int d, float scale, int window, int topk, hs2_bf16* out,
+                                                      float* lse, int32_t* idx, void* workspace,
+                                                      size_t workspace_bytes, hs2_stream stream);
+
 /* ---------------------------------------------------------------------------------
  * Sparse attention over selected tokens (one sparse layer)
  * ---------------------------------------------------------------------------------

@@ -72,6 +72,11 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_full_attn_select_fp8kv.argtypes = [P, P, P, f32, f32, i32, P, i32, P, i32, i32, i32, i32, f32, i32, i32,
                                                P, P, P, P, sz, P]
     lib.hs2_full_attn_select_fp8kv.restype = i32
+    lib.hs2_full_attn_select_prefill_fp8kv_workspace_bytes.argtypes = [i32] * 7
+    lib.hs2_full_attn_select_prefill_fp8kv_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select_prefill_fp8kv.argtypes = [P, P, P, f32, f32, i32, i32, i32, i32, i32, f32, i32, i32, P, P,
+                                                       P, P, sz, P]
+    lib.hs2_full_attn_select_prefill_fp8kv.restype = i32
     lib.hs2_sparse_attn_fp8kv.argtypes = [P, P, P, f32, f32, P, i32, i32, i32, P, i32, i32, i32, i32, i32, f32, P, P,
                                           P, sz, P]
     lib.hs2_sparse_attn_fp8kv.restype = i32
@@ -337,6 +342,32 @@ def full_attn_select_fp8kv(q, k8, v8, k_scale, v_scale, *, lens=None, page_table
                                           lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
                                           ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(code, "hs2_full_attn_select_fp8kv")
+    return out, lse, idx
+
+
+def full_attn_select_prefill_fp8kv(q, k8, v8, k_scale, v_scale, *, scale=None, window=WINDOW, topk=TOPK, out=None,
+                                   lse=None, idx=None, workspace=None, stream=None):
+    """Full attention + selection of Lq queries over an e4m3 K/V cache [B,Lk,d]
+    (hs2_full_attn_select_prefill_fp8kv): a whole prompt (Lq == Lk), a chunk (Lq < Lk) or one
+    decode query. Returns (out, lse, idx) as full_attn_select."""
+    _need(q, "q", torch.bfloat16, 4)
+    B, Lq, H, d = q.shape
+    Lk, _, _ = _fp8_cache(k8, v8, None, B, d)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = window + topk
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, Lq, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    nbytes = int(lib.hs2_full_attn_select_prefill_fp8kv_workspace_bytes(B, Lq, Lk, H, d, window, topk))
+    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    code = lib.hs2_full_attn_select_prefill_fp8kv(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(k_scale),
+                                                  float(v_scale), B, Lq, Lk, H, d, scale, window, topk, out.data_ptr(),
+                                                  lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select_prefill_fp8kv")
     return out, lse, idx
 
 

@@ -1,6 +1,7 @@
 // C ABI of the hs2 library (declared in include/hs2.h): argument validation, workspace
 // layout, TMA descriptor set-up and dispatch to the kernel files. No allocation, no
 // synchronisation and no host fallback on the compute paths.
+#include <algorithm>
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
@@ -270,6 +271,29 @@ __global__ void selftest_e4m3_kernel(const uint8_t* x, uint16_t* y_f16, uint16_t
   y_f16[2 * i + 1] = (uint16_t)(h >> 16);
   y_bf16[2 * i] = (uint16_t)(bf & 0xFFFFu);
   y_bf16[2 * i + 1] = (uint16_t)(bf >> 16);
+}
+
+// e4m3 codes times `scale` -> bf16 (exact when the scale is a power of two), 16 codes per thread
+// per step; n16 = number of 16-code groups
+__global__ void widen_e4m3_kernel(const uint8_t* x, float scale, __nv_bfloat16* y, long long n16) {
+  griddep_wait();
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n16; i += stride) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(x) + i);
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t h0, h1;
+      e4m3x4_to_f16x4(in[j], h0, h1);
+      const uint32_t b0 = e4m3_f16x2_to_bf16x2(h0), b1 = e4m3_f16x2_to_bf16x2(h1);
+      o[2 * j] = pack_bf16x2(__uint_as_float(b0 << 16) * scale, __uint_as_float(b0 & 0xFFFF0000u) * scale);
+      o[2 * j + 1] = pack_bf16x2(__uint_as_float(b1 << 16) * scale, __uint_as_float(b1 & 0xFFFF0000u) * scale);
+    }
+    uint4* d = reinterpret_cast<uint4*>(y) + 2 * i;
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
 }
 
 }  // namespace hs2
@@ -565,6 +589,60 @@ hs2_status hs2_sparse_attn_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uin
   }
   return run_sparse(Q, K8, V8, idx, B, Lq, Lk, H, d, S, scale, out, lse, workspace, workspace_bytes, stream,
                     page_table, page_table ? max_pages : 0, page_table ? n_pages : 0, true, k_scale, v_scale);
+}
+
+// The whole-prompt / chunk entry over an e4m3 cache: one query per sequence goes to the FP8
+// decode kernels; otherwise the cache is widened once into the workspace and the prefill kernels
+// (tensor-bound: the cache is read from L2 many times) run on the bf16 copy.
+static size_t fp8_cache_copy_bytes(int B, int Lk, int d) { return align256((size_t)B * Lk * d * 2); }
+
+size_t hs2_full_attn_select_prefill_fp8kv_workspace_bytes(int B, int Lq, int Lk, int H, int d, int window, int topk) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H <= 0 || d <= 0 || window < 1 || topk < 0) return 0;
+  if (Lq == 1 && H == 64 && d == 128) return hs2_full_attn_select_fp8kv_workspace_bytes(B, nullptr, Lk, H, d, window, topk);
+  const int sms = num_sms() > 0 ? num_sms() : 148;
+  return align256(prefill::workspace_bytes(B, Lq, Lk, H, d, window, topk, sms, kStatusBytes)) +
+         2 * fp8_cache_copy_bytes(B, Lk, d);
+}
+
+hs2_status hs2_full_attn_select_prefill_fp8kv(const hs2_bf16* Q, const uint8_t* K8, const uint8_t* V8, float k_scale,
+                                              float v_scale, int B, int Lq, int Lk, int H, int d, float scale,
+                                              int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
+                                              void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (Lq == 1 && H == 64 && d == 128)
+    return hs2_full_attn_select_fp8kv(Q, K8, V8, k_scale, v_scale, B, nullptr, Lk, nullptr, 0, 0, H, d, scale, window,
+                                      topk, out, lse, idx, workspace, workspace_bytes, stream);
+  if (!Q || !K8 || !V8 || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K8) || !aligned16(V8) || !aligned16(out) || !aligned16(lse) || !aligned16(idx))
+    return HS2_ERR_INVALID_ARG;
+  if (!kv_scale_ok(k_scale) || !kv_scale_ok(v_scale)) return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || window < 1 || topk < 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (window + topk > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!shape_ok(H, d)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  const size_t need = hs2_full_attn_select_prefill_fp8kv_workspace_bytes(B, Lq, Lk, H, d, window, topk);
+  if (need == 0 || workspace_bytes < need) return HS2_ERR_WORKSPACE;
+  const int sms = num_sms();
+  const size_t pre = align256(prefill::workspace_bytes(B, Lq, Lk, H, d, window, topk, sms, kStatusBytes));
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* kb = reinterpret_cast<__nv_bfloat16*>(base + pre);
+  __nv_bfloat16* vb = reinterpret_cast<__nv_bfloat16*>(base + pre + fp8_cache_copy_bytes(B, Lk, d));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long n16 = (long long)B * Lk * d / 16;
+  const int grid = (int)std::min<long long>((n16 + 255) / 256, (long long)sms * 8);
+  {
+    LaunchScope ls("widen_e4m3", st);
+    if (launch_k(widen_e4m3_kernel, dim3(grid), dim3(256), 0, st, true, K8, k_scale, kb, n16) != cudaSuccess)
+      return HS2_ERR_CUDA;
+  }
+  {
+    LaunchScope ls("widen_e4m3", st);
+    if (launch_k(widen_e4m3_kernel, dim3(grid), dim3(256), 0, st, true, V8, v_scale, vb, n16) != cudaSuccess)
+      return HS2_ERR_CUDA;
+  }
+  return prefill::run(Q, reinterpret_cast<const hs2_bf16*>(kb), reinterpret_cast<const hs2_bf16*>(vb), B, Lq, Lk, H,
+                      d, scale * 1.4426950408889634f, window, topk, out, lse, idx, workspace, pre, sms, kStatusBytes,
+                      st);
 }
 
 hs2_status hs2_selftest_e4m3(const uint8_t* x, uint16_t* y_f16, uint16_t* y_bf16, int n, hs2_stream stream) {

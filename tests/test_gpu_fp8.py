@@ -207,3 +207,26 @@ def test_fp8_rejects_bad_scales(hs2):
     for ks in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(hs2.HS2Error):
             hs2.full_attn_select_fp8kv(q, c.k8_d, c.v8_d, ks, c.vs)
+
+
+@pytest.mark.parametrize("name,kw", [("tiny_prefill", {"Lq": 1500, "Lk": 1500}),
+                                     ("prefill_32k", {"B": 2, "Lq": 1100, "Lk": 1100}),
+                                     ("prefill_32k", {"B": 1, "Lq": 700, "Lk": 2500}),
+                                     ("prefill_32k", {"B": 2, "Lq": 1, "Lk": 3000})])
+def test_fp8_prefill_and_chunks(hs2, name, kw):
+    """Whole prompts, a chunk of 700 queries appended to a 1,800-token cache and a single query over
+    an FP8 cache, every row against the oracle on the dequantised cache."""
+    wl = synth.small(name, **kw)
+    g = synth.SyntheticInputs(wl)
+    c = Fp8Cache(g)
+    out, lse, idx = hs2.full_attn_select_prefill_fp8kv(to_torch_bf16(g.q), c.k8_d, c.v8_d, c.ks, c.vs, scale=wl.scale,
+                                                       window=wl.window, topk=wl.topk)
+    torch.cuda.synchronize()
+    assert hs2.read_device_status(hs2.cached_workspace("full")) == 0
+    rows = np.arange(wl.B * wl.Lq)
+    ora = oracle.full_attn_select(g.q, c.k, c.v, wl.scale, wl.window, wl.topk, want_score=True)
+    assert_out_close(bf16_to_f64(out).reshape(ora["out"].shape), ora["out"], f"{wl.name} output (FP8 cache)")
+    assert np.abs(lse.double().cpu().numpy().reshape(ora["lse"].shape) - ora["lse"]).max() < 2e-3
+    st = check_selection(idx.cpu().numpy().reshape(wl.B * wl.Lq, -1), ora["idx"], ora["score"],
+                         wl.Lk - wl.Lq + rows % wl.Lq, wl.window, wl.topk)
+    assert st.ok(), st.failures
