@@ -37,14 +37,16 @@
 // Every wait is bounded; on timeout the kernel records it in the status word and unwinds with
 // its barrier sequence intact.
 //
-// FP8 cache (F8): K and V arrive as e4m3 tiles (16 KB, half the bytes) through a 6-slot ring and
-// the softmax warps widen them exactly to f16: a K row into TMEM, where the S MMA reads its A
-// operand (each thread writes its own key's row: lane = key), a V row into an f16 tile in shared
-// memory for the PV MMA; the query is rewritten in place as f16 when it lands and P is packed
-// as f16, so every MMA is f16 x f16 with fp32 accumulation. The cache's scales are folded into
-// the logit factor c and the output combine. f16 P holds values below 65504: the references are
-// offset (p' = 4 p'' in the sampled pass, 2^12 p in the exact redo, both cancelling in O / L')
-// and a key whose head sum passes 65504 is flagged for the redo.
+// FP8 cache (F8, 448 threads): K and V arrive as e4m3 tiles (16 KB, half the bytes) through an
+// 8-slot ring, and a fourth warpgroup (warps 10..13) widens them exactly to f16: a K row into
+// TMEM, where the S MMA reads its A operand (each thread writes its own key's row: lane = key),
+// a V row into the f16 tile in shared memory that the next PV MMA reads; it also rewrites each
+// segment's query in place as f16, and P is packed as f16, so every MMA is f16 x f16 with fp32
+// accumulation. The softmax warps keep each row's p' per head in TMEM and sum the rows once per
+// segment. The cache's scales are folded into the logit factor c and the output combine. f16 P
+// holds values below 65504: the references are offset (p' = 4 p'' in the sampled pass, 2^12 p in
+// the exact redo, both cancelling in O / L') and a key whose head sum passes 65504 is flagged
+// for the redo.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
