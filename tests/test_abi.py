@@ -81,3 +81,38 @@ def test_ragged_workspace_query_and_argument_checks():
                                          None, 0, None) == hs2.ERR_INVALID_ARG
     with pytest.raises(ValueError):
         hs2.full_attn_select_ragged_workspace_bytes([10, 0], 100, 64, 128)
+
+
+def test_fp8_workspace_queries_and_argument_checks():
+    import long_context_mqa_b200 as hs2
+    L = hs2.lib
+    # decode over an e4m3 cache: the ragged call's workspace (lens NULL: every sequence full)
+    assert hs2.full_attn_select_fp8kv_workspace_bytes(8, None, 262144, 64, 128) == \
+        hs2.full_attn_select_ragged_workspace_bytes([262144] * 8, 262144, 64, 128)
+    lens = [40000, 3000, 1]
+    assert hs2.full_attn_select_fp8kv_workspace_bytes(3, lens, 40000, 64, 128) == \
+        hs2.full_attn_select_ragged_workspace_bytes(lens, 40000, 64, 128)
+    # prompts and chunks: room for the widened bf16 K and V; one query: the decode workspace
+    ws = L.hs2_full_attn_select_prefill_fp8kv_workspace_bytes(2, 1000, 3000, 64, 128, 128, 1024)
+    assert ws >= 2 * 2 * 3000 * 128 * 2
+    assert L.hs2_full_attn_select_prefill_fp8kv_workspace_bytes(2, 1, 3000, 64, 128, 128, 1024) == \
+        hs2.full_attn_select_fp8kv_workspace_bytes(2, None, 3000, 64, 128)
+    assert L.hs2_full_attn_select_prefill_fp8kv_workspace_bytes(2, 3001, 3000, 64, 128, 128, 1024) == 0
+    # rejected before any device work: null pointers, then (with aligned stand-in addresses that
+    # are never dereferenced) scales that are not positive and finite, and a page table whose
+    # width does not match Lk
+    assert L.hs2_full_attn_select_fp8kv(None, None, None, 1.0, 1.0, 1, None, 100, None, 0, 0, 64, 128, 0.1, 128, 1024,
+                                        None, None, None, None, 0, None) == hs2.ERR_INVALID_ARG
+    a = 1 << 20
+    for ks in (0.0, -2.0, float("inf"), float("nan")):
+        assert L.hs2_full_attn_select_fp8kv(a, a, a, ks, 1.0, 1, None, 100, None, 0, 0, 64, 128, 0.1, 128, 1024,
+                                            a, a, a, a, 1 << 20, None) == hs2.ERR_INVALID_ARG
+        assert L.hs2_sparse_attn_fp8kv(a, a, a, 1.0, ks, a, 1, 1, 100, None, 0, 0, 64, 128, 1152, 0.1, a, None, a,
+                                       1 << 20, None) == hs2.ERR_INVALID_ARG
+        assert L.hs2_full_attn_select_prefill_fp8kv(a, a, a, ks, 1.0, 1, 50, 100, 64, 128, 0.1, 128, 1024, a, a, a, a,
+                                                    1 << 20, None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_full_attn_select_fp8kv(a, a, a, 1.0, 1.0, 1, None, 1000, a, 4, 10, 64, 128, 0.1, 128, 1024,
+                                        a, a, a, a, 1 << 20, None) == hs2.ERR_INVALID_ARG  # 4 pages != 1000 rows
+    assert L.hs2_sparse_attn_fp8kv(a, a, a, 1.0, 1.0, a, 1, 1, 1000, a, 4, 10, 64, 128, 1152, 0.1, a, None, a,
+                                   1 << 20, None) == hs2.ERR_INVALID_ARG
+    assert L.hs2_selftest_e4m3(a, a, a, 3, None) == hs2.ERR_INVALID_ARG  # odd count
