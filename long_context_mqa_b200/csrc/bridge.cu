@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t a = sdesc_at(da, kk * 32);
             const uint64_t b = sdesc_at(db, kk * 2048);
-            umma_bf16(tmem + ab * BN, a, b, IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
+            umma_ss(tmem + ab * BN, a, b, IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
         }

@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t a = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
             const uint64_t bq = sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32);
-            umma_bf16(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
+            umma_ss(tmem + tS + buf * H, a, bq, IDESC_S, kk > 0);
           }
           umma_commit(&s_full[buf]);
           umma_commit(&r_empty[s]);
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
         for (int kk = 0; kk < TILE / 16; ++kk) {
           const uint64_t a = sdesc_at(va, kk * 2048);
           const uint64_t bb = sdesc_at(pa, kk * 2048);
-          umma_bf16(tmem + tO, a, bb, IDESC_O, (first && kk == 0) ? 0u : 1u);
+          umma_ss(tmem + tO, a, bb, IDESC_O, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&p_empty[buf]);
         umma_commit(F8 ? &v16_empty : &r_empty[s]);

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t a = sdesc_at(qa, (kk / 4) * (128 * 128) + (kk % 4) * 32);
           const uint64_t bk = sdesc_at(ka, (kk / 4) * (128 * 128) + (kk % 4) * 32);
-          umma_bf16(tmem + tS + 128 * w, a, bk, IDESC_S, kk > 0);
+          umma_ss(tmem + tS + 128 * w, a, bk, IDESC_S, kk > 0);
         }
         umma_commit(&s_full[w]);
         ns[w]++;
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int kk = 0; kk < 128 / 16; ++kk) {
           const uint64_t a = sdesc_at(pa, (kk / 4) * (128 * 128) + (kk % 4) * 32);
           const uint64_t bv = sdesc_at(va, kk * 2048);
-          umma_bf16(tmem + tO + D * w, a, bv, IDESC_O, (first && kk == 0) ? 0u : 1u);
+          umma_ss(tmem + tO + D * w, a, bv, IDESC_O, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&pv_done[w]);
         npv[w]++;
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(NT, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t a = sdesc_at(ka, (kk / 4) * (128 * 128) + (kk % 4) * 32);
             const uint64_t bq = sdesc_at(qd, (kk / 4) * (256 * 128) + (kk % 4) * 32);
-            umma_bf16(tmem + buf * 256, a, bq, IDESC, kk > 0);
+            umma_ss(tmem + buf * 256, a, bq, IDESC, kk > 0);
           }
           umma_commit(&s_full[buf]);
           umma_commit(&k_empty[s]);

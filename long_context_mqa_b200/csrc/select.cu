@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(128) sel_rescore_kernel(SelParams p) {
       const uint64_t ka = sdesc(smem_u32(sK), 16, 1024), qa = sdesc(smem_u32(sQ), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_bf16(tmem, sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32),
+        umma_ss(tmem, sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32),
                   sdesc_at(qa, (kk / 4) * (H * 128) + (kk % 4) * 32), IDESC, kk > 0);
       umma_commit(&mma_bar);
     }

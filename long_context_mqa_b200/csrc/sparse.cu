@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t a = sdesc_at(qa, (kk / 4) * (MH * 128) + (kk % 4) * 32);
         const uint64_t bk = sdesc_at(ka, (kk / 4) * (TILE * 128) + (kk % 4) * 32);
-        umma_bf16(tmem + tS, a, bk, IDESC, kk > 0);
+        umma_ss(tmem + tS, a, bk, IDESC, kk > 0);
       }
       umma_commit(&mma_bar);
     }
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
       for (int kk = 0; kk < TILE / 16; ++kk) {
         const uint64_t a = sdesc_at(pa, (kk / 4) * (MH * 128) + (kk % 4) * 32);
         const uint64_t bv = sdesc_at(va, kk * 2048);
-        umma_bf16(tmem + tO, a, bv, IDESC, (t == 0 && kk == 0) ? 0u : 1u);
+        umma_ss(tmem + tO, a, bv, IDESC, (t == 0 && kk == 0) ? 0u : 1u);
       }
       umma_commit(&mma_bar);
     }
