@@ -16,7 +16,7 @@ namespace dec {
 struct DecParams {
   int B, N, W, K;          // sequences, cache rows per sequence in K/V (the longest length), window, top-k
   Sched sch;               // per-sequence lengths and tiles, contiguous tile ranges per CTA
-  float c;                 // scale * log2(e)
+  float c;                 // scale * log2(e) (FP8 cache: times K's scale)
   long long wait_ns;       // bound of every device-side wait
   float* ml;               // [B*cmax][2][H] phase-1 partial (max, sum), log2 domain
   float* lse_out;          // [B][H] natural log (caller's lse)
@@ -76,7 +76,7 @@ struct SelParams {
   const __nv_bfloat16* kc;       // [B][N][D] the K cache (sequence b's first seq_len[b] rows)
   const uint8_t* kc8;            // the same as e4m3 codes (FP8 cache; kc unused), c includes its scale
   const float* lse2x;            // [B][H] exact lse, log2 units
-  float c;                       // scale * log2(e)
+  float c;                       // scale * log2(e) (FP8 cache: times K's scale)
   int sms;
   unsigned* gbar;                // the decode kernel's grid-barrier counters, re-armed here
   const int32_t* ptab;           // paged cache: [B][max_pages] page ids, kc is the page pool (NULL: contiguous)
@@ -95,7 +95,7 @@ struct SpParams {
   int B, Lq, Lk, S;
   int nsplit, split_slots;    // CTAs per query row (a cluster when > 1, at most 16) and the
                               // idx slots each handles (a multiple of 128)
-  float c;                    // scale * log2(e)
+  float c;                    // scale * log2(e) (FP8 cache: times K's scale)
   __nv_bfloat16* out;
   float* lse;                 // may be null
   long long wait_ns;

@@ -8,9 +8,10 @@
 //  2. collect  : every score' above b_hi sets its bit in the sequence's selection bitmap (one bit
 //                per older token, cleared by the decode kernel); band keys are listed by index
 //                (one list-counter update per warp).
-//  3. rescore  : the band keys' K rows are gathered and their exact scores computed (tcgen05,
-//                exact lse), as unique 64-bit keys (score bits << 32 | ~index: larger key ==
-//                higher score, then lower index).
+//  3. rescore  : the band keys' K rows are gathered (an e4m3 cache's rows widened exactly to
+//                bf16 on the way) and their exact scores computed (tcgen05, exact lse), as unique
+//                64-bit keys (score bits << 32 | ~index: larger key == higher score, then lower
+//                index).
 //  4. final    : MSB-first 8-bit radix select of the `need` largest band keys (starting at the
 //                highest bit on which they differ, stopping as soon as the chosen bucket holds
 //                exactly the remaining need) sets their bits; one pass over the bitmap with a
@@ -18,7 +19,7 @@
 //                forced window (every index of which is larger) is appended. Extra CTAs of the
 //                same launch produce the decode output (independent of the selection): per
 //                (sequence, head), the sum of the output records of the CTAs covering the
-//                sequence, divided by L'.
+//                sequence, divided by L' (and multiplied by an e4m3 V cache's scale).
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"

@@ -2,7 +2,8 @@
 //
 // One CTA = one query row (b, i) x one split of its index list. For each tile of 128 index
 // slots the CTA gathers the 128 selected K rows and V rows ONCE for all H heads (MQA: every
-// head reads the same rows) with 16-byte cp.async into 128B-swizzled shared memory, then
+// head reads the same rows) with 16-byte cp.async into 128B-swizzled shared memory (an e4m3
+// cache: 16-byte loads of 16 codes, widened exactly to bf16 in registers, then stored), then
 //   S = Q K_sel^T            tcgen05, M = 64 rows = the heads (padded to 64), N = 128 keys
 //   softmax per head         in-thread: the thread owning a head row holds its 128 logits,
 //                            keeps a running (max, sum) across tiles and rescales its O row
