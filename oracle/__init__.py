@@ -157,6 +157,49 @@ def sparse_attn(q, k, v, idx, scale, rows=None, threads=0):
     return {"out": out, "lse": lse}
 
 
+def block_select(score_row, t, block=64, n_blocks=16):
+    """The HySparse (v1) selection of one query at position t: the n_blocks blocks of `block`
+    consecutive tokens with the largest block score, ties to the lower block; returns the chosen
+    blocks' tokens at or before t, ascending (every token 0..t when at most n_blocks blocks exist).
+
+    The pages give the selection's shape (1,024 global tokens chosen in 64-token blocks, beside a
+    separate 128-token sliding-window branch fused by a gate: arex-research.com, section "外层 KV
+    Bridging，内层 KV Reuse", the paragraph on the two changes from HySparse) but not the block
+    score. Reading taken: a block's score is the sum of the token scores (the full layer's
+    head-summed attention probabilities) of its tokens at or before t; every block that starts at
+    or before t is a candidate (the window branch is separate, so recent blocks compete too).
+    score_row: [>= t + 1] float64 token scores.
+    """
+    score_row = np.asarray(score_row, dtype=np.float64)
+    nb = t // block + 1                       # blocks meeting 0..t
+    if nb <= n_blocks:
+        return np.arange(t + 1, dtype=np.int64)
+    bs = np.array([score_row[j * block:min((j + 1) * block, t + 1)].sum() for j in range(nb)])
+    order = sorted(range(nb), key=lambda j: (-bs[j], j))
+    chosen = sorted(order[:n_blocks])
+    return np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in chosen]).astype(np.int64)
+
+
+def sparse_attn_v1(q, k, v, block_idx, gate, scale, window=128, threads=0):
+    """HySparse (v1) sparse layer: softmax attention over the selected blocks' tokens and over the
+    last `window` tokens (the sliding-window branch), fused per (query, head) as
+    gate * blocks + (1 - gate) * window (same page and section as block_select; the gate is a
+    learned function of the hidden state that the pages do not specify, so it is an input here).
+    q: [B,Lq,H,d], k/v: [B,Lk,d] (bf16 bits); block_idx: [B,Lq,S] token indices (-1 = empty);
+    gate: [B,Lq,H] in [0, 1]. Returns dict(out [B*Lq,H,d] f64)."""
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    gate = np.asarray(gate, dtype=np.float64).reshape(B * Lq, H)
+    win = np.full((B, Lq, window), -1, np.int32)
+    for i in range(Lq):
+        t = Lk - Lq + i
+        lo = max(0, t - window + 1)
+        win[:, i, :t - lo + 1] = np.arange(lo, t + 1, dtype=np.int32)
+    ob = sparse_attn(q, k, v, block_idx, scale, threads=threads)["out"]
+    ow = sparse_attn(q, k, v, win, scale, threads=threads)["out"]
+    return {"out": gate[:, :, None] * ob + (1.0 - gate[:, :, None]) * ow}
+
+
 def bridge_kv_proj(h, w, rows=None, threads=0):
     """KV Bridging. h: [T, hidden], w: [n, 2, hidden, d] -> KV [n, 2, n_rows, d] (f64)."""
     h, w = _u16(h), _u16(w)

@@ -345,3 +345,49 @@ def test_attention_on_e4m3_cache_matches_torch_sdpa():
     V = dec(v8, vs)[:, None].expand(-1, H, -1, -1)
     o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=0.25).permute(0, 2, 1, 3).numpy()
     np.testing.assert_allclose(r["out"], o.reshape(B * Lq, H, d), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# HySparse (v1) block selection and gated window fusion
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("t,block,nb", [(40, 4, 3), (33, 5, 2), (23, 3, 4)])
+def test_block_select_brute_force(t, block, nb):
+    """The chosen blocks maximise the total score of their tokens at or before t over every set
+    of the same size, and among equal totals the lexicographically lowest set wins."""
+    rng = np.random.default_rng(t)
+    # quantised scores so that equal block totals (ties) occur
+    score = rng.integers(0, 4, size=t + 1).astype(np.float64)
+    got = oracle.block_select(score, t, block=block, n_blocks=nb)
+    blocks = range(t // block + 1)
+    total = lambda S: sum(score[j * block:min((j + 1) * block, t + 1)].sum() for j in S)
+    best = max(itertools.combinations(blocks, nb), key=lambda S: (total(S), [-j for j in S]))
+    want = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in sorted(best)])
+    assert np.array_equal(got, want)
+
+
+def test_block_select_closed_forms():
+    # equal scores: the lowest blocks; at most n_blocks blocks: every token 0..t
+    assert np.array_equal(oracle.block_select(np.ones(2000), 1999), np.arange(16 * 64))
+    assert np.array_equal(oracle.block_select(np.ones(1000), 700), np.arange(701))
+    # a block past t never competes; the partial block at t counts only its tokens <= t
+    s = np.zeros(2000); s[1990:] = 100.0; s[0] = 1.0
+    got = oracle.block_select(s, 1500, block=64, n_blocks=1)
+    assert np.array_equal(got, np.arange(64))
+
+
+def test_gated_window_fusion_reduces_to_its_branches():
+    """gate 1: plain attention over the blocks' tokens; gate 0: the window branch, which for a
+    query with fewer than `window` tokens before it is dense causal attention (torch SDPA)."""
+    rng = np.random.default_rng(21)
+    B, Lq, Lk, H, d = 1, 3, 90, 2, 8
+    q, k, v = _rand_bf16(rng, (B, Lq, H, d)), _rand_bf16(rng, (B, Lk, d)), _rand_bf16(rng, (B, Lk, d))
+    idx = np.full((B, Lq, 40), -1, np.int32)
+    for i in range(Lq):
+        sel = rng.choice(Lk - Lq + i + 1, size=40, replace=False)
+        idx[0, i] = np.sort(sel)
+    one = oracle.sparse_attn_v1(q, k, v, idx, np.ones((B, Lq, H)), 0.3, window=128)["out"]
+    np.testing.assert_allclose(one, oracle.sparse_attn(q, k, v, idx, 0.3)["out"], rtol=0, atol=1e-13)
+    zero = oracle.sparse_attn_v1(q, k, v, idx, np.zeros((B, Lq, H)), 0.3, window=128)["out"]
+    np.testing.assert_allclose(zero, _torch_dense(q, k, v, 0.3).reshape(B * Lq, H, d), rtol=0, atol=1e-12)
+    half = oracle.sparse_attn_v1(q, k, v, idx, np.full((B, Lq, H), 0.25), 0.3, window=128)["out"]
+    np.testing.assert_allclose(half, 0.25 * one + 0.75 * zero, rtol=0, atol=1e-13)
