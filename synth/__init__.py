@@ -183,10 +183,16 @@ class SyntheticInputs:
         return f32_to_bf16_bits(self._k_f32)
 
     @cached_property
+    def _v_f32(self) -> np.ndarray:
+        # drawn once: a SeedSequence hands out new children on every spawn, so a second draw
+        # from the same stream would be a different sample
+        wl = self.wl
+        return _normal_f32(self._s[4], (wl.B, wl.Lk, wl.d))
+
+    @cached_property
     def v(self) -> np.ndarray:
         """[B, Lk, d] values (one KV head)."""
-        wl = self.wl
-        return f32_to_bf16_bits(_normal_f32(self._s[4], (wl.B, wl.Lk, wl.d)))
+        return f32_to_bf16_bits(self._v_f32)
 
     @cached_property
     def _k_f32(self) -> np.ndarray:
@@ -206,7 +212,7 @@ class SyntheticInputs:
     @cached_property
     def v8(self) -> tuple[np.ndarray, float]:
         """([B, Lk, d] e4m3 codes, power-of-two scale) of the same value samples as ``v``."""
-        v = _normal_f32(self._s[4], (self.wl.B, self.wl.Lk, self.wl.d))
+        v = self._v_f32
         sc = e4m3_scale(v)
         return f32_to_e4m3(v, sc), sc
 

@@ -391,3 +391,21 @@ def test_gated_window_fusion_reduces_to_its_branches():
     np.testing.assert_allclose(zero, _torch_dense(q, k, v, 0.3).reshape(B * Lq, H, d), rtol=0, atol=1e-12)
     half = oracle.sparse_attn_v1(q, k, v, idx, np.full((B, Lq, H), 0.25), 0.3, window=128)["out"]
     np.testing.assert_allclose(half, 0.25 * one + 0.75 * zero, rtol=0, atol=1e-13)
+
+
+def test_e4m3_cache_of_the_workload_is_the_bf16_cache_rounded():
+    """The input generator's e4m3 cache decodes to within one e4m3 rounding of the same samples'
+    bf16 cache (relative 2^-4 for normal values, half the subnormal step 2^-10 * scale below),
+    and is deterministic."""
+    g = synth.SyntheticInputs(synth.small("decode_32k", B=2, Lk=700))
+    (k8, ks), (v8, vs) = g.k8, g.v8
+    assert k8.dtype == np.uint8 and k8.shape == (2, 700, 128) and v8.shape == k8.shape
+    for codes, sc, bf in ((k8, ks, g.k), (v8, vs, g.v)):
+        deq = bf16_bits_to_f32(oracle.e4m3_to_bf16(codes, sc)).astype(np.float64)
+        ref = bf16_bits_to_f32(bf).astype(np.float64)
+        err = np.abs(deq - ref)
+        # bf16 itself is within 2^-9 of the float32 sample; e4m3 within 2^-4 (or the subnormal step)
+        assert np.all(err <= np.maximum(np.abs(ref) * (2.0 ** -4 + 2.0 ** -8), 2.0 ** -10 * sc + 1e-12))
+        assert np.abs(deq).max() <= 448 * sc
+    g2 = synth.SyntheticInputs(synth.small("decode_32k", B=2, Lk=700))
+    assert np.array_equal(g2.k8[0], k8) and g2.k8[1] == ks
