@@ -52,7 +52,9 @@ def _load():
             lib.oracle_full_attn_select.argtypes = [P, P, P, i, i, i, i, i, d, i, i, P, i64, P, P, P, P, i]
             lib.oracle_sparse_attn.argtypes = [P, P, P, P, i, i, i, i, i, i, d, P, i64, P, P, i]
             lib.oracle_bridge_kv_proj.argtypes = [P, i, i, P, i, i, P, i64, P, i]
-            for f in (lib.oracle_full_attn_select, lib.oracle_sparse_attn, lib.oracle_bridge_kv_proj):
+            lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, i, i, i, i, i, i, d, P, i64, P, P, P, i]
+            for f in (lib.oracle_full_attn_select, lib.oracle_sparse_attn, lib.oracle_bridge_kv_proj,
+                      lib.oracle_attn_bwd):
                 f.restype = ctypes.c_int
             lib.oracle_default_threads.restype = ctypes.c_int
             _lib = lib
@@ -157,6 +159,14 @@ def sparse_attn(q, k, v, idx, scale, rows=None, threads=0):
     return {"out": out, "lse": lse}
 
 
+def block_scores(score_row, t, block=64):
+    """Score of every block meeting 0..t: the sum of its tokens' scores at or before t (the
+    reading of the HySparse block score stated in block_select)."""
+    score_row = np.asarray(score_row, dtype=np.float64)
+    nb = t // block + 1
+    return np.array([score_row[j * block:min((j + 1) * block, t + 1)].sum() for j in range(nb)])
+
+
 def block_select(score_row, t, block=64, n_blocks=16):
     """The HySparse (v1) selection of one query at position t: the n_blocks blocks of `block`
     consecutive tokens with the largest block score, ties to the lower block; returns the chosen
@@ -170,11 +180,10 @@ def block_select(score_row, t, block=64, n_blocks=16):
     or before t is a candidate (the window branch is separate, so recent blocks compete too).
     score_row: [>= t + 1] float64 token scores.
     """
-    score_row = np.asarray(score_row, dtype=np.float64)
     nb = t // block + 1                       # blocks meeting 0..t
     if nb <= n_blocks:
         return np.arange(t + 1, dtype=np.int64)
-    bs = np.array([score_row[j * block:min((j + 1) * block, t + 1)].sum() for j in range(nb)])
+    bs = block_scores(score_row, t, block)
     order = sorted(range(nb), key=lambda j: (-bs[j], j))
     chosen = sorted(order[:n_blocks])
     return np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in chosen]).astype(np.int64)
@@ -198,6 +207,35 @@ def sparse_attn_v1(q, k, v, block_idx, gate, scale, window=128, threads=0):
     ob = sparse_attn(q, k, v, block_idx, scale, threads=threads)["out"]
     ow = sparse_attn(q, k, v, win, scale, threads=threads)["out"]
     return {"out": gate[:, :, None] * ob + (1.0 - gate[:, :, None]) * ow}
+
+
+def attn_bwd(q, k, v, do, scale, idx=None, rows=None, want_kv=True, threads=0):
+    """Gradients of causal MQA attention (idx None: query i at t = Lk - Lq + i reads keys 0..t)
+    or of sparse attention over idx [B,Lq,S] (-1 = empty), for the output gradient do
+    [B,Lq,H,d] (bf16 bits like q). Returns dict(dq [n,H,d] f64 for `rows` (default all),
+    dk, dv [B,Lk,d] f64 when want_kv (then rows must be None))."""
+    q, k, v, do = _u16(q), _u16(k), _u16(v), _u16(do)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    assert do.shape == q.shape and k.shape == (B, Lk, d) and v.shape == k.shape
+    if want_kv and rows is not None:
+        raise ValueError("dk, dv need every row")
+    S = 0
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        assert idx.shape[:2] == (B, Lq)
+        S = idx.shape[2]
+    r, n = _rows(rows, B * Lq)
+    dq = np.empty((n, H, d), np.float64)
+    dk = np.empty((B, Lk, d), np.float64) if want_kv else None
+    dv = np.empty((B, Lk, d), np.float64) if want_kv else None
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(idx), B, Lq, Lk, H, d, S, float(scale),
+                                 _ptr(r), n, _ptr(dq), _ptr(dk), _ptr(dv), threads)
+    _check(rc, "attn_bwd")
+    res = {"dq": dq}
+    if want_kv:
+        res["dk"], res["dv"] = dk, dv
+    return res
 
 
 def bridge_kv_proj(h, w, rows=None, threads=0):

@@ -26,6 +26,12 @@
  *    内层 KV Reuse"; toolnavs.com, section "Was HySparse2 tut"); it is plain softmax
  *    attention restricted to the selected tokens (the separate SWA branch and its gate
  *    are removed, same sections).
+ *  - attn_bwd: the gradients of the full layer's and the sparse layers' attention (the full
+ *    layers are trained natively as indexers, arex-research.com, section "外层 KV Bridging，
+ *    内层 KV Reuse"), i.e. of out = softmax(scale q K_set^T) V_set with respect to Q, K and V for
+ *    a given output gradient dO, the key set of a row being its causal row (full layer) or its
+ *    selected slots (sparse layer; the selection is a constant: it has no gradient). K and V
+ *    gradients sum over every head and every row that reads the key.
  *  - bridge_kv_proj: KV Bridging; each cross-decoder full-attention layer l forms its own
  *    K_l = H W_k^l and V_l = H W_v^l from one shared self-decoder hidden state H
  *    (arex-research.com, section "外层 KV Bridging，内层 KV Reuse"; toolnavs.com,
@@ -398,6 +404,219 @@ int oracle_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, 
   free(all);
   if (rc != ORC_OK) return rc;
   return atomic_load(&c.bad);
+}
+
+/* ------------------------------------------------------------------ attention backward */
+/*
+ * For one row (query i of sequence b at t = Lk - Lq + i) and head h, with key set J (the
+ * causal row 0..t, or the row's selected slots):
+ *   s_j = scale <q, k_j>, p_j = exp(s_j - lse), lse = log sum_j exp(s_j)   (the forward)
+ *   dP_j = <dO, v_j>,  D = sum_j p_j dP_j,  dS_j = p_j (dP_j - D)
+ *   dQ   = scale sum_j dS_j k_j
+ *   dK_j += scale dS_j q        dV_j += p_j dO     (summed over every (row, head) reading j)
+ */
+typedef struct {
+  const uint16_t *Q, *K, *V, *dO;
+  const int32_t* idx; /* [B, Lq, S] or NULL (causal rows) */
+  int B, Lq, Lk, H, d, S;
+  double scale;
+  const int64_t* rows;
+  int64_t n_rows;
+  double* dQ;    /* [n_rows, H, d] */
+  double* lse;   /* [B * Lq, H] (pass 2: every row) */
+  double* D;     /* [B * Lq, H] */
+  double *dK, *dV;   /* [B, Lk, d] */
+  const int64_t* inv_start; /* [B * Lk + 1] rows reading key (b, j): inv_rows[inv_start[.]..] */
+  const int64_t* inv_rows;
+  atomic_int bad;
+} bwd_ctx;
+
+/* the key of slot n of row `flat` (or -1), causal rows: slot n is key n for n <= t */
+static int bwd_key(const bwd_ctx* c, int64_t flat, int n) {
+  if (!c->idx) {
+    const int t = c->Lk - c->Lq + (int)(flat % c->Lq);
+    return n <= t ? n : -1;
+  }
+  return c->idx[flat * c->S + n];
+}
+
+/* task (row, head): lse, D and dQ of one head of one row; s[] holds the slots' logits */
+static void bwd_task_row(void* vctx, int64_t task, double* s) {
+  bwd_ctx* c = (bwd_ctx*)vctx;
+  const int64_t r = task / c->H;
+  const int h = (int)(task % c->H);
+  const int64_t flat = c->rows[r];
+  const int b = (int)(flat / c->Lq);
+  const int n_slots = c->idx ? c->S : c->Lk;
+  const uint16_t* q = c->Q + (flat * c->H + h) * c->d;
+  const uint16_t* g = c->dO + (flat * c->H + h) * c->d;
+  double m = -INFINITY;
+  int n_valid = 0;
+  for (int n = 0; n < n_slots; ++n) {
+    const int j = bwd_key(c, flat, n);
+    if (j == -1) continue;
+    if (j < 0 || j >= c->Lk) {
+      atomic_store(&c->bad, ORC_EINDEX);
+      return;
+    }
+    const uint16_t* k = c->K + ((int64_t)b * c->Lk + j) * c->d;
+    double acc = 0.0;
+    for (int x = 0; x < c->d; ++x) acc += widen(q[x]) * widen(k[x]);
+    s[n] = c->scale * acc;
+    if (s[n] > m) m = s[n];
+    n_valid++;
+  }
+  if (n_valid == 0) {
+    atomic_store(&c->bad, ORC_EINDEX);
+    return;
+  }
+  double sum = 0.0;
+  for (int n = 0; n < n_slots; ++n)
+    if (bwd_key(c, flat, n) != -1) sum += exp(s[n] - m);
+  const double lse = m + log(sum);
+  /* dP_j and D = sum_j p_j dP_j */
+  double D = 0.0;
+  for (int n = 0; n < n_slots; ++n) {
+    const int j = bwd_key(c, flat, n);
+    if (j == -1) continue;
+    const uint16_t* v = c->V + ((int64_t)b * c->Lk + j) * c->d;
+    double dp = 0.0;
+    for (int x = 0; x < c->d; ++x) dp += widen(g[x]) * widen(v[x]);
+    D += exp(s[n] - lse) * dp;
+  }
+  c->lse[flat * c->H + h] = lse;
+  c->D[flat * c->H + h] = D;
+  if (!c->dQ) return;
+  double* dq = c->dQ + (r * c->H + h) * c->d;
+  for (int x = 0; x < c->d; ++x) dq[x] = 0.0;
+  for (int n = 0; n < n_slots; ++n) {
+    const int j = bwd_key(c, flat, n);
+    if (j == -1) continue;
+    const uint16_t* k = c->K + ((int64_t)b * c->Lk + j) * c->d;
+    const uint16_t* v = c->V + ((int64_t)b * c->Lk + j) * c->d;
+    double dp = 0.0;
+    for (int x = 0; x < c->d; ++x) dp += widen(g[x]) * widen(v[x]);
+    const double ds = exp(s[n] - lse) * (dp - D);
+    for (int x = 0; x < c->d; ++x) dq[x] += c->scale * ds * widen(k[x]);
+  }
+}
+
+/* task (sequence, key): dK and dV of one key, from every (row, head) whose set reads it */
+static void bwd_task_key(void* vctx, int64_t task, double* unused) {
+  (void)unused;
+  bwd_ctx* c = (bwd_ctx*)vctx;
+  const int b = (int)(task / c->Lk);
+  const int j = (int)(task % c->Lk);
+  const uint16_t* k = c->K + ((int64_t)b * c->Lk + j) * c->d;
+  const uint16_t* v = c->V + ((int64_t)b * c->Lk + j) * c->d;
+  double* dk = c->dK + ((int64_t)b * c->Lk + j) * c->d;
+  double* dv = c->dV + ((int64_t)b * c->Lk + j) * c->d;
+  for (int x = 0; x < c->d; ++x) dk[x] = dv[x] = 0.0;
+  int64_t r0, r1;
+  if (c->idx) {
+    r0 = c->inv_start[task];
+    r1 = c->inv_start[task + 1];
+  } else {  /* causal: rows i with t = Lk - Lq + i >= j */
+    const int64_t i0 = (int64_t)j - (c->Lk - c->Lq);
+    r0 = i0 > 0 ? i0 : 0;
+    r1 = c->Lq;
+  }
+  for (int64_t e = r0; e < r1; ++e) {
+    const int64_t flat = c->idx ? c->inv_rows[e] : (int64_t)b * c->Lq + e;
+    for (int h = 0; h < c->H; ++h) {
+      const uint16_t* q = c->Q + (flat * c->H + h) * c->d;
+      const uint16_t* g = c->dO + (flat * c->H + h) * c->d;
+      double acc = 0.0, dp = 0.0;
+      for (int x = 0; x < c->d; ++x) {
+        acc += widen(q[x]) * widen(k[x]);
+        dp += widen(g[x]) * widen(v[x]);
+      }
+      const double p = exp(c->scale * acc - c->lse[flat * c->H + h]);
+      const double ds = p * (dp - c->D[flat * c->H + h]);
+      for (int x = 0; x < c->d; ++x) {
+        dk[x] += c->scale * ds * widen(q[x]);
+        dv[x] += p * widen(g[x]);
+      }
+    }
+  }
+}
+
+/*
+ * Gradients of attention over per-row key sets. Q, dO: [B, Lq, H, d]; K, V: [B, Lk, d] (bf16
+ * bits); idx: [B, Lq, S] selected slots (-1 = empty), or NULL for the causal rows (query i at
+ * t = Lk - Lq + i reads keys 0..t). dQ: [n_rows, H, d] for the rows `rows` (NULL: every row; dQ
+ * may be NULL). dK, dV: [B, Lk, d] (both or neither; they need every row, so rows must then be
+ * NULL). Returns ORC_EINDEX for an index outside [0, Lk) or a row without a valid key.
+ */
+int oracle_attn_bwd(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* dO, const int32_t* idx,
+                    int B, int Lq, int Lk, int H, int d, int S, double scale, const int64_t* rows, int64_t n_rows,
+                    double* dQ, double* dK, double* dV, int n_threads) {
+  if (!Q || !K || !V || !dO || (!dK) != (!dV)) return ORC_EINVAL;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || H <= 0 || d <= 0 || (idx && S <= 0)) return ORC_EINVAL;
+  if (dK && rows) return ORC_EINVAL;
+  const int64_t all_rows = (int64_t)B * Lq;
+  int64_t* all = NULL;
+  if (!rows) {
+    n_rows = all_rows;
+    all = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_rows);
+    if (!all) return ORC_ENOMEM;
+    for (int64_t r = 0; r < n_rows; ++r) all[r] = r;
+    rows = all;
+  }
+  for (int64_t r = 0; r < n_rows; ++r)
+    if (rows[r] < 0 || rows[r] >= all_rows) {
+      free(all);
+      return ORC_EINVAL;
+    }
+  double* lse = (double*)malloc(sizeof(double) * (size_t)all_rows * H);
+  double* Dv = (double*)malloc(sizeof(double) * (size_t)all_rows * H);
+  int64_t* inv_start = NULL;
+  int64_t* inv_rows = NULL;
+  int rc = (lse && Dv) ? ORC_OK : ORC_ENOMEM;
+  if (rc == ORC_OK && dK && idx) {
+    /* rows reading each key (b, j), one entry per slot, rows ascending */
+    inv_start = (int64_t*)calloc((size_t)B * Lk + 1, sizeof(int64_t));
+    if (!inv_start) rc = ORC_ENOMEM;
+    for (int64_t f = 0; rc == ORC_OK && f < all_rows; ++f)
+      for (int n = 0; n < S; ++n) {
+        const int32_t j = idx[f * S + n];
+        if (j == -1) continue;
+        if (j < 0 || j >= Lk) { rc = ORC_EINDEX; break; }
+        inv_start[(f / Lq) * Lk + j + 1]++;
+      }
+    if (rc == ORC_OK) {
+      for (int64_t e = 0; e < (int64_t)B * Lk; ++e) inv_start[e + 1] += inv_start[e];
+      inv_rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)(inv_start[(int64_t)B * Lk] + 1));
+      int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * (size_t)B * Lk);
+      if (!inv_rows || !fill) rc = ORC_ENOMEM;
+      else {
+        memcpy(fill, inv_start, sizeof(int64_t) * (size_t)B * Lk);
+        for (int64_t f = 0; f < all_rows; ++f)
+          for (int n = 0; n < S; ++n) {
+            const int32_t j = idx[f * S + n];
+            if (j != -1) inv_rows[fill[(f / Lq) * Lk + j]++] = f;
+          }
+      }
+      free(fill);
+    }
+  }
+  bwd_ctx c;
+  c.Q = Q; c.K = K; c.V = V; c.dO = dO; c.idx = idx;
+  c.B = B; c.Lq = Lq; c.Lk = Lk; c.H = H; c.d = d; c.S = S;
+  c.scale = scale;
+  c.rows = rows; c.n_rows = n_rows;
+  c.dQ = dQ; c.lse = lse; c.D = Dv; c.dK = dK; c.dV = dV;
+  c.inv_start = inv_start; c.inv_rows = inv_rows;
+  atomic_init(&c.bad, 0);
+  if (rc == ORC_OK) rc = run_tasks(bwd_task_row, &c, n_rows * H, (size_t)(idx ? S : Lk), n_threads);
+  if (rc == ORC_OK) rc = atomic_load(&c.bad);
+  if (rc == ORC_OK && dK) rc = run_tasks(bwd_task_key, &c, (int64_t)B * Lk, 0, n_threads);
+  free(inv_rows);
+  free(inv_start);
+  free(Dv);
+  free(lse);
+  free(all);
+  return rc;
 }
 
 /* ------------------------------------------------------------------ KV Bridging projection */

@@ -21,6 +21,9 @@ positions per sequence (drawn without replacement) and to every query vector (al
 all layers), so that the top-k selection is not trivial. V is not planted. The bridge
 hidden state is N(0, 1) and the projection weights are N(0, 0.02^2).
 
+Backward pass: the upstream gradient of each layer's output is N(0, 1), rounded to bf16
+(``grad_out``).
+
 FP8 cache: the same float32 K and V samples stored as OCP e4m3 codes (1 sign, 4 exponent bits
 with bias 7, 3 mantissa bits, subnormals, no infinities) times one power-of-two scale per
 tensor, the smallest for which the largest magnitude fits under 448; each value rounds to the
@@ -29,7 +32,9 @@ nearest code, ties to the even code.
 from __future__ import annotations
 
 import math
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 from functools import cached_property
 
@@ -78,12 +83,28 @@ WORKLOADS = {
 }
 
 
+def _threads() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 to bf16 (nearest, ties to even); returns the uint16 bit patterns."""
+    """Round float32 to bf16 (nearest, ties to even); returns the uint16 bit patterns.
+    Large arrays are converted in chunks on several threads (element-wise: same result)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32)
-    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
-    return r.astype(np.uint16)
+    flat = x.reshape(-1)
+    out = np.empty(flat.shape, np.uint16)
+
+    def conv(lo, hi):
+        u = flat[lo:hi].view(np.uint32)
+        out[lo:hi] = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+
+    n = flat.size
+    if n <= _CHUNK:
+        conv(0, n)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(lambda c: conv(c, min(n, c + _CHUNK)), range(0, n, _CHUNK)))
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -135,9 +156,16 @@ def _normal_f32(seq: np.random.SeedSequence, shape) -> np.ndarray:
     out = np.empty(n, dtype=np.float32)
     n_chunks = max(1, (n + _CHUNK - 1) // _CHUNK)
     kids = seq.spawn(n_chunks)
-    for c in range(n_chunks):
+
+    def fill(c):  # each chunk from its own stream: the result does not depend on the threads
         lo, hi = c * _CHUNK, min(n, (c + 1) * _CHUNK)
         np.random.Generator(np.random.PCG64(kids[c])).standard_normal(hi - lo, dtype=np.float32, out=out[lo:hi])
+
+    if n_chunks == 1:
+        fill(0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(fill, range(n_chunks)))
     return out.reshape(shape)
 
 
@@ -222,6 +250,21 @@ class SyntheticInputs:
         key = f"_qs{layer}"
         if key not in self.__dict__:
             self.__dict__[key] = self._query(8 + layer)
+        return self.__dict__[key]
+
+    def grad_out(self, layer: int) -> np.ndarray:
+        """[B, Lq, H, d] upstream gradient dL/d(out) of layer `layer` of the hybrid block (0: the
+        full layer, 1..n_sparse: the sparse layers), N(0, 1) rounded to bf16, for the backward
+        pass. Each layer draws from its own child of stream 7, derived by its spawn key so that
+        the draw does not depend on the order of the calls."""
+        assert 0 <= layer <= self.wl.n_sparse
+        key = f"_go{layer}"
+        if key not in self.__dict__:
+            parent = self._s[7]
+            child = np.random.SeedSequence(parent.entropy, spawn_key=tuple(parent.spawn_key) + (layer,),
+                                           pool_size=parent.pool_size)
+            wl = self.wl
+            self.__dict__[key] = f32_to_bf16_bits(_normal_f32(child, (wl.B, wl.Lq, wl.H, wl.d)))
         return self.__dict__[key]
 
     @cached_property

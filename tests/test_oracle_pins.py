@@ -409,3 +409,117 @@ def test_e4m3_cache_of_the_workload_is_the_bf16_cache_rounded():
         assert np.abs(deq).max() <= 448 * sc
     g2 = synth.SyntheticInputs(synth.small("decode_32k", B=2, Lk=700))
     assert np.array_equal(g2.k8[0], k8) and g2.k8[1] == ks
+
+
+# ---------------------------------------------------------------------------------------------
+# Attention backward (gradients of the full and sparse layers)
+# ---------------------------------------------------------------------------------------------
+def _torch_grads(q, k, v, do, scale, mask):
+    """Gradients of torch SDPA (fp64) with K, V shared by every head (expanded, so autograd sums
+    their gradients over the heads): q/do [B,Lq,H,d], k/v [B,Lk,d], mask [B or 1, Lq, Lk] bool."""
+    Q = _t64(q).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    K = _t64(k).clone().requires_grad_(True)
+    V = _t64(v).clone().requires_grad_(True)
+    H = q.shape[2]
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K[:, None].expand(-1, H, -1, -1),
+                                                         V[:, None].expand(-1, H, -1, -1),
+                                                         attn_mask=mask[:, None], scale=scale)
+    o.backward(_t64(do).permute(0, 2, 1, 3))
+    return Q.grad.permute(0, 2, 1, 3).numpy(), K.grad.numpy(), V.grad.numpy()
+
+
+@pytest.mark.parametrize("B,Lq,Lk,H,d", [(2, 13, 13, 3, 8), (1, 4, 19, 2, 16), (2, 1, 23, 4, 8)])
+def test_attention_backward_matches_torch_autograd(B, Lq, Lk, H, d):
+    rng = np.random.default_rng(40 + Lk)
+    q, k, v, do = (_rand_bf16(rng, (B, Lq, H, d)), _rand_bf16(rng, (B, Lk, d)), _rand_bf16(rng, (B, Lk, d)),
+                   _rand_bf16(rng, (B, Lq, H, d)))
+    scale = 1.0 / math.sqrt(d)
+    r = oracle.attn_bwd(q, k, v, do, scale)
+    dq, dk, dv = _torch_grads(q, k, v, do, scale, _causal_mask(Lq, Lk)[None])
+    np.testing.assert_allclose(r["dq"], dq.reshape(B * Lq, H, d), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(r["dk"], dk, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(r["dv"], dv, rtol=0, atol=1e-11)
+    # sampled rows give the same dQ rows
+    rows = [0, B * Lq - 1]
+    rs = oracle.attn_bwd(q, k, v, do, scale, rows=rows, want_kv=False)
+    np.testing.assert_allclose(rs["dq"], r["dq"][rows], rtol=0, atol=0)
+
+
+def test_sparse_attention_backward_matches_torch_autograd():
+    """Sparse rows (random index sets, -1 padded) against autograd of SDPA with the same index
+    mask; a repeated slot counts twice in the oracle, so the sets here are duplicate-free."""
+    rng = np.random.default_rng(44)
+    B, Lq, Lk, H, d, S = 2, 5, 30, 3, 8, 12
+    q, k, v, do = (_rand_bf16(rng, (B, Lq, H, d)), _rand_bf16(rng, (B, Lk, d)), _rand_bf16(rng, (B, Lk, d)),
+                   _rand_bf16(rng, (B, Lq, H, d)))
+    idx = np.full((B, Lq, S), -1, np.int32)
+    mask = torch.zeros((B, Lq, Lk), dtype=torch.bool)
+    for b in range(B):
+        for i in range(Lq):
+            n = int(rng.integers(1, S + 1))
+            sel = np.sort(rng.choice(Lk, size=n, replace=False))
+            idx[b, i, :n] = sel
+            mask[b, i, torch.from_numpy(sel.astype(np.int64))] = True
+    r = oracle.attn_bwd(q, k, v, do, 0.4, idx=idx)
+    dq, dk, dv = _torch_grads(q, k, v, do, 0.4, mask)
+    np.testing.assert_allclose(r["dq"], dq.reshape(B * Lq, H, d), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(r["dk"], dk, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(r["dv"], dv, rtol=0, atol=1e-11)
+
+
+def test_attention_backward_is_the_derivative_of_the_forward():
+    """Central differences of the oracle's own forward, loss = sum(dO * out), against the
+    backward, for a few coordinates of Q, K and V (inputs perturbed in float64 through a
+    value that bf16 represents exactly: the forward only reads bf16, so the step is 2^-4 of a
+    coordinate that is a power of two)."""
+    rng = np.random.default_rng(45)
+    B, L, H, d = 1, 6, 2, 4
+    q, k, v, do = (_rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d)), _rand_bf16(rng, (B, L, d)),
+                   _rand_bf16(rng, (B, L, H, d)))
+    scale = 0.5
+    g = oracle.attn_bwd(q, k, v, do, scale)
+    dof = bf16_bits_to_f32(do).astype(np.float64)
+
+    def loss(qq, kk, vv):
+        return float((oracle.full_attn_select(qq, kk, vv, scale, 1, 0)["out"] * dof.reshape(B * L, H, d)).sum())
+
+    def setv(bits, pos, val):
+        out = bits.copy()
+        out[pos] = f32_to_bf16_bits(np.array([val], np.float32))[0]
+        return out
+
+    # the grid of exactly representable values around 1.0 with step 2^-7 is fine in bf16:
+    # differences of +-2^-7 around a coordinate set to 1.0
+    h = 2.0 ** -7
+    for name, arr, pos, grad in (("q", q, (0, 3, 1, 2), g["dq"][3, 1, 2]), ("k", k, (0, 2, 1), g["dk"][0, 2, 1]),
+                                 ("v", v, (0, 4, 3), g["dv"][0, 4, 3])):
+        base = setv(arr, pos, 1.0)
+        up, dn = setv(arr, pos, 1.0 + h), setv(arr, pos, 1.0 - h)
+        args = {"q": q, "k": k, "v": v}
+        args[name] = up
+        lu = loss(args["q"], args["k"], args["v"])
+        args[name] = dn
+        ld = loss(args["q"], args["k"], args["v"])
+        args[name] = base
+        gb = oracle.attn_bwd(args["q"], args["k"], args["v"], do, scale)
+        gval = {"q": gb["dq"][pos[1], pos[2], pos[3]] if name == "q" else None,
+                "k": gb["dk"][pos] if name == "k" else None, "v": gb["dv"][pos] if name == "v" else None}[name]
+        fd = (lu - ld) / (2 * h)
+        assert abs(fd - gval) <= 1e-3 * max(1.0, abs(gval)), (name, fd, gval)
+
+
+def test_attention_backward_identities():
+    """Every row's dS sums to zero, so sum_j dK_j = 0; every row's p sums to one, so
+    sum_j dV_j = sum of dO over rows and heads; K = 0 gives dQ = 0; the first row (one key)
+    has dS = 0."""
+    rng = np.random.default_rng(46)
+    B, L, H, d = 2, 15, 3, 8
+    q, k, v, do = (_rand_bf16(rng, (B, L, H, d)), _rand_bf16(rng, (B, L, d)), _rand_bf16(rng, (B, L, d)),
+                   _rand_bf16(rng, (B, L, H, d)))
+    r = oracle.attn_bwd(q, k, v, do, 0.35)
+    np.testing.assert_allclose(r["dk"].sum(axis=1), 0.0, atol=1e-11)
+    dof = bf16_bits_to_f32(do).astype(np.float64)
+    np.testing.assert_allclose(r["dv"].sum(axis=1), dof.sum(axis=(1, 2)), atol=1e-11)
+    np.testing.assert_allclose(r["dq"].reshape(B, L, H, d)[:, 0], 0.0, atol=1e-14)
+    z = oracle.attn_bwd(q, np.zeros_like(k), v, do, 0.35)
+    np.testing.assert_allclose(z["dq"], 0.0, atol=1e-14)
