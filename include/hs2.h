@@ -233,13 +233,21 @@ HS2_API hs2_status hs2_sparse_attn_fp8kv(const hs2_bf16* Q, const uint8_t* K8, c
  * more scratch than that (hs2_sparse_attn_workspace_bytes(...) > 4 KiB; with the current
  * kernels every supported shape needs only its 256-byte status word). The first call on
  * each device performs a one-time set-up (it looks up the array's device address) and should
- * come before any stream capture. All calls share the array: calls whose GPU work overlaps
- * (e.g. on different streams) race. The device status word of these calls is internal.
+ * come before any stream capture; the address is cached per device with the device's context,
+ * and looked up again when a call finds another context (after cudaDeviceReset). All calls
+ * share the array: calls whose GPU work overlaps (e.g. on different streams) race. Each call
+ * clears the status word in the array before its kernels run.
  * No cudaMalloc / cudaFree is ever called.
  */
 HS2_API hs2_status hs2_sparse_attn_noalloc(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
                                            const int32_t* idx, int B, int Lq, int Lk, int H, int d, int S,
                                            float scale, hs2_bf16* out, float* lse, hs2_stream stream);
+/* Device status of the latest hs2_sparse_attn_noalloc call on the current device: waits for
+ * `stream` (the stream of that call) and returns HS2_OK, HS2_ERR_DEVICE_BOUNDS (an idx entry
+ * outside [0, Lk): it was skipped, so that row's output is unspecified) or
+ * HS2_ERR_DEVICE_TIMEOUT (a bounded wait gave up), as hs2_read_device_status does for a
+ * workspace; HS2_ERR_WORKSPACE if no call has set up this device yet. */
+HS2_API hs2_status hs2_sparse_attn_noalloc_status(hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * KV Bridging projection

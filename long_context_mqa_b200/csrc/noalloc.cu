@@ -12,10 +12,15 @@
 // memory), so every supported shape fits; larger needs are still rejected, not overrun. Host code
 // cannot use the array's name as a device address (it is a host-side stand-in), so the first
 // call on each device looks the address up with cudaGetSymbolAddress while that device is
-// current, and caches it per device. That first call on a device should therefore happen before
-// any stream capture. All calls share the one array and it keeps what the last call left there:
-// each call clears the status word it needs at zero. Calls whose GPU work overlaps (for example on two streams) race on the
-// array. Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
+// current, and caches it per device together with the device's current context; a call that
+// finds another context (the old one was destroyed, e.g. by cudaDeviceReset) looks it up again.
+// That first call on a device should therefore happen before any stream capture. All calls share
+// the one array and it keeps what the last call left there: each call clears the status word it
+// needs at zero, and hs2_sparse_attn_noalloc_status reads what the last call recorded there.
+// Calls whose GPU work overlaps (for example on two streams) race on the array. Nothing here calls
+// cudaMalloc, cudaFree or an allocating library routine.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/hs2.h"
@@ -29,16 +34,37 @@ __device__ __align__(256) unsigned char g_sparse_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of g_sparse_scratch on the current device (set up once per device).
-hs2_status scratch_for_current_device(void** out) {
+// cuCtxGetCurrent through the runtime's driver entry point (the library does not link libcuda).
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<Fn>(nullptr);
+    return reinterpret_cast<Fn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_sparse_scratch on the current device: looked up once per device (again
+// only if the device's context has changed since). `setup` false: report HS2_ERR_WORKSPACE
+// instead of looking it up (nothing has run there yet).
+hs2_status scratch_for_current_device(void** out, bool setup = true) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HS2_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
+  if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != current_context()) {
+    if (!setup) return HS2_ERR_WORKSPACE;
+    void* p = nullptr;  // the lookup also makes the device's primary context current
     if (cudaGetSymbolAddress(&p, g_sparse_scratch) != cudaSuccess || p == nullptr) return HS2_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_ptr[dev];
   return HS2_OK;
@@ -59,4 +85,11 @@ extern "C" hs2_status hs2_sparse_attn_noalloc(const hs2_bf16* Q, const hs2_bf16*
   // the status word at the start of the scratch must start at zero for this call
   if (cudaMemsetAsync(scratch, 0, 16, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HS2_ERR_CUDA;
   return hs2_sparse_attn(Q, K, V, idx, B, Lq, Lk, H, d, S, scale, out, lse, scratch, kScratchBytes, stream);
+}
+
+extern "C" hs2_status hs2_sparse_attn_noalloc_status(hs2_stream stream) {
+  void* scratch = nullptr;
+  const hs2_status st = scratch_for_current_device(&scratch, false);
+  if (st != HS2_OK) return st;
+  return hs2_read_device_status(scratch, stream);
 }
