@@ -340,6 +340,10 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 (e4m3) K/V cache decode clause")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the decode_32k, decode_1m and tiny_prefill clauses")
+    ap.add_argument("--no-v1", action="store_true", help="skip the HySparse (v1) block-level decode clause")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="time only the FP8-cache decode step (--steps/--warmup; small profiling cases with --batch)")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training-shape backward clause")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph of the steps")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (small profiling cases)")
     ap.add_argument("--cache", type=int, default=0, help="override cache length (small profiling cases)")
@@ -353,7 +357,29 @@ def main():
         return run_reference(args)
     if args.prefill_only:
         return run_prefill_only(args)
+    if args.fp8_only:
+        return run_fp8_only(args)
     return run_gpu(args)
+
+
+def run_fp8_only(args):
+    """The FP8-cache decode step alone on the decode workload (or a reduced --batch/--cache case);
+    one JSON line."""
+    import torch
+    import long_context_mqa_b200 as hs2
+    world, rank, local = _dist_init()
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[WORKLOAD]
+    if args.batch or args.cache:
+        wl = wl.with_(name=f"{WORKLOAD}_b{args.batch or wl.B}_n{args.cache or wl.Lk}", B=args.batch or wl.B,
+                      Lk=args.cache or wl.Lk)
+    g = synth.SyntheticInputs(wl, seed=args.seed + rank)
+    q, k, v = _bf16(g.q, dev), _bf16(g.k, dev), _bf16(g.v, dev)
+    qs = [_bf16(g.q_sparse(i), dev) for i in range(wl.n_sparse)]
+    res = bench_fp8(args, world, wl, hs2, q, k, v, qs, _peaks(), steps=max(1, args.steps), warmup=args.warmup)
+    if rank == 0:
+        print(json.dumps({"fp8_kv": res}), flush=True)
+    return 0
 
 
 def run_prefill_only(args):
@@ -559,10 +585,20 @@ def run_gpu(args):
     if not args.no_fp8:
         fp8 = bench_fp8(args, world, wl, hs2, q, k, v, qs, peaks)
 
+    # ---------------- the HySparse (v1) block-level step at the same budget
+    v1 = None
+    if not args.no_v1:
+        v1 = bench_v1(args, world, wl, hs2, q, k, v, qs, peaks, value)
+
     # ---------------- prefill (secondary clause of the metric)
     prefill = None
     if not args.no_prefill:
         prefill = bench_prefill(args, world, dev, peaks)
+
+    # ---------------- backward of a hybrid block at the training shape
+    backward = None
+    if not args.no_backward:
+        backward = bench_backward(args, world, dev, peaks)
 
     # ---------------- the other configurations of the method's synthetic workloads
     configs = None
@@ -597,7 +633,7 @@ def run_gpu(args):
                     "steps": e2e_steps, "note": "public Python API; per step one H2D copy of the five layers' queries from pinned memory, the new token's K/V rows, one D2H copy of the outputs and indices, a stream synchronize"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
             "device_status": [status, status_sp], "cpu_baseline": cpu, "selection_check": sel,
-            "ragged": ragged, "fp8_kv": fp8, "prefill": prefill, "configs": configs,
+            "ragged": ragged, "fp8_kv": fp8, "v1": v1, "prefill": prefill, "backward": backward, "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -800,6 +836,156 @@ def bench_tiny(args, world, rank, dev, peaks, reps=50):
         from parity import check_selection
         st = check_selection(idx.reshape(L, S).cpu().numpy(), r["idx"], r["score"], np.arange(L), wl.window, wl.topk)
         res["selection_check"] = {"rows": st.rows, "swaps": st.swaps, "max_swap_rel": st.max_swap_rel, "ok": st.ok()}
+    return res
+
+
+def bench_v1(args, world, wl, hs2, q, k, v, qs, peaks, token_value, steps=200, warmup=5):
+    """The HySparse (v1) decode step on the headline inputs, at the same budget as the token-level
+    step (1,024 tokens by score + the 128-token window): hs2_full_attn_select_v1 (16 blocks of 64
+    tokens), then the sparse layers as hs2_sparse_attn_v1 (block branch + window branch, mixed by
+    a seeded gate in [0, 1] per (sequence, head)), one CUDA graph; device-timed like the main line."""
+    import torch
+    S = 16 * 64 + wl.window
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, 1, wl.H), dtype=torch.float32, device=q.device)
+    idx = torch.empty((wl.B, 1, S), dtype=torch.int32, device=q.device)
+    outs = [torch.empty_like(q) for _ in range(wl.n_sparse)]
+    rng = np.random.default_rng(7)
+    gates = [torch.from_numpy(rng.uniform(0.0, 1.0, size=(wl.B, 1, wl.H)).astype(np.float32)).to(q.device)
+             for _ in range(wl.n_sparse)]
+    ws = torch.zeros(hs2.full_attn_select_v1_workspace_bytes(wl.B, wl.Lk, wl.H, wl.d), dtype=torch.uint8,
+                     device=q.device)
+    ws_sp = [torch.zeros(hs2.sparse_attn_workspace_bytes(wl.B, 1, wl.Lk, wl.H, wl.d, S), dtype=torch.uint8,
+                         device=q.device) for _ in range(wl.n_sparse)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hs2.full_attn_select_v1(q, k, v, scale=wl.scale, out=out, lse=lse, idx=idx, workspace=ws)
+        for i in range(wl.n_sparse):
+            hs2.sparse_attn_v1(qs[i], k, v, idx, gates[i], scale=wl.scale, out=outs[i], workspace=ws_sp[i])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            step()
+    graph.replay()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    _barrier(world)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    del graph
+    hs2.profile_enable("*")
+    for _ in range(20):
+        step()
+    torch.cuda.synchronize()
+    hs2.profile_enable(None)
+    kern = {}
+    for name in ("dec_fused", "dec_redo", "blk_bound", "blk_rescore", "blk_final", "sparse_attn"):
+        kms, kn = hs2.profile_read(name)
+        if kn:
+            kern[name] = kms / 20
+    value = _throughput(world, steps, ms)
+    return {"workload": f"{wl.name} inputs, HySparse (v1): 16 blocks of 64 tokens by block score + a gated "
+                        f"{wl.window}-token window branch, {wl.n_sparse} gated sparse layers per step (the same "
+                        f"1,152-token budget as the token-level step)",
+            "value": value, "unit": "steps/s", "ms_per_step": ms / steps,
+            "vs_token_level": value / token_value if token_value else None,
+            "kernel_ms_per_step": kern, "device_status": [hs2.read_device_status(ws),
+                                                          max(hs2.read_device_status(w) for w in ws_sp)]}
+
+
+def bench_backward(args, world, dev, peaks, reps=3):
+    """Backward of one hybrid block at the training shape (prefill_32k: L = 32,768, 64 heads,
+    d = 128): the full layer's hs2_full_attn_bwd and the sparse layers' hs2_sparse_attn_bwd (each
+    over the full layer's selection with its own Q), adding into one pair of fp32 dK, dV buffers.
+    Reported as tok/s of the block's backward and the tensor rate of each kernel family."""
+    import torch
+    import long_context_mqa_b200 as hs2
+    wl = synth.WORKLOADS[PREFILL_WORKLOAD]
+    g = synth.SyntheticInputs(wl, seed=args.seed)
+    q, k, v = _bf16(g.q, dev), _bf16(g.k, dev), _bf16(g.v, dev)
+    out, lse, idx = hs2.full_attn_select(q, k, v, scale=wl.scale)
+    S = wl.window + wl.topk
+    qs = [_bf16(g.q_sparse(i), dev) for i in range(wl.n_sparse)]
+    fw = [hs2.sparse_attn(qs[i], k, v, idx, scale=wl.scale, want_lse=True) for i in range(wl.n_sparse)]
+    dos = [_bf16(g.grad_out(i), dev) for i in range(wl.n_sparse + 1)]
+    dq = torch.empty_like(q)
+    dqs = [torch.empty_like(q) for _ in range(wl.n_sparse)]
+    dk = torch.zeros((1, wl.Lk, wl.d), dtype=torch.float32, device=dev)
+    dv = torch.zeros_like(dk)
+    ws = torch.zeros(hs2.attn_bwd_workspace_bytes(1, wl.Lq, wl.Lk, wl.H, wl.d), dtype=torch.uint8, device=dev)
+
+    def block_bwd():
+        dk.zero_()
+        dv.zero_()
+        hs2.full_attn_bwd(q, k, v, out, lse, dos[0], scale=wl.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+        for i in range(wl.n_sparse):
+            hs2.sparse_attn_bwd(qs[i], k, v, idx, fw[i][0], fw[i][1], dos[i + 1], scale=wl.scale, dq=dqs[i], dk=dk,
+                                dv=dv, workspace=ws)
+
+    block_bwd()
+    torch.cuda.synchronize()
+    _barrier(world)
+    s = torch.cuda.current_stream()
+    hs2.profile_enable("*")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        block_bwd()
+    e1.record(s)
+    e1.synchronize()
+    hs2.profile_enable(None)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world) / reps
+    kern = {}
+    for name in ("bwd_prep", "bwd_dq", "bwd_dkdv", "sparse_bwd"):
+        kms, kn = hs2.profile_read(name)
+        if kn:
+            kern[name] = kms / reps
+    P = wl.Lq * (wl.Lq + 1) / 2
+    dq_fl, kv_fl = 6 * wl.H * wl.d * P, 8 * wl.H * wl.d * P      # executed: S, dP recomputed by both
+    sel_pairs = sum(min(t + 1, S) for t in range(wl.Lq))
+    sp_fl = 10 * wl.H * wl.d * sel_pairs                          # per sparse layer: S, dP, dQ, dK, dV
+    res = {"workload": f"{wl.name}: backward of one hybrid block (full layer + {wl.n_sparse} sparse layers), "
+                       f"L={wl.Lq}, H={wl.H}, d={wl.d}; dK, dV accumulated over the layers",
+           "tok_per_s": world * wl.Lq / (ms / 1e3), "ms": ms, "kernel_ms": kern,
+           "status": hs2.read_device_status(ws)}
+    if "bwd_dq" in kern and "bwd_dkdv" in kern:
+        full_ms = kern["bwd_dq"] + kern["bwd_dkdv"]
+        tf = (dq_fl + kv_fl) / (full_ms / 1e3) / 1e12
+        res["full_roofline"] = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": tf / peaks["bf16_tflops"],
+                                "flops": "executed 14*H*d*L(L+1)/2 (dq kernel: S, dP, dQ; dkdv kernel: S^T, dP^T, dV, dK)",
+                                "algorithmic_tflops": 10 * wl.H * wl.d * P / (full_ms / 1e3) / 1e12,
+                                "dq_tflops": dq_fl / (kern["bwd_dq"] / 1e3) / 1e12,
+                                "dkdv_tflops": kv_fl / (kern["bwd_dkdv"] / 1e3) / 1e12}
+    if "sparse_bwd" in kern:
+        per = kern["sparse_bwd"] / wl.n_sparse
+        tf = sp_fl / (per / 1e3) / 1e12
+        res["sparse_roofline"] = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": tf / peaks["bf16_tflops"], "ms_per_layer": per,
+                                  "flops": "10*H*d*sum_t min(t+1, S) per layer"}
+    if world == 1 and not args.no_cpu_baseline and int(os.environ.get("RANK", "0")) == 0:
+        import oracle
+        rows = np.concatenate([np.arange(8) + int((i + 0.5) * wl.Lq / 8) - 4 for i in range(8)])
+        t0 = time.perf_counter()
+        oracle.attn_bwd(g.q, g.k, g.v, g.grad_out(0), wl.scale, rows=rows, want_kv=False)
+        dt = time.perf_counter() - t0
+        # the dQ rows' share of the full layer's backward: the K/V side repeats the same row work
+        est = dt * wl.Lq / rows.size * 2.0
+        res["cpu_baseline"] = {"value": wl.Lq / est, "unit": "tok/s", "cores": oracle.default_threads(),
+                               "kind": "oracle", "sample": f"the full layer's dQ on {rows.size} rows (8 evenly spaced "
+                               f"strata), {dt:.1f} s, x{wl.Lq // rows.size} rows x2 for the key-side pass of the same "
+                               f"work (extrapolated; the sparse layers are not included)"}
+    del q, k, v, out, lse, idx, qs, fw, dos, dq, dqs, dk, dv
+    torch.cuda.empty_cache()
     return res
 
 

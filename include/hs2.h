@@ -222,6 +222,82 @@ HS2_API hs2_status hs2_sparse_attn_fp8kv(const hs2_bf16* Q, const uint8_t* K8, c
                                          size_t workspace_bytes, hs2_stream stream);
 
 /* ---------------------------------------------------------------------------------
+ * Backward pass (training the hybrid block)
+ * ---------------------------------------------------------------------------------
+ * The full-attention layers are trained natively as the indexer (arex-research.com, section
+ * "外层 KV Bridging，内层 KV Reuse"), and the sparse layers train through the selection, which is
+ * a constant of the backward pass (it has no gradient). For the upstream gradient dO of a layer's
+ * output these calls compute, with p the forward's softmax probabilities over a row's key set
+ * (the causal row 0..t for the full layer, the selected slots for a sparse layer):
+ *   dQ = scale sum_j dS_j k_j,  dK_j += scale sum dS_j q,  dV_j += sum p_j dO,
+ *   dS_j = p_j (dO.v_j - dO.out),
+ * the K and V sums running over every head and every row that reads key j.
+ * Q, dO, out [B, Lq, H, d] bf16 (out and lse are the forward call's outputs for these Q, K, V:
+ *     hs2_full_attn_select's, or hs2_sparse_attn's with its lse); lse [B, Lq, H] fp32 natural log;
+ * K, V [B, Lk, d] bf16; idx [B, Lq, S] (sparse: the forward's selection).
+ * dQ [B, Lq, H, d] bf16 (written).
+ * dK, dV [B, Lk, d] fp32, ACCUMULATED (+=): the full layer and every sparse layer of a block read
+ *     the same K/V (KV Reuse), so their backward calls add into one pair of buffers; zero them
+ *     before the block's first backward call. The additions use atomics (their order, and so the
+ *     last bits of the sums, may vary from run to run).
+ * Causal alignment as in the forward (query i at t = Lk - Lq + i). Supported: (H, d) in
+ * {(64, 128), (16, 64)}; sparse S <= 4096. Workspace: hs2_attn_bwd_workspace_bytes (status block
+ * plus two floats per (query, head) row).
+ */
+HS2_API size_t hs2_attn_bwd_workspace_bytes(int B, int Lq, int Lk, int H, int d);
+HS2_API hs2_status hs2_full_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const hs2_bf16* out,
+                                     const float* lse, const hs2_bf16* dO, int B, int Lq, int Lk, int H, int d,
+                                     float scale, hs2_bf16* dQ, float* dK, float* dV, void* workspace,
+                                     size_t workspace_bytes, hs2_stream stream);
+HS2_API hs2_status hs2_sparse_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                                       const hs2_bf16* out, const float* lse, const hs2_bf16* dO, int B, int Lq,
+                                       int Lk, int H, int d, int S, float scale, hs2_bf16* dQ, float* dK, float* dV,
+                                       void* workspace, size_t workspace_bytes, hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
+ * HySparse (v1) variant: block-level selection and a gated sliding-window branch
+ * ---------------------------------------------------------------------------------
+ * The predecessor design the pages compare HySparse2 against (arex-research.com, section
+ * "外层 KV Bridging，内层 KV Reuse", the paragraph on what HySparse2 changes): the full layer picks
+ * its 1,024 global tokens as 16 blocks of 64 consecutive tokens, and each sparse layer adds a
+ * separate 128-token sliding-window branch fused with the block branch by a gate. The pages do not
+ * give the block score or the gate; this library reads them as:
+ *  - block score of block J for the query at t: the sum of score(t, j) (the head-summed
+ *    probability defined for hs2_full_attn_select) over the block's tokens j <= t; every block
+ *    starting at or before t competes; ties go to the lower block. With at most n_blocks blocks
+ *    meeting 0..t, every token 0..t is taken.
+ *  - gate: a caller-given g in [0, 1] per (query, head), out = g * O_blocks + (1 - g) * O_window,
+ *    each branch its own softmax.
+ *
+ * hs2_full_attn_select_v1: the decode step's full layer (one query per sequence, at t = Lk - 1)
+ * Q [B, 1, H, d], K, V [B, Lk, d] bf16; out, lse as for hs2_full_attn_select.
+ * idx [B, 1, n_blocks * block + window] int32: slots [0, n_blocks * block) hold the chosen blocks'
+ *     tokens <= t in ascending order, then -1; slots [n_blocks * block, +window) hold the window
+ *     t - window + 1 .. t (clamped at 0) ascending, then -1.
+ * Supported: (H, d) = (64, 128), block = 64, 1 <= n_blocks <= 32, n_blocks * block + window <= 2048,
+ * 1 <= B <= 256. The selection is exact: the decode kernel's bounded token scores bound every
+ * block's score, and the blocks that can reach the top n_blocks are re-scored exactly.
+ * Workspace: hs2_full_attn_select_v1_workspace_bytes (zero-filled before first use).
+ *
+ * hs2_sparse_attn_v1: one sparse layer of the v1 design, with the full layer's K/V and idx.
+ * idx [B, Lq, S]: slots [0, branch) the block branch, [branch, S) the window branch (-1 skipped;
+ *     each branch needs one valid entry); gate [B, Lq, H] fp32 in [0, 1] (DEVICE).
+ * out [B, Lq, H, d] bf16 = gate * softmax-attention over the block branch + (1 - gate) *
+ *     softmax-attention over the window branch. branch % 128 == 0, 0 < branch < S <= 2048,
+ *     (H, d) = (64, 128). Workspace: hs2_sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S).
+ */
+HS2_API size_t hs2_full_attn_select_v1_workspace_bytes(int B, int Lk, int H, int d, int window, int block,
+                                                       int n_blocks);
+HS2_API hs2_status hs2_full_attn_select_v1(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lk,
+                                           int H, int d, float scale, int window, int block, int n_blocks,
+                                           hs2_bf16* out, float* lse, int32_t* idx, void* workspace,
+                                           size_t workspace_bytes, hs2_stream stream);
+HS2_API hs2_status hs2_sparse_attn_v1(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                                      const float* gate, int B, int Lq, int Lk, int H, int d, int S, int branch,
+                                      float scale, hs2_bf16* out, void* workspace, size_t workspace_bytes,
+                                      hs2_stream stream);
+
+/* ---------------------------------------------------------------------------------
  * Sparse attention without a caller workspace
  * ---------------------------------------------------------------------------------
  * No counterpart in the paper: a library convenience for callers that cannot allocate

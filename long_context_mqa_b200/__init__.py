@@ -82,6 +82,18 @@ def _load_library() -> ctypes.CDLL:
     lib.hs2_sparse_attn_fp8kv.restype = i32
     lib.hs2_selftest_e4m3.argtypes = [P, P, P, i32, P]
     lib.hs2_selftest_e4m3.restype = i32
+    lib.hs2_full_attn_select_v1_workspace_bytes.argtypes = [i32] * 7
+    lib.hs2_full_attn_select_v1_workspace_bytes.restype = sz
+    lib.hs2_full_attn_select_v1.argtypes = [P, P, P, i32, i32, i32, i32, f32, i32, i32, i32, P, P, P, P, sz, P]
+    lib.hs2_full_attn_select_v1.restype = i32
+    lib.hs2_sparse_attn_v1.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, P, P, sz, P]
+    lib.hs2_sparse_attn_v1.restype = i32
+    lib.hs2_attn_bwd_workspace_bytes.argtypes = [i32] * 5
+    lib.hs2_attn_bwd_workspace_bytes.restype = sz
+    lib.hs2_full_attn_bwd.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, P, P, sz, P]
+    lib.hs2_full_attn_bwd.restype = i32
+    lib.hs2_sparse_attn_bwd.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, P, sz, P]
+    lib.hs2_sparse_attn_bwd.restype = i32
     lib.hs2_bridge_kv_proj_workspace_bytes.argtypes = [i32] * 4
     lib.hs2_bridge_kv_proj_workspace_bytes.restype = sz
     lib.hs2_bridge_kv_proj.argtypes = [P, i32, i32, P, i32, i32, P, P, sz, P]
@@ -184,6 +196,136 @@ def full_attn_select(q, k, v, *, scale=None, window=WINDOW, topk=TOPK, out=None,
                                     ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(code, "hs2_full_attn_select")
     return out, lse, idx
+
+
+V1_BLOCK = 64
+V1_BLOCKS = 16
+
+
+def full_attn_select_v1_workspace_bytes(B, Lk, H, d, window=WINDOW, block=V1_BLOCK, n_blocks=V1_BLOCKS) -> int:
+    return int(lib.hs2_full_attn_select_v1_workspace_bytes(B, Lk, H, d, window, block, n_blocks))
+
+
+def full_attn_select_v1(q, k, v, *, scale=None, window=WINDOW, block=V1_BLOCK, n_blocks=V1_BLOCKS, out=None,
+                        lse=None, idx=None, workspace=None, stream=None):
+    """Decode full layer with HySparse (v1) block selection (hs2_full_attn_select_v1).
+
+    q [B,1,H,d]; k, v [B,Lk,d]. Returns (out [B,1,H,d] bf16, lse [B,1,H] fp32, idx
+    [B,1,n_blocks*block+window] int32: the chosen blocks' tokens, then the window).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    if Lq != 1 or tuple(k.shape) != (B, Lk, d) or tuple(v.shape) != (B, Lk, d):
+        raise ValueError("q must be [B,1,H,d] and k, v [B,Lk,d]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    S = n_blocks * block + window
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, 1, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    idx = torch.empty((B, 1, S), dtype=torch.int32, device=q.device) if idx is None else idx
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    nbytes = full_attn_select_v1_workspace_bytes(B, Lk, H, d, window, block, n_blocks)
+    ws = _workspace(nbytes, q.device, "full_v1") if workspace is None else workspace
+    code = lib.hs2_full_attn_select_v1(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Lk, H, d, scale, window, block,
+                                       n_blocks, out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                       ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_select_v1")
+    return out, lse, idx
+
+
+def sparse_attn_v1(q, k, v, idx, gate, *, branch=V1_BLOCK * V1_BLOCKS, scale=None, out=None, workspace=None,
+                   stream=None):
+    """Sparse layer of the v1 design (hs2_sparse_attn_v1): gate * attention over idx slots
+    [0, branch) + (1 - gate) * attention over slots [branch, S). gate [B,Lq,H] fp32."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(idx, "idx", torch.int32, 3)
+    _need(gate, "gate", torch.float32, 3)
+    B, Lq, H, d = q.shape
+    Lk, S = k.shape[1], idx.shape[2]
+    if tuple(idx.shape[:2]) != (B, Lq) or tuple(gate.shape) != (B, Lq, H):
+        raise ValueError("idx must be [B,Lq,S] and gate [B,Lq,H]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", torch.bfloat16, 4)
+    nbytes = sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S)
+    ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
+    code = lib.hs2_sparse_attn_v1(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), gate.data_ptr(), B, Lq,
+                                  Lk, H, d, S, branch, scale, out.data_ptr(), ws.data_ptr(),
+                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_sparse_attn_v1")
+    return out
+
+
+def attn_bwd_workspace_bytes(B, Lq, Lk, H, d) -> int:
+    return int(lib.hs2_attn_bwd_workspace_bytes(B, Lq, Lk, H, d))
+
+
+def _bwd_outputs(q, k, dq, dk, dv):
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.zeros((B, Lk, d), dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.zeros((B, Lk, d), dtype=torch.float32, device=q.device) if dv is None else dv
+    _need(dq, "dq", torch.bfloat16, 4)
+    _need(dk, "dk", torch.float32, 3)
+    _need(dv, "dv", torch.float32, 3)
+    return dq, dk, dv
+
+
+def full_attn_bwd(q, k, v, out, lse, do, *, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward of the full layer's causal attention (hs2_full_attn_bwd).
+
+    out, lse: the forward's outputs for q, k, v; do: [B,Lq,H,d] bf16 upstream gradient.
+    Returns (dq [B,Lq,H,d] bf16, dk, dv [B,Lk,d] fp32). dk and dv are ADDED into when given
+    (zeros otherwise): the layers of a block share K and V.
+    """
+    for t, n in ((q, "q"), (out, "out"), (do, "do")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 3)
+    B, Lq, H, d = q.shape
+    Lk = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = _bwd_outputs(q, k, dq, dk, dv)
+    nbytes = attn_bwd_workspace_bytes(B, Lq, Lk, H, d)
+    ws = _workspace(nbytes, q.device, "bwd") if workspace is None else workspace
+    code = lib.hs2_full_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), B, Lq, Lk, H, d, scale, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                 ws.data_ptr(), ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(code, "hs2_full_attn_bwd")
+    return dq, dk, dv
+
+
+def sparse_attn_bwd(q, k, v, idx, out, lse, do, *, scale=None, dq=None, dk=None, dv=None, workspace=None,
+                    stream=None):
+    """Backward of a sparse layer over the selected tokens (hs2_sparse_attn_bwd); out and lse
+    are the forward sparse layer's (sparse_attn with want_lse=True). Returns (dq, dk, dv) as
+    full_attn_bwd, dk and dv accumulated."""
+    for t, n in ((q, "q"), (out, "out"), (do, "do")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 3)
+    _need(idx, "idx", torch.int32, 3)
+    B, Lq, H, d = q.shape
+    Lk, S = k.shape[1], idx.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = _bwd_outputs(q, k, dq, dk, dv)
+    nbytes = attn_bwd_workspace_bytes(B, Lq, Lk, H, d)
+    ws = _workspace(nbytes, q.device, "bwd") if workspace is None else workspace
+    code = lib.hs2_sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), do.data_ptr(), B, Lq, Lk, H, d, S, scale, dq.data_ptr(),
+                                   dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                   _stream_ptr(stream))
+    _check(code, "hs2_sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def _lens_array(lens, B, Lk):

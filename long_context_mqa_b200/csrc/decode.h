@@ -86,6 +86,69 @@ struct SelParams {
 cudaError_t launch_select(const SelParams& p, cudaStream_t stream);
 }  // namespace sel
 
+namespace blk {
+// HySparse (v1) block-level selection after the fused decode kernel (blocksel.cu).
+struct BlkParams {
+  int B, H, D, W;                // sequences, heads, head dim, window
+  int NB, BLK, S;                // blocks chosen, tokens per block (64), idx row length NB * BLK + W
+  dec::Sched sch;                // per-sequence lengths (query at t = seq_len - 1)
+  const float* sc;               // [B][ncand] the decode kernel's bounded scores score' of the older tokens
+  int ncand;
+  const float* lsum;             // [B][H] L'_h
+  const float* lse2x;            // [B][H] exact lse, log2 units
+  int max_blocks;                // ceil(N / BLK): the stride of cand and bsc
+  int* cnt;                      // [B] candidate blocks of each sequence
+  int* cand;                     // [B][max_blocks] candidate block ids
+  float* bsc;                    // [B][max_blocks] their exact block scores (S' of full blocks in between)
+  int32_t* idx;                  // [B][S] output
+  unsigned* gbar;                // the decode kernel's grid-barrier counters, re-armed here
+  // exact re-score
+  const __nv_bfloat16* qry;      // [B][H][D]
+  const __nv_bfloat16* kc;       // [B][N][D]
+  int N;
+  float c;                       // scale * log2(e)
+  int sms;
+  long long wait_ns;
+  // decode output (the decode kernel's records / L')
+  const float* opart;
+  float oscale;
+  __nv_bfloat16* out;
+  DevStatus* st;
+};
+cudaError_t launch_block_select(const BlkParams& p, cudaStream_t stream);
+}  // namespace blk
+
+namespace bwd {
+// Backward pass of the full layer (causal MQA attention) and of a sparse layer (backward.cu).
+struct BwdParams {
+  int B, Lq, Lk, H, D;
+  int off;                    // Lk - Lq: query i sits at position off + i
+  int rows_per_batch;         // Lq * H (query, head) rows per sequence
+  int tiles_per_batch;        // ceil(rows_per_batch / 128)
+  int kv_tiles;               // ceil(Lk / 128)
+  int chunk;                  // row tiles per key-side work item
+  int n_chunks;               // ceil(tiles_per_batch / chunk)
+  float c;                    // scale * log2(e)
+  float scale;
+  const float* lse2;          // [B * Lq * H] forward logsumexp, log2 units
+  const float* Dv;            // [B * Lq * H] <dO, out> per row
+  __nv_bfloat16* dQ;          // [B, Lq, H, D]
+  float* dK;                  // [B, Lk, D] accumulated (+=)
+  float* dV;
+  // sparse layer
+  const __nv_bfloat16 *Q, *K, *V, *dO;
+  const int32_t* idx;         // [B, Lq, S]
+  int S;
+  long long wait_ns;
+  DevStatus* st;
+};
+cudaError_t launch_prep(const __nv_bfloat16* dO, const __nv_bfloat16* out, const float* lse, float* Dv, float* lse2,
+                        long long n_rows, int D, cudaStream_t stream);
+cudaError_t launch_full_bwd(const CUtensorMap& tmQ, const CUtensorMap& tmdO, const CUtensorMap& tmK,
+                            const CUtensorMap& tmV, const BwdParams& p, int sms, cudaStream_t stream);
+cudaError_t launch_sparse_bwd(const BwdParams& p, int sms, cudaStream_t stream);
+}  // namespace bwd
+
 namespace sparse {
 struct SpParams {
   const __nv_bfloat16 *Q, *K, *V;
@@ -101,6 +164,11 @@ struct SpParams {
   long long wait_ns;
   const int32_t* ptab;        // paged cache: [B][max_pages] page ids, K/V are the page pools of
   int max_pages, n_pages;     // n_pages x 128 rows (NULL: K/V are [B][Lk] rows)
+  // two gated branches (HySparse v1): splits [0, branch_split) attend over the block branch,
+  // the rest over the window branch; out = g * (block branch) + (1 - g) * (window branch) with
+  // g = gate[row][head]. NULL: one softmax over every slot.
+  const float* gate;
+  int branch_split;
   DevStatus* st;
 };
 size_t sparse_smem_bytes(int H, int D, int nsplit);

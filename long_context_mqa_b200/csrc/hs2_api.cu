@@ -333,13 +333,13 @@ size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d,
 // The decode path (one query per sequence at the end of its lens[b]-token cache). K, V are
 // [B][Lk] rows, or (ptab != NULL) pools of n_pages pages of 128 rows with Lk = max_pages * 128;
 // bf16, or (f8) e4m3 codes with c including K's scale and oscale V's.
-static hs2_status run_decode(const void* Q, const void* K, const void* V, int B, const int* lens, int Lk,
-                             int H, int d, float c, int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
-                             void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
-                             const int32_t* ptab = nullptr, int max_pages = 0, int n_pages = 0, bool f8 = false,
-                             float oscale = 1.f) {
+// The fused decode kernel (and its exact redo) alone; w receives the workspace layout.
+static hs2_status launch_decode_fused(DecodeWs& w, const void* Q, const void* K, const void* V, int B,
+                                      const int* lens, int Lk, int H, int d, float c, int window, int topk,
+                                      float* lse, void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
+                                      const int32_t* ptab, int max_pages, int n_pages, bool f8) {
   if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
-  DecodeWs w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
+  w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
   if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
   if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
   w.p.c = c;
@@ -359,6 +359,18 @@ static hs2_status run_decode(const void* Q, const void* K, const void* V, int B,
       !make_tmap_3d(&tmQ, Q, d, H, B, d, (uint64_t)H * d, 64, H))
     return HS2_ERR_CUDA;
   if (dec::launch_decode_attn(tmK, tmV, tmQ, w.p, f8, st) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+static hs2_status run_decode(const void* Q, const void* K, const void* V, int B, const int* lens, int Lk,
+                             int H, int d, float c, int window, int topk, hs2_bf16* out, float* lse, int32_t* idx,
+                             void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
+                             const int32_t* ptab = nullptr, int max_pages = 0, int n_pages = 0, bool f8 = false,
+                             float oscale = 1.f) {
+  DecodeWs w{};
+  const hs2_status rc = launch_decode_fused(w, Q, K, V, B, lens, Lk, H, d, c, window, topk, lse, workspace,
+                                            workspace_bytes, sms, st, ptab, max_pages, n_pages, f8);
+  if (rc != HS2_OK) return rc;
   sel::SelParams sp;
   sp.opart = w.p.opart;
   sp.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -532,6 +544,243 @@ hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, con
   if (n_pages <= 0 || max_pages <= 0 || max_pages > (1 << 23)) return HS2_ERR_INVALID_ARG;
   return run_sparse(Q, K_pages, V_pages, idx, B, Lq, max_pages * 128, H, d, S, scale, out, lse, workspace,
                     workspace_bytes, stream, page_table, max_pages, n_pages);
+}
+
+// ------------------------------------------------------------------------------------------
+// HySparse (v1): block-level selection and the gated two-branch sparse layer
+// ------------------------------------------------------------------------------------------
+struct V1Ws {
+  size_t dec_bytes, bytes;
+  int max_blocks;
+  int* cnt;
+  int* cand;
+  float* bsc;
+};
+
+// the decode workspace, then the candidate count, list and scores of the block selection
+static V1Ws carve_v1(void* ws, size_t dec_bytes, int B, int Lk, int block) {
+  V1Ws v{};
+  v.dec_bytes = dec_bytes;
+  v.max_blocks = (Lk + block - 1) / block;
+  Carve c{(uint8_t*)ws, dec_bytes};
+  v.cnt = c.take<int>((size_t)B);
+  v.cand = c.take<int>((size_t)B * v.max_blocks);
+  v.bsc = c.take<float>((size_t)B * v.max_blocks);
+  v.bytes = c.off;
+  return v;
+}
+
+static bool v1_shape_ok(int H, int d, int window, int block, int n_blocks) {
+  return H == 64 && d == 128 && block == 64 && n_blocks >= 1 && n_blocks <= 32 && window >= 1 &&
+         n_blocks * block + window <= 2048;
+}
+
+size_t hs2_full_attn_select_v1_workspace_bytes(int B, int Lk, int H, int d, int window, int block, int n_blocks) {
+  if (B <= 0 || B > dec::kMaxSeqs || Lk <= 0 || !v1_shape_ok(H, d, window, block, n_blocks)) return 0;
+  const int sms = num_sms() > 0 ? num_sms() : 148;
+  std::vector<int> lens((size_t)B, Lk);
+  const DecodeWs w = carve_decode(nullptr, B, lens.data(), Lk, H, d, window, n_blocks * block, sms);
+  if (!w.ok) return 0;
+  return carve_v1(nullptr, w.bytes, B, Lk, block).bytes;
+}
+
+hs2_status hs2_full_attn_select_v1(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lk, int H,
+                                   int d, float scale, int window, int block, int n_blocks, hs2_bf16* out,
+                                   float* lse, int32_t* idx, void* workspace, size_t workspace_bytes,
+                                   hs2_stream stream) {
+  if (!Q || !K || !V || !out || !lse || !idx) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(lse) || !aligned16(idx))
+    return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lk <= 0 || window < 1 || block <= 0 || n_blocks <= 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (B > dec::kMaxSeqs || !v1_shape_ok(H, d, window, block, n_blocks)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  const int sms = num_sms();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float c = scale * 1.4426950408889634f;
+  std::vector<int> lens((size_t)B, Lk);
+  // the decode kernel's own bounds are computed for a top-k of n_blocks * block tokens (unused here)
+  DecodeWs w{};
+  if (workspace_bytes < hs2_full_attn_select_v1_workspace_bytes(B, Lk, H, d, window, block, n_blocks))
+    return HS2_ERR_WORKSPACE;
+  const hs2_status rc = launch_decode_fused(w, Q, K, V, B, lens.data(), Lk, H, d, c, window, n_blocks * block, lse,
+                                            workspace, workspace_bytes, sms, st, nullptr, 0, 0, false);
+  if (rc != HS2_OK) return rc;
+  const V1Ws v = carve_v1(workspace, w.bytes, B, Lk, block);
+  blk::BlkParams bp{};
+  bp.B = B; bp.H = H; bp.D = d; bp.W = window;
+  bp.NB = n_blocks; bp.BLK = block; bp.S = n_blocks * block + window;
+  bp.sch = w.p.sch;
+  bp.sc = w.p.sc; bp.ncand = w.p.sc_stride;
+  bp.lsum = w.p.lsum; bp.lse2x = w.p.lse2x;
+  bp.max_blocks = v.max_blocks; bp.cnt = v.cnt; bp.cand = v.cand; bp.bsc = v.bsc;
+  bp.idx = idx;
+  bp.gbar = w.p.gbar;
+  bp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
+  bp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
+  bp.N = Lk;
+  bp.c = c;
+  bp.sms = sms;
+  bp.wait_ns = w.p.wait_ns;
+  bp.opart = w.p.opart; bp.oscale = 1.f;
+  bp.out = reinterpret_cast<__nv_bfloat16*>(out);
+  bp.st = w.p.st;
+  if (blk::launch_block_select(bp, st) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+hs2_status hs2_sparse_attn_v1(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                              const float* gate, int B, int Lq, int Lk, int H, int d, int S, int branch, float scale,
+                              hs2_bf16* out, void* workspace, size_t workspace_bytes, hs2_stream stream) {
+  if (!Q || !K || !V || !idx || !gate || !out) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HS2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) != 0 || (reinterpret_cast<uintptr_t>(gate) & 3u) != 0)
+    return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || S <= 0 || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (branch <= 0 || branch >= S || branch % 128 != 0) return HS2_ERR_INVALID_ARG;
+  if (H != 64 || d != 128 || S > 2048) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * Lq > 2147483647LL / 16) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  sparse::SpParams p{};
+  const size_t need = carve_sparse(workspace, B, Lq, H, d, S, num_sms(), &p);
+  if (workspace_bytes < need) return HS2_ERR_WORKSPACE;
+  // one split (CTA of the row's cluster) per 128 slots, so the branch boundary falls between splits
+  p.nsplit = (S + 127) / 128;
+  p.split_slots = 128;
+  p.branch_split = branch / 128;
+  p.gate = gate;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.oscale = 1.f;
+  p.idx = idx;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.S = S;
+  p.c = scale * 1.4426950408889634f;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = nullptr;
+  p.wait_ns = wait_limit_ns();
+  if (sparse::launch_sparse(p, H, d, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// backward pass of the full layer and of a sparse layer
+// ------------------------------------------------------------------------------------------
+struct BwdWs {
+  DevStatus* st;
+  float* Dv;
+  float* lse2;
+  size_t bytes;
+};
+
+// status block | D per (query, head) row | lse2 per row; both arrays padded by a 128-row tile (the
+// key-side kernel copies a whole tile's values with its Q tile)
+static BwdWs carve_bwd(void* ws, long long rows) {
+  BwdWs w{};
+  Carve c{(uint8_t*)ws, 0};
+  w.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
+  w.Dv = c.take<float>((size_t)rows + 128);
+  w.lse2 = c.take<float>((size_t)rows + 128);
+  w.bytes = c.off;
+  return w;
+}
+
+size_t hs2_attn_bwd_workspace_bytes(int B, int Lq, int Lk, int H, int d) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || !shape_ok(H, d)) return 0;
+  return carve_bwd(nullptr, (long long)B * Lq * H).bytes;
+}
+
+static hs2_status bwd_args_ok(const void* Q, const void* K, const void* V, const void* out, const float* lse,
+                              const void* dO, const void* dQ, const float* dK, const float* dV, int B, int Lq, int Lk,
+                              int H, int d, float scale, const void* workspace) {
+  if (!Q || !K || !V || !out || !lse || !dO || !dQ || !dK || !dV) return HS2_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return HS2_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || !(scale > 0.f)) return HS2_ERR_INVALID_ARG;
+  if (!shape_ok(H, d)) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * Lq * H > 2147483647LL - 256 || (long long)B * Lk > 2147483647LL / 128)
+    return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!device_is_sm100()) return HS2_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || !aligned16(workspace)) return HS2_ERR_WORKSPACE;
+  return HS2_OK;
+}
+
+hs2_status hs2_full_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const hs2_bf16* out,
+                             const float* lse, const hs2_bf16* dO, int B, int Lq, int Lk, int H, int d, float scale,
+                             hs2_bf16* dQ, float* dK, float* dV, void* workspace, size_t workspace_bytes,
+                             hs2_stream stream) {
+  const hs2_status rc = bwd_args_ok(Q, K, V, out, lse, dO, dQ, dK, dV, B, Lq, Lk, H, d, scale, workspace);
+  if (rc != HS2_OK) return rc;
+  const long long rows = (long long)B * Lq * H;
+  const BwdWs w = carve_bwd(workspace, rows);
+  if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  CUtensorMap tmQ, tmdO, tmK, tmV;
+  if (!make_tmap_2d(&tmQ, Q, d, (uint64_t)rows, d, 64, 128) || !make_tmap_2d(&tmdO, dO, d, (uint64_t)rows, d, 64, 128) ||
+      !make_tmap_3d(&tmK, K, d, Lk, B, d, (uint64_t)Lk * d, 64, 128) ||
+      !make_tmap_3d(&tmV, V, d, Lk, B, d, (uint64_t)Lk * d, 64, 128))
+    return HS2_ERR_CUDA;
+  const __nv_bfloat16* bQ = reinterpret_cast<const __nv_bfloat16*>(Q);
+  if (bwd::launch_prep(reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(out), lse,
+                       w.Dv, w.lse2, rows, d, st) != cudaSuccess)
+    return HS2_ERR_CUDA;
+  bwd::BwdParams p{};
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = H; p.D = d;
+  p.off = Lk - Lq;
+  p.rows_per_batch = Lq * H;
+  p.tiles_per_batch = (Lq * H + 127) / 128;
+  p.kv_tiles = (Lk + 127) / 128;
+  // key-side work items: a key tile and at most `chunk` row tiles, about a dozen per SM at 32k
+  p.chunk = p.tiles_per_batch / 16 > 16 ? p.tiles_per_batch / 16 : 16;
+  p.n_chunks = (p.tiles_per_batch + p.chunk - 1) / p.chunk;
+  p.c = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.lse2 = w.lse2; p.Dv = w.Dv;
+  p.dQ = reinterpret_cast<__nv_bfloat16*>(dQ);
+  p.dK = dK; p.dV = dV;
+  p.Q = bQ;
+  p.wait_ns = wait_limit_ns();
+  p.st = w.st;
+  if (bwd::launch_full_bwd(tmQ, tmdO, tmK, tmV, p, sms, st) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
+}
+
+hs2_status hs2_sparse_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, const int32_t* idx,
+                               const hs2_bf16* out, const float* lse, const hs2_bf16* dO, int B, int Lq, int Lk, int H,
+                               int d, int S, float scale, hs2_bf16* dQ, float* dK, float* dV, void* workspace,
+                               size_t workspace_bytes, hs2_stream stream) {
+  hs2_status rc = bwd_args_ok(Q, K, V, out, lse, dO, dQ, dK, dV, B, Lq, Lk, H, d, scale, workspace);
+  if (rc != HS2_OK) return rc;
+  if (!idx || (reinterpret_cast<uintptr_t>(idx) & 3u) != 0 || S <= 0) return HS2_ERR_INVALID_ARG;
+  if (S > 4096) return HS2_ERR_UNSUPPORTED_SHAPE;
+  const long long rows = (long long)B * Lq * H;
+  const BwdWs w = carve_bwd(workspace, rows);
+  if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (bwd::launch_prep(reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(out), lse,
+                       w.Dv, w.lse2, rows, d, st) != cudaSuccess)
+    return HS2_ERR_CUDA;
+  bwd::BwdParams p{};
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = H; p.D = d;
+  p.off = Lk - Lq;
+  p.S = S;
+  p.c = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.lse2 = w.lse2; p.Dv = w.Dv;
+  p.dQ = reinterpret_cast<__nv_bfloat16*>(dQ);
+  p.dK = dK; p.dV = dV;
+  p.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  p.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  p.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  p.dO = reinterpret_cast<const __nv_bfloat16*>(dO);
+  p.idx = idx;
+  p.wait_ns = wait_limit_ns();
+  p.st = w.st;
+  if (bwd::launch_sparse_bwd(p, num_sms(), st) != cudaSuccess) return HS2_ERR_CUDA;
+  return HS2_OK;
 }
 
 static bool kv_scale_ok(float s) { return s > 0.f && s < INFINITY; }

@@ -20,6 +20,7 @@
 //                same launch produce the decode output (independent of the selection): per
 //                (sequence, head), the sum of the output records of the CTAs covering the
 //                sequence, divided by L' (and multiplied by an e4m3 V cache's scale).
+#include "combine.cuh"
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -29,29 +30,9 @@ namespace sel {
 
 constexpr int NT = 1024;
 
-// The decode output of head h of sequence b, by one warp (lane = 4 columns): the decode kernel's
-// CTAs c_lo..c_hi covering the sequence left one unnormalised record each, in consecutive slots
-// from b * cmax; their sum divided by L'_h.
+// The decode output of head h of sequence b, by one warp (lane = 4 columns).
 __device__ __forceinline__ void combine_output(const SelParams& p, int b, int h, unsigned lane) {
-  int g, c_lo, c_hi;
-  p.sch.covering(b, g, c_lo, c_hi);
-  const int n_slots = c_hi - c_lo + 1;
-  if (n_slots > p.sch.cmax || p.D != 128) {
-    if (lane == 0) report_status(p.st, kStatusBounds, 303);
-    return;
-  }
-  const float4* rec = reinterpret_cast<const float4*>(p.opart + ((size_t)p.sch.slot(b, c_lo, c_lo) * p.H + h) * p.D) + lane;
-  const size_t rstride = (size_t)p.H * p.D / 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-  for (int i = 0; i < n_slots; ++i) {
-    const float4 v = __ldcg(rec + i * rstride);
-    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-  }
-  const float inv = p.oscale / p.lsum[b * p.H + h];  // the records are sums of p' v, p' unnormalised
-  __nv_bfloat16* o = p.out + ((size_t)b * p.H + h) * p.D + 4 * lane;
-  reinterpret_cast<__nv_bfloat162*>(o)[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  reinterpret_cast<__nv_bfloat162*>(o)[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  combine_decode_output(p.opart, p.lsum, p.oscale, p.out, p.H, p.D, p.sch, p.st, b, h, lane);
 }
 
 // Scores one bitmap CTA of the collect kernel classifies: 256 threads x 8 steps x 4 scores.

@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
   cluster_sync_all();  // all partials have landed; nothing reads another CTA's memory after this
   // merge weights of this rank's heads (thread k < HPR: head rank + k*n)
-  if (tid < HPR) {
+  if (tid < HPR && !p.gate) {
     const int h = (int)rank + tid * n;
     if (h < H) {
       float M = -INFINITY, L = 0.f;
@@ -394,6 +394,28 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
       }
       wgt[16 * MH + tid] = L > 0.f ? p.oscale / L : 0.f;
       if (p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
+    }
+  } else if (tid < HPR) {
+    // two branches, each its own softmax (splits below branch_split: the blocks; the rest: the
+    // window), mixed by the gate: the weights carry each branch's normalisation and its share
+    const int h = (int)rank + tid * n;
+    if (h < H) {
+      const float g = p.gate[(size_t)r * H + h];
+      float M[2] = {-INFINITY, -INFINITY}, L[2] = {0.f, 0.f};
+      for (int s2 = 0; s2 < n; ++s2) {
+        const int br = s2 < p.branch_split ? 0 : 1;
+        if (xl[s2 * MH + h] > 0.f) M[br] = fmaxf(M[br], xm[s2 * MH + h]);
+      }
+      for (int s2 = 0; s2 < n; ++s2) {
+        const int br = s2 < p.branch_split ? 0 : 1;
+        const float l = xl[s2 * MH + h];
+        const float w = l > 0.f ? exp2f(xm[s2 * MH + h] - M[br]) : 0.f;
+        wgt[s2 * MH + tid] = w;
+        L[br] += l * w;
+      }
+      const float f0 = L[0] > 0.f ? g / L[0] : 0.f, f1 = L[1] > 0.f ? (1.f - g) / L[1] : 0.f;
+      for (int s2 = 0; s2 < n; ++s2) wgt[s2 * MH + tid] *= s2 < p.branch_split ? f0 : f1;
+      wgt[16 * MH + tid] = p.oscale;
     }
   }
   __syncthreads();
@@ -454,6 +476,9 @@ static cudaError_t launch_t(const SpParams& p, cudaStream_t stream) {
 
 cudaError_t launch_sparse(const SpParams& p, int H, int D, cudaStream_t stream) {
   if (p.nsplit < 1 || p.nsplit > 16) return cudaErrorInvalidValue;  // merge table and cluster size
+  // the gated branches merge across the cluster: at least one split on each side of the boundary
+  if (p.gate && (p.nsplit < 2 || p.branch_split < 1 || p.branch_split >= p.nsplit || p.lse))
+    return cudaErrorInvalidValue;
   if (H == 64 && D == 128) return launch_t<64, 128>(p, stream);
   if (H == 16 && D == 64) return launch_t<16, 64>(p, stream);
   return cudaErrorInvalidValue;

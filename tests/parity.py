@@ -97,3 +97,49 @@ def assert_out_close(gpu, ref, what: str, max_abs=OUT_MAX_ABS, rel_l2=OUT_REL_L2
     ma, rl = out_errors(gpu, ref)
     assert ma <= max_abs and rl <= rel_l2, f"{what}: max-abs {ma:.3g} (<= {max_abs}), rel-L2 {rl:.3g} (<= {rel_l2})"
     return ma, rl
+
+
+def check_block_selection(gpu_row: np.ndarray, ora_tokens: np.ndarray, ora_bscore: np.ndarray, t: int,
+                          block: int, n_blocks: int, window: int, rel_tol: float = SWAP_REL_TOL) -> SelStats:
+    """One query's HySparse (v1) selection row: slots [0, n_blocks * block) must hold whole blocks'
+    tokens <= t ascending then -1, the chosen blocks equal to the oracle's except swaps whose
+    oracle block scores differ by <= rel_tol relative (paired in oracle-score order); slots
+    [n_blocks * block, +window) must hold the window exactly."""
+    st = SelStats(rows=1)
+    nbs = n_blocks * block
+    g = gpu_row[:nbs]
+    n_valid = int((g >= 0).sum())
+    gv = g[:n_valid]
+    problems = []
+    if not (g[n_valid:] == -1).all():
+        problems.append("block slots: -1 padding not at the tail")
+    if n_valid and ((gv > t).any() or not (np.diff(gv) > 0).all()):
+        problems.append("block slots: not ascending / not causal")
+    blocks = np.unique(gv // block)
+    want_tok = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in blocks]) if len(blocks) else gv
+    if not np.array_equal(gv, want_tok):
+        problems.append("block slots: not whole blocks")
+    ob = np.unique(ora_tokens // block)
+    a = np.setdiff1d(blocks, ob)
+    b = np.setdiff1d(ob, blocks)
+    if len(a) != len(b):
+        problems.append(f"block set sizes differ ({len(blocks)} vs {len(ob)})")
+    else:
+        a = a[np.argsort(-ora_bscore[a], kind="stable")]
+        b = b[np.argsort(-ora_bscore[b], kind="stable")]
+        for x, y in zip(a, b):
+            m = max(ora_bscore[x], ora_bscore[y])
+            rel = abs(ora_bscore[x] - ora_bscore[y]) / m if m > 0 else 0.0
+            st.max_swap_rel = max(st.max_swap_rel, rel)
+            if rel > rel_tol:
+                problems.append(f"block swap {x}<->{y} scores {ora_bscore[x]:.9g} vs {ora_bscore[y]:.9g}")
+                break
+            st.swaps += 1
+    lo = max(0, t - window + 1)
+    win = np.full(window, -1, np.int64)
+    win[:t - lo + 1] = np.arange(lo, t + 1)
+    if not np.array_equal(gpu_row[nbs:nbs + window], win):
+        problems.append("window slots differ")
+    if problems:
+        st.failures.append((0, t, problems))
+    return st
