@@ -888,7 +888,7 @@ def bench_v1(args, world, wl, hs2, q, k, v, qs, peaks, token_value, steps=200, w
     torch.cuda.synchronize()
     hs2.profile_enable(None)
     kern = {}
-    for name in ("dec_fused", "dec_redo", "blk_bound", "blk_rescore", "blk_final", "sparse_attn"):
+    for name in ("dec_fused", "dec_redo", "blk_score", "blk_final", "sparse_attn"):
         kms, kn = hs2.profile_read(name)
         if kn:
             kern[name] = kms / 20

@@ -25,8 +25,10 @@
 //           memory), then dQ += dS K_sel (M = 64) and dK_sel = dS^T Q, dV_sel = P^T dO (M = 128
 //           keys: the same shared-memory tiles read MN-major), scattered into dK, dV by
 //           red.global.add.v4 (a key selected by many rows receives many adds).
-// Warp roles of dq / dkdv (192 threads): warp 0 TMA producer, warp 1 tcgen05 issuer + TMEM owner,
-// warps 2..5 the row (or key) threads. Every wait is bounded and reports a timeout.
+// Warp roles of dq / dkdv (320 threads): warp 0 TMA producer, warp 1 tcgen05 issuer + TMEM owner,
+// warps 2..9 the row (or key) threads: a TMEM lane (row or key) is owned by one warp of each of
+// the two warpgroups, which split its 128 columns (warpgroup g takes columns 64 g .. 64 g + 63).
+// Every wait is bounded and reports a timeout.
 #include "decode.h"
 #include "host_util.h"
 #include "tc.cuh"
@@ -35,7 +37,7 @@ namespace hs2 {
 namespace bwd {
 
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr int NT = 192;
+constexpr int NT = 320;  // dq / dkdv: producer warp, issuer warp, two warpgroups of row (key) threads
 
 __device__ __forceinline__ bool wait_abortable(uint64_t* bar, uint32_t parity, long long limit, volatile int* abort_flag,
                                                DevStatus* st, unsigned where) {
@@ -146,9 +148,9 @@ __global__ void __launch_bounds__(NT, 1)
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1); mbar_init(&q_empty, 1);
     for (int i = 0; i < C::RING; ++i) { mbar_init(&r_full[i], 1); mbar_init(&r_empty[i], 1); }
-    mbar_init(&s_full, 1); mbar_init(&s_empty, 4);
-    mbar_init(&ds_full, 4); mbar_init(&ds_empty, 1);
-    mbar_init(&dq_full, 1); mbar_init(&dq_empty, 4);
+    mbar_init(&s_full, 1); mbar_init(&s_empty, 8);
+    mbar_init(&ds_full, 8); mbar_init(&ds_empty, 1);
+    mbar_init(&dq_full, 1); mbar_init(&dq_empty, 8);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -256,8 +258,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ row threads (one row each)
+    // ------------------------------------------------------------------ row threads (half a row each)
     const int quarter = warp & 3;
+    const int grp = (warp - 2) >> 2;  // this warpgroup's keys: grp * 64 .. grp * 64 + 63
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t ds_base = smem_u32(smem + C::OFF_DS);
@@ -277,22 +280,21 @@ __global__ void __launch_bounds__(NT, 1)
         if (!warp_wait(&s_full, ns & 1, limit, &abort_flag, p.st, 721)) { ok = false; break; }
         ++ns;
         tc_fence_after();
-        const int kvis = valid ? t - j * 128 : -1;  // keys 0..kvis of this tile are in the row
-        const bool masked = __any_sync(0xffffffffu, kvis < 127);
-        uint32_t pk[64];  // the row's dS, bf16 pairs
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        const int kvis = valid ? t - j * 128 - grp * 64 : -1;  // keys 0..kvis of this half are in the row
+        const bool masked = __any_sync(0xffffffffu, kvis < 63);
+        uint32_t pk[32];  // the row's dS over this half, bf16 pairs
+        {
           float sv[2][32], dv[2][32];
-          tmem_ld32(tmem + lane_base + tS + hh * 64, sv[0]);
-          tmem_ld32(tmem + lane_base + tS + hh * 64 + 32, sv[1]);
-          tmem_ld32(tmem + lane_base + tP + hh * 64, dv[0]);
-          tmem_ld32(tmem + lane_base + tP + hh * 64 + 32, dv[1]);
+          tmem_ld32(tmem + lane_base + tS + grp * 64, sv[0]);
+          tmem_ld32(tmem + lane_base + tS + grp * 64 + 32, sv[1]);
+          tmem_ld32(tmem + lane_base + tP + grp * 64, dv[0]);
+          tmem_ld32(tmem + lane_base + tP + grp * 64 + 32, dv[1]);
           tmem_ld_wait();
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2)
 #pragma unroll
             for (int x = 0; x < 32; x += 2) {
-              const int col = hh * 64 + c2 * 32 + x;
+              const int col = c2 * 32 + x;
               float e0, e1;
               ffma2(e0, e1, sv[c2][x], sv[c2][x + 1], c, c, nl2, nl2);
               float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
@@ -307,12 +309,11 @@ __global__ void __launch_bounds__(NT, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty);  // S and dP read: the next tile's may be issued
         if (!warp_wait(&ds_empty, (nds & 1) ^ 1, limit, &abort_flag, p.st, 722)) { ok = false; break; }
+        // keys grp * 64.. of the row: the dS tile's K-major block grp
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            st_shared_v4(ds_base + blk * (128 * 128) + sw128_off(row, q), pk[blk * 32 + 4 * q], pk[blk * 32 + 4 * q + 1],
-                         pk[blk * 32 + 4 * q + 2], pk[blk * 32 + 4 * q + 3]);
+        for (int q = 0; q < 8; ++q)
+          st_shared_v4(ds_base + grp * (128 * 128) + sw128_off(row, q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                       pk[4 * q + 3]);
         fence_async_smem();  // read by the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&ds_full);
@@ -322,7 +323,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (!warp_wait(&dq_full, nit & 1, limit, &abort_flag, p.st, 723)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int c3 = 0; c3 < D / 64; ++c3) {  // this warpgroup's half of the dQ row
+        const int cc = grp * (D / 64) + c3;
         float o[32];
         tmem_ld32(tmem + lane_base + tQ + cc * 32, o);
         tmem_ld_wait();
@@ -399,8 +401,8 @@ __global__ void __launch_bounds__(NT, 1)
   if (threadIdx.x == 0) {
     mbar_init(&kv_in_full, 1); mbar_init(&kv_in_empty, 1);
     for (int i = 0; i < C::RING; ++i) { mbar_init(&r_full[i], 1); mbar_init(&r_empty[i], 1); }
-    mbar_init(&s_full, 1); mbar_init(&ps_full, 4); mbar_init(&step_done, 1);
-    mbar_init(&kv_full, 1); mbar_init(&kv_empty, 4);
+    mbar_init(&s_full, 1); mbar_init(&ps_full, 8); mbar_init(&step_done, 1);
+    mbar_init(&kv_full, 1); mbar_init(&kv_empty, 8);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -496,8 +498,11 @@ __global__ void __launch_bounds__(NT, 1)
           const uint64_t dmn = sdesc(daddr, 128 * 128, 1024), qmn = sdesc(qaddr, 128 * 128, 1024);
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
-            umma_ts(tmem + tV, tmem + tS + kk * 8, sdesc_at(dmn, kk * 2048), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
-            umma_ts(tmem + tK, tmem + tP + kk * 8, sdesc_at(qmn, kk * 2048), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+            // rows 64 g .. 64 g + 63 of the tile (K steps 4 g .. 4 g + 3) were packed by warpgroup g
+            // into columns 64 g .. 64 g + 31 of the S^T / dP^T regions
+            const uint32_t acol = (kk / 4) * 64 + (kk % 4) * 8;
+            umma_ts(tmem + tV, tmem + tS + acol, sdesc_at(dmn, kk * 2048), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tmem + tK, tmem + tP + acol, sdesc_at(qmn, kk * 2048), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&r_empty[qs % C::RING]);
           umma_commit(&r_empty[ds % C::RING]);
@@ -512,8 +517,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ key threads (one key each)
+    // ------------------------------------------------------------------ key threads (half a key's columns each)
     const int quarter = warp & 3;
+    const int grp = (warp - 2) >> 2;  // this warpgroup's columns (rows of the tile): grp * 64 ..
     const int krow = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float c = p.c;
@@ -534,30 +540,27 @@ __global__ void __launch_bounds__(NT, 1)
         const float* dcol = &s_side[ri % C::RING][1][0];
         const int rbase = rt * 128;
         auto t_of = [&](int col) { return rbase + col < p.rows_per_batch ? p.off + (rbase + col) / H : -1; };
+        // 32 columns at a time: their P^T and dS^T packed two per column into the first half of
+        // this warpgroup's 64-column window (chunk c2 -> columns 16 c2 .., all already read)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float sv[2][32], dv[2][32];
-          tmem_ld32(tmem + lane_base + tS + hh * 64, sv[0]);
-          tmem_ld32(tmem + lane_base + tS + hh * 64 + 32, sv[1]);
-          tmem_ld32(tmem + lane_base + tP + hh * 64, dv[0]);
-          tmem_ld32(tmem + lane_base + tP + hh * 64 + 32, dv[1]);
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float sv[32], dv[32];
+          tmem_ld32(tmem + lane_base + tS + grp * 64 + c2 * 32, sv);
+          tmem_ld32(tmem + lane_base + tP + grp * 64 + c2 * 32, dv);
           tmem_ld_wait();
-          uint32_t pp[32], dd[32];
+          float pp[16], dd[16];  // bf16 pairs, as 32-bit patterns
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const int col = hh * 64 + c2 * 32 + x;
-              float e0, e1;
-              ffma2(e0, e1, sv[c2][x], sv[c2][x + 1], c, c, -l2c[col], -l2c[col + 1]);
-              const float p0 = kglob <= t_of(col) ? fast_exp2(e0) : 0.f;
-              const float p1 = kglob <= t_of(col + 1) ? fast_exp2(e1) : 0.f;
-              pp[(c2 * 32 + x) / 2] = pack_bf16x2(p0, p1);
-              dd[(c2 * 32 + x) / 2] = pack_bf16x2(p0 * (dv[c2][x] - dcol[col]), p1 * (dv[c2][x + 1] - dcol[col + 1]));
-            }
-          // columns hh*32.. of the packed operands: S^T / dP^T columns already read
-          tmem_st32(tmem + lane_base + tS + hh * 32, pp);
-          tmem_st32(tmem + lane_base + tP + hh * 32, dd);
+          for (int x = 0; x < 32; x += 2) {
+            const int col = grp * 64 + c2 * 32 + x;
+            float e0, e1;
+            ffma2(e0, e1, sv[x], sv[x + 1], c, c, -l2c[col], -l2c[col + 1]);
+            const float p0 = kglob <= t_of(col) ? fast_exp2(e0) : 0.f;
+            const float p1 = kglob <= t_of(col + 1) ? fast_exp2(e1) : 0.f;
+            pp[x / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+            dd[x / 2] = __uint_as_float(pack_bf16x2(p0 * (dv[x] - dcol[col]), p1 * (dv[x + 1] - dcol[col + 1])));
+          }
+          tmem_st16(tmem + lane_base + tS + grp * 64 + c2 * 16, pp);
+          tmem_st16(tmem + lane_base + tP + grp * 64 + c2 * 16, dd);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -571,7 +574,8 @@ __global__ void __launch_bounds__(NT, 1)
       float* dKr = p.dK + ((long long)w.b * p.Lk + kglob) * D;
       float* dVr = p.dV + ((long long)w.b * p.Lk + kglob) * D;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int c3 = 0; c3 < D / 64; ++c3) {  // this warpgroup's half of the key's dK, dV rows
+        const int cc = grp * (D / 64) + c3;
         float a[32], v[32];
         tmem_ld32(tmem + lane_base + tK + cc * 32, a);
         tmem_ld32(tmem + lane_base + tV + cc * 32, v);

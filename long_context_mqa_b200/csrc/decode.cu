@@ -803,6 +803,10 @@ __global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
             }
             la += v[0];
             lb += v[1];
+            if (p.blk_part) {  // the warp's 32-key sums per head (exact block scores of HySparse v1)
+              float* grp = p.blk_part + ((size_t)b * p.blk_groups + (size_t)lt * 4 + quarter) * H;
+              reinterpret_cast<float2*>(grp)[lane] = make_float2(v[0], v[1]);
+            }
           }
           const bool is_cand = valid && key < ncand;
           if (is_cand) p.sc[(size_t)b * p.sc_stride + key] = score;

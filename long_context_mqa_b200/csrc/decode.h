@@ -39,6 +39,8 @@ struct DecParams {
   int fallback;            // 0: the sampled schedule; 1: redo the flagged sequences with every tile
   const int32_t* ptab;     // paged cache: [B][max_pages] page of each 128-token tile (NULL: contiguous)
   int max_pages, n_pages;  // table width, pages in the K/V pools
+  float* blk_part;         // bf16 cache only, or NULL: [B][blk_groups][H] sums of p' over each group of
+  int blk_groups;          // 32 consecutive keys per head (HySparse v1 block scores); ceil(N / 32)
   DevStatus* st;
 };
 size_t fused_smem_bytes(int H, int D, bool f8);
@@ -92,23 +94,13 @@ struct BlkParams {
   int B, H, D, W;                // sequences, heads, head dim, window
   int NB, BLK, S;                // blocks chosen, tokens per block (64), idx row length NB * BLK + W
   dec::Sched sch;                // per-sequence lengths (query at t = seq_len - 1)
-  const float* sc;               // [B][ncand] the decode kernel's bounded scores score' of the older tokens
-  int ncand;
-  const float* lsum;             // [B][H] L'_h
-  const float* lse2x;            // [B][H] exact lse, log2 units
-  int max_blocks;                // ceil(N / BLK): the stride of cand and bsc
-  int* cnt;                      // [B] candidate blocks of each sequence
-  int* cand;                     // [B][max_blocks] candidate block ids
-  float* bsc;                    // [B][max_blocks] their exact block scores (S' of full blocks in between)
+  const float* blk_part;         // [B][blk_groups][H] the decode kernel's per-32-key sums of p'
+  int blk_groups;
+  const float* lsum;             // [B][H] L'_h (the exact p of a key is p' / L'_h)
+  int max_blocks;                // ceil(N / BLK): the stride of bsc
+  float* bsc;                    // [B][max_blocks] exact block scores
   int32_t* idx;                  // [B][S] output
   unsigned* gbar;                // the decode kernel's grid-barrier counters, re-armed here
-  // exact re-score
-  const __nv_bfloat16* qry;      // [B][H][D]
-  const __nv_bfloat16* kc;       // [B][N][D]
-  int N;
-  float c;                       // scale * log2(e)
-  int sms;
-  long long wait_ns;
   // decode output (the decode kernel's records / L')
   const float* opart;
   float oscale;

@@ -71,19 +71,32 @@ long long wait_limit_ns() {
   return g_wait_ns;
 }
 
+// Per-device attributes, queried once per device (every call needs them on the host)
+constexpr int kMaxDevices = 64;
+static std::atomic<int> g_sms[kMaxDevices];       // 0: not queried yet
+static std::atomic<int> g_is_sm100[kMaxDevices];  // 0: not queried yet, 1: yes, 2: no
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices && (n = g_sms[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices) g_sms[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 bool device_is_sm100() {
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int known = g_is_sm100[dev].load(std::memory_order_relaxed);
+    if (known) return known == 1;
+  }
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
-  return major == 10 && minor == 0;
+  const bool yes = major == 10 && minor == 0;
+  if (dev >= 0 && dev < kMaxDevices) g_is_sm100[dev].store(yes ? 1 : 2, std::memory_order_relaxed);
+  return yes;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -207,8 +220,11 @@ static DecodeWs carve_decode(void* ws, int B, const int* lens, int N, int H, int
   p.lse2x = c.take<float>((size_t)B * H);
   p.ovf = c.take<int>((size_t)B + 1);
   p.fallback = 0;
-  // phase 1 estimates each head's logsumexp from about 64 tiles (8k keys) per sequence
-  p.sample_tiles = 64;
+  // phase 1 estimates each head's logsumexp from a sample of each sequence's tiles: 64 tiles (8k
+  // keys) per sequence up to 8 sequences, then a budget of about 512 sampled tiles in all (at
+  // least 16 per sequence), so that phase 1 stays a few tiles per CTA for large batches of
+  // shorter caches (the estimate only sets how many keys the exact band re-score sees)
+  p.sample_tiles = B <= 8 ? 64 : (512 / B > 16 ? 512 / B : 16);
   p.sc_stride = stride;
   p.sc = c.take<float>((size_t)B * stride);
   p.hist = c.take<unsigned>((size_t)B * sel::NBINS);
@@ -337,11 +353,14 @@ size_t hs2_full_attn_select_workspace_bytes(int B, int Lq, int Lk, int H, int d,
 static hs2_status launch_decode_fused(DecodeWs& w, const void* Q, const void* K, const void* V, int B,
                                       const int* lens, int Lk, int H, int d, float c, int window, int topk,
                                       float* lse, void* workspace, size_t workspace_bytes, int sms, cudaStream_t st,
-                                      const int32_t* ptab, int max_pages, int n_pages, bool f8) {
+                                      const int32_t* ptab, int max_pages, int n_pages, bool f8,
+                                      float* blk_part = nullptr, int blk_groups = 0) {
   if (H != 64 || d != 128) return HS2_ERR_UNSUPPORTED_SHAPE;
   w = carve_decode(workspace, B, lens, Lk, H, d, window, topk, sms);
   if (!w.ok) return HS2_ERR_UNSUPPORTED_SHAPE;
   if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
+  w.p.blk_part = blk_part;
+  w.p.blk_groups = blk_groups;
   w.p.c = c;
   w.p.wait_ns = wait_limit_ns();
   w.p.lse_out = lse;
@@ -551,20 +570,19 @@ hs2_status hs2_sparse_attn_paged(const hs2_bf16* Q, const hs2_bf16* K_pages, con
 // ------------------------------------------------------------------------------------------
 struct V1Ws {
   size_t dec_bytes, bytes;
-  int max_blocks;
-  int* cnt;
-  int* cand;
+  int max_blocks, groups;
+  float* part;
   float* bsc;
 };
 
-// the decode workspace, then the candidate count, list and scores of the block selection
-static V1Ws carve_v1(void* ws, size_t dec_bytes, int B, int Lk, int block) {
+// the decode workspace, then the decode kernel's per-32-key head sums and the block scores
+static V1Ws carve_v1(void* ws, size_t dec_bytes, int B, int Lk, int H, int block) {
   V1Ws v{};
   v.dec_bytes = dec_bytes;
   v.max_blocks = (Lk + block - 1) / block;
+  v.groups = 4 * ((Lk + 127) / 128);  // every group of every (possibly partial) 128-key tile
   Carve c{(uint8_t*)ws, dec_bytes};
-  v.cnt = c.take<int>((size_t)B);
-  v.cand = c.take<int>((size_t)B * v.max_blocks);
+  v.part = c.take<float>((size_t)B * v.groups * H);
   v.bsc = c.take<float>((size_t)B * v.max_blocks);
   v.bytes = c.off;
   return v;
@@ -581,7 +599,7 @@ size_t hs2_full_attn_select_v1_workspace_bytes(int B, int Lk, int H, int d, int 
   std::vector<int> lens((size_t)B, Lk);
   const DecodeWs w = carve_decode(nullptr, B, lens.data(), Lk, H, d, window, n_blocks * block, sms);
   if (!w.ok) return 0;
-  return carve_v1(nullptr, w.bytes, B, Lk, block).bytes;
+  return carve_v1(nullptr, w.bytes, B, Lk, H, block).bytes;
 }
 
 hs2_status hs2_full_attn_select_v1(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V, int B, int Lk, int H,
@@ -603,25 +621,22 @@ hs2_status hs2_full_attn_select_v1(const hs2_bf16* Q, const hs2_bf16* K, const h
   DecodeWs w{};
   if (workspace_bytes < hs2_full_attn_select_v1_workspace_bytes(B, Lk, H, d, window, block, n_blocks))
     return HS2_ERR_WORKSPACE;
+  // the layout of the decode part first (for the offset of the v1 buffers after it)
+  const DecodeWs w0 = carve_decode(nullptr, B, lens.data(), Lk, H, d, window, n_blocks * block, sms);
+  const V1Ws v = carve_v1(workspace, w0.bytes, B, Lk, H, block);
   const hs2_status rc = launch_decode_fused(w, Q, K, V, B, lens.data(), Lk, H, d, c, window, n_blocks * block, lse,
-                                            workspace, workspace_bytes, sms, st, nullptr, 0, 0, false);
+                                            workspace, workspace_bytes, sms, st, nullptr, 0, 0, false, v.part,
+                                            v.groups);
   if (rc != HS2_OK) return rc;
-  const V1Ws v = carve_v1(workspace, w.bytes, B, Lk, block);
   blk::BlkParams bp{};
   bp.B = B; bp.H = H; bp.D = d; bp.W = window;
   bp.NB = n_blocks; bp.BLK = block; bp.S = n_blocks * block + window;
   bp.sch = w.p.sch;
-  bp.sc = w.p.sc; bp.ncand = w.p.sc_stride;
-  bp.lsum = w.p.lsum; bp.lse2x = w.p.lse2x;
-  bp.max_blocks = v.max_blocks; bp.cnt = v.cnt; bp.cand = v.cand; bp.bsc = v.bsc;
+  bp.blk_part = v.part; bp.blk_groups = v.groups;
+  bp.lsum = w.p.lsum;
+  bp.max_blocks = v.max_blocks; bp.bsc = v.bsc;
   bp.idx = idx;
   bp.gbar = w.p.gbar;
-  bp.qry = reinterpret_cast<const __nv_bfloat16*>(Q);
-  bp.kc = reinterpret_cast<const __nv_bfloat16*>(K);
-  bp.N = Lk;
-  bp.c = c;
-  bp.sms = sms;
-  bp.wait_ns = w.p.wait_ns;
   bp.opart = w.p.opart; bp.oscale = 1.f;
   bp.out = reinterpret_cast<__nv_bfloat16*>(out);
   bp.st = w.p.st;
@@ -674,10 +689,11 @@ struct BwdWs {
   size_t bytes;
 };
 
-// status block | D per (query, head) row | lse2 per row; both arrays padded by a 128-row tile (the
+// status block | D per (query, head) row | lse2 per row (both padded by a 128-row tile: the
 // key-side kernel copies a whole tile's values with its Q tile)
-static BwdWs carve_bwd(void* ws, long long rows) {
+static BwdWs carve_bwd(void* ws, int B, int Lq, int Lk, int H, int d) {
   BwdWs w{};
+  const long long rows = (long long)B * Lq * H;
   Carve c{(uint8_t*)ws, 0};
   w.st = c.take<DevStatus>(kStatusBytes / sizeof(DevStatus));
   w.Dv = c.take<float>((size_t)rows + 128);
@@ -688,7 +704,7 @@ static BwdWs carve_bwd(void* ws, long long rows) {
 
 size_t hs2_attn_bwd_workspace_bytes(int B, int Lq, int Lk, int H, int d) {
   if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || !shape_ok(H, d)) return 0;
-  return carve_bwd(nullptr, (long long)B * Lq * H).bytes;
+  return carve_bwd(nullptr, B, Lq, Lk, H, d).bytes;
 }
 
 static hs2_status bwd_args_ok(const void* Q, const void* K, const void* V, const void* out, const float* lse,
@@ -714,7 +730,7 @@ hs2_status hs2_full_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf1
   const hs2_status rc = bwd_args_ok(Q, K, V, out, lse, dO, dQ, dK, dV, B, Lq, Lk, H, d, scale, workspace);
   if (rc != HS2_OK) return rc;
   const long long rows = (long long)B * Lq * H;
-  const BwdWs w = carve_bwd(workspace, rows);
+  const BwdWs w = carve_bwd(workspace, B, Lq, Lk, H, d);
   if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms();
@@ -757,7 +773,7 @@ hs2_status hs2_sparse_attn_bwd(const hs2_bf16* Q, const hs2_bf16* K, const hs2_b
   if (!idx || (reinterpret_cast<uintptr_t>(idx) & 3u) != 0 || S <= 0) return HS2_ERR_INVALID_ARG;
   if (S > 4096) return HS2_ERR_UNSUPPORTED_SHAPE;
   const long long rows = (long long)B * Lq * H;
-  const BwdWs w = carve_bwd(workspace, rows);
+  const BwdWs w = carve_bwd(workspace, B, Lq, Lk, H, d);
   if (workspace_bytes < w.bytes) return HS2_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (bwd::launch_prep(reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(out), lse,
