@@ -135,9 +135,17 @@ def _workspace(nbytes: int, device: torch.device, key: str) -> torch.Tensor:
         return ws
 
 
-def _stream_ptr(stream) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream_ptr(stream, t: torch.Tensor | None = None) -> int:
+    """The cudaStream_t of `stream`, else of the current stream of t's device (read without
+    building a Stream object: this is on every call's path)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and t is not None:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _check(code: int, what: str):
@@ -146,14 +154,15 @@ def _check(code: int, what: str):
 
 
 def _need(t: torch.Tensor, name: str, dtype, dim: int):
+    if t.dtype is dtype and t.is_cuda and t.dim() == dim and t.is_contiguous():
+        return
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != dim:
         raise ValueError(f"{name} must have {dim} dims, got shape {tuple(t.shape)}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+    raise ValueError(f"{name} must be contiguous")
 
 
 def full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window=WINDOW, topk=TOPK) -> int:
@@ -189,11 +198,11 @@ def full_attn_select(q, k, v, *, scale=None, window=WINDOW, topk=TOPK, out=None,
     _need(out, "out", torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 3)
     _need(idx, "idx", torch.int32, 3)
-    nbytes = full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window, topk)
-    ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
+    ws = workspace if workspace is not None else _workspace(
+        full_attn_select_workspace_bytes(B, Lq, Lk, H, d, window, topk), q.device, "full")
     code = lib.hs2_full_attn_select(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Lq, Lk, H, d, scale, window, topk,
-                                    out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                    ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                    out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(), ws.nbytes,
+                                    _stream_ptr(stream, q))
     _check(code, "hs2_full_attn_select")
     return out, lse, idx
 
@@ -232,7 +241,7 @@ def full_attn_select_v1(q, k, v, *, scale=None, window=WINDOW, block=V1_BLOCK, n
     ws = _workspace(nbytes, q.device, "full_v1") if workspace is None else workspace
     code = lib.hs2_full_attn_select_v1(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Lk, H, d, scale, window, block,
                                        n_blocks, out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                       ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                       ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_select_v1")
     return out, lse, idx
 
@@ -257,7 +266,7 @@ def sparse_attn_v1(q, k, v, idx, gate, *, branch=V1_BLOCK * V1_BLOCKS, scale=Non
     ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
     code = lib.hs2_sparse_attn_v1(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), gate.data_ptr(), B, Lq,
                                   Lk, H, d, S, branch, scale, out.data_ptr(), ws.data_ptr(),
-                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                  ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_sparse_attn_v1")
     return out
 
@@ -298,7 +307,7 @@ def full_attn_bwd(q, k, v, out, lse, do, *, scale=None, dq=None, dk=None, dv=Non
     ws = _workspace(nbytes, q.device, "bwd") if workspace is None else workspace
     code = lib.hs2_full_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                  do.data_ptr(), B, Lq, Lk, H, d, scale, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                 ws.data_ptr(), ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                 ws.data_ptr(), ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_bwd")
     return dq, dk, dv
 
@@ -367,7 +376,7 @@ def full_attn_select_ragged(q, k, v, lens, *, scale=None, window=WINDOW, topk=TO
     ws = _workspace(nbytes, q.device, "full") if workspace is None else workspace
     code = lib.hs2_full_attn_select_ragged(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, lens_c, Lk, H, d, scale, window,
                                            topk, out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                           ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                           ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_select_ragged")
     return out, lse, idx
 
@@ -405,7 +414,7 @@ def full_attn_select_paged(q, k_pages, v_pages, page_table, lens, *, scale=None,
     code = lib.hs2_full_attn_select_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), n_pages,
                                           page_table.data_ptr(), max_pages, B, lens_c, H, d, scale, window, topk,
                                           out.data_ptr(), lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                          ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                          ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_select_paged")
     return out, lse, idx
 
@@ -426,8 +435,8 @@ def sparse_attn_paged(q, k_pages, v_pages, page_table, idx, *, scale=None, out=N
     ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
     code = lib.hs2_sparse_attn_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), n_pages,
                                      page_table.data_ptr(), max_pages, idx.data_ptr(), B, Lq, H, d, S, scale,
-                                     out.data_ptr(), None, ws.data_ptr(), ws.numel() * ws.element_size(),
-                                     _stream_ptr(stream))
+                                     out.data_ptr(), None, ws.data_ptr(), ws.nbytes,
+                                     _stream_ptr(stream, ws))
     _check(code, "hs2_sparse_attn_paged")
     return out
 
@@ -482,7 +491,7 @@ def full_attn_select_fp8kv(q, k8, v8, k_scale, v_scale, *, lens=None, page_table
                                           lens_c, Lk, page_table.data_ptr() if page_table is not None else None,
                                           max_pages, n_pages, H, d, scale, window, topk, out.data_ptr(),
                                           lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                          ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                          ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_select_fp8kv")
     return out, lse, idx
 
@@ -508,7 +517,7 @@ def full_attn_select_prefill_fp8kv(q, k8, v8, k_scale, v_scale, *, scale=None, w
     code = lib.hs2_full_attn_select_prefill_fp8kv(q.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(k_scale),
                                                   float(v_scale), B, Lq, Lk, H, d, scale, window, topk, out.data_ptr(),
                                                   lse.data_ptr(), idx.data_ptr(), ws.data_ptr(),
-                                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                                  ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_full_attn_select_prefill_fp8kv")
     return out, lse, idx
 
@@ -537,7 +546,7 @@ def sparse_attn_fp8kv(q, k8, v8, k_scale, v_scale, idx, *, page_table=None, scal
                                      idx.data_ptr(), B, Lq, Lk, page_table.data_ptr() if page_table is not None else None,
                                      max_pages, n_pages, H, d, S, scale, out.data_ptr(),
                                      lse.data_ptr() if lse is not None else None, ws.data_ptr(),
-                                     ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                     ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_sparse_attn_fp8kv")
     return (out, lse) if lse is not None else out
 
@@ -565,11 +574,11 @@ def sparse_attn(q, k, v, idx, *, scale=None, out=None, lse=None, want_lse=False,
         lse = torch.empty((B, Lq, H), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32, 3)
-    nbytes = sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S)
-    ws = _workspace(nbytes, q.device, "sparse") if workspace is None else workspace
+    ws = workspace if workspace is not None else _workspace(
+        sparse_attn_workspace_bytes(B, Lq, Lk, H, d, S), q.device, "sparse")
     code = lib.hs2_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), B, Lq, Lk, H, d, S, scale,
                                out.data_ptr(), lse.data_ptr() if lse is not None else None, ws.data_ptr(),
-                               ws.numel() * ws.element_size(), _stream_ptr(stream))
+                               ws.nbytes, _stream_ptr(stream, q))
     _check(code, "hs2_sparse_attn")
     return (out, lse) if lse is not None else out
 
@@ -587,7 +596,7 @@ def bridge_kv_proj(h, w, *, out=None, workspace=None, stream=None):
     nbytes = bridge_kv_proj_workspace_bytes(T, hidden, n, d)
     ws = _workspace(nbytes, h.device, "bridge") if workspace is None else workspace
     code = lib.hs2_bridge_kv_proj(h.data_ptr(), T, hidden, w.data_ptr(), n, d, out.data_ptr(), ws.data_ptr(),
-                                  ws.numel() * ws.element_size(), _stream_ptr(stream))
+                                  ws.nbytes, _stream_ptr(stream, ws))
     _check(code, "hs2_bridge_kv_proj")
     return out
 
