@@ -31,6 +31,7 @@
 // Every wait is bounded and reports a timeout.
 #include "decode.h"
 #include "host_util.h"
+#include "pair_union.cuh"
 #include "tc.cuh"
 
 namespace hs2 {
@@ -849,6 +850,258 @@ __global__ void __launch_bounds__(128, 1) sparse_bwd_kernel(BwdParams p) {
 }
 
 // =============================================================================================
+// sparse layer backward, two adjacent query rows per CTA (64 heads): over the union of their
+// selections, with M = 128 MMAs (both rows' heads) and one add per key for both rows
+// =============================================================================================
+template <int D>
+struct PairCfg {
+  static constexpr int T_BYTES = 128 * D * 2;   // Q / dO of the two rows, or a gathered K / V tile
+  static constexpr int P_BYTES = 128 * 128 * 2;  // P, dS: K-major [128 rows x 128 keys]
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = T_BYTES;
+  static constexpr int OFF_P = 2 * T_BYTES;
+  static constexpr int OFF_DS = OFF_P + P_BYTES;
+  static constexpr int OFF_K = OFF_DS + P_BYTES;
+  static constexpr int OFF_V = OFF_K + T_BYTES;
+  static constexpr int OFF_UKEY = OFF_V + T_BYTES;           // int32 [PAIR_MAX]
+  static constexpr int OFF_UFLAG = OFF_UKEY + PAIR_MAX * 4;  // uint8 [PAIR_MAX]
+  static constexpr int SMEM = 1024 + OFF_UFLAG + PAIR_MAX;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1) sparse_bwd_pair_kernel(BwdParams p) {
+  using C = PairCfg<D>;
+  constexpr int H = 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  int32_t* ukey = reinterpret_cast<int32_t*>(smem + C::OFF_UKEY);
+  uint8_t* uflag = smem + C::OFF_UFLAG;
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ float s_nl2[128], s_D[128];
+  __shared__ int s_warp[4], s_n[2];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // TMEM: S (later dV_sel), dP, dQ of the two rows, dK_sel
+  constexpr uint32_t tS = 0, tP = 128, tQ = 256, tK = 384;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (tid == 0) { mbar_init(&mma_bar, 1); fence_mbar_init(); }
+  if (warp == 0) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const float c = p.c;
+  const int pairs_per_b = (p.Lq + 1) / 2;
+  const int n_pairs = p.B * pairs_per_b;
+  uint32_t phase = 0;
+  bool ok = true, bad = false;
+  auto mma_wait = [&](unsigned where) -> bool {
+    bool w_ok = true;
+    if (tid == 0) w_ok = mbar_wait(&mma_bar, phase, p.wait_ns);
+    phase ^= 1;
+    if (!__syncthreads_and(w_ok)) {
+      if (tid == 0) report_status(p.st, kStatusTimeout, where);
+      return false;
+    }
+    tc_fence_after();
+    return true;
+  };
+  for (int pr = blockIdx.x; pr < n_pairs && ok; pr += gridDim.x) {
+    const int b = pr / pairs_per_b;
+    const int i0 = 2 * (pr % pairs_per_b);
+    const bool two = i0 + 1 < p.Lq;
+    const int r0 = b * p.Lq + i0, r1 = r0 + 1;
+    const __nv_bfloat16* Kb = p.K + (size_t)b * p.Lk * D;
+    const __nv_bfloat16* Vb = p.V + (size_t)b * p.Lk * D;
+    // ---- Q and dO of both rows -> shared (K-major, 128B swizzle): row m = 64 * (row of the pair) + head
+    for (int cidx = tid; cidx < 128 * D / 8; cidx += 128) {
+      const int m = cidx / (D / 8), ch = cidx % (D / 8);
+      const uint32_t off = (ch / 8) * (128 * 128) + sw128_off(m, ch % 8);
+      const bool have = m < H || two;
+      const size_t src = ((size_t)(m < H ? r0 : r1) * H + (m & (H - 1))) * D + ch * 8;
+      if (have) {
+        cp_async_16(smem_u32(smem + C::OFF_Q) + off, p.Q + src, true);
+        cp_async_16(smem_u32(smem + C::OFF_DO) + off, p.dO + src, true);
+      } else {
+        st_shared_v4(smem_u32(smem + C::OFF_Q) + off, 0u, 0u, 0u, 0u);
+        st_shared_v4(smem_u32(smem + C::OFF_DO) + off, 0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
+    {
+      const int m = tid;  // 128 rows, one per thread
+      const bool have = m < H || two;
+      const size_t g = (size_t)(m < H ? r0 : r1) * H + (m & (H - 1));
+      s_nl2[m] = have ? -__ldg(p.lse2 + g) : 0.f;
+      s_D[m] = have ? __ldg(p.Dv + g) : 0.f;
+    }
+    // ---- the union of the two rows' selections. Lists that are strictly ascending with any -1
+    // slots at the tail (the full layer's output) are merged without duplicates (a key in both
+    // rows gets both bits); any other lists are concatenated (each slot once, as the forward
+    // counts them). Out-of-range keys are reported and left out.
+    // the two index lists, staged in the P buffer (free until the first tile's softmax), and their
+    // union into ukey / uflag
+    const int U = pair_union(p.idx, p.S, p.Lk, r0, two, reinterpret_cast<int32_t*>(smem + C::OFF_P), ukey, uflag,
+                             s_warp, s_n, bad);
+    const int ntiles = (U + 127) / 128;
+    cp_async_wait_all();
+    __syncthreads();
+    for (int t = 0; t < ntiles && ok; ++t) {
+      // ---- gather the tile's K and V rows (16 lanes per 256-byte row, the key by shuffle)
+      const int slot = t * 128 + tid;
+      const int j = slot < U ? ukey[slot] : -1;
+      const unsigned fl = slot < U ? uflag[slot] : 0u;
+      {
+        constexpr int LPR = D * 2 / 16, RPS = 32 / LPR;
+        const int sub = lane / LPR, ch = lane % LPR;
+        const uint32_t kd = smem_u32(smem + C::OFF_K), vd = smem_u32(smem + C::OFF_V);
+#pragma unroll
+        for (int it = 0; it < 32 / RPS; ++it) {
+          const int rr = it * RPS + sub;
+          const int kr = __shfl_sync(0xffffffffu, j, rr);
+          const uint32_t off = (ch / 8) * (128 * 128) + sw128_off(warp * 32 + rr, ch % 8);
+          const size_t src = (size_t)(kr >= 0 ? kr : 0) * D + ch * 8;
+          cp_async_16(kd + off, Kb + src, kr >= 0);
+          cp_async_16(vd + off, Vb + src, kr >= 0);
+        }
+        cp_async_commit();
+      }
+      // the tile's membership bits per key, for every row thread: keys 32 q .. of row q's warp
+      __shared__ unsigned s_m0[4], s_m1[4];
+      {
+        const unsigned b0 = __ballot_sync(0xffffffffu, (fl & 1u) != 0), b1 = __ballot_sync(0xffffffffu, (fl & 2u) != 0);
+        if (lane == 0) { s_m0[warp] = b0; s_m1[warp] = b1; }
+      }
+      cp_async_wait_all();
+      fence_async_smem();
+      __syncthreads();
+      // ---- S = Q K_sel^T, dP = dO V_sel^T (M = 128 rows: both rows' heads, N = 128 keys)
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t IDESC = idesc_bf16(128, 128, 0, 0);
+        const uint64_t qa = sdesc(smem_u32(smem + C::OFF_Q), 16, 1024), da = sdesc(smem_u32(smem + C::OFF_DO), 16, 1024);
+        const uint64_t ka = sdesc(smem_u32(smem + C::OFF_K), 16, 1024), va = sdesc(smem_u32(smem + C::OFF_V), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+          umma_ss(tmem + tS, sdesc_at(qa, o), sdesc_at(ka, o), IDESC, kk > 0);
+          umma_ss(tmem + tP, sdesc_at(da, o), sdesc_at(va, o), IDESC, kk > 0);
+        }
+        umma_commit(&mma_bar);
+      }
+      if (!mma_wait(811)) { ok = false; break; }
+      // ---- P and dS rows (bf16, K-major [128 rows x 128 keys]); thread tid owns row tid
+      {
+        const int m = tid;
+        const bool row1 = m >= H;
+        const float nl2 = s_nl2[m], Dr = s_D[m];
+        const uint32_t pb = smem_u32(smem + C::OFF_P), db = smem_u32(smem + C::OFF_DS);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {  // keys 32 cc .. 32 cc + 31
+          float sv[32], dv[32];
+          tmem_ld32(tmem + lane_base + tS + cc * 32, sv);
+          tmem_ld32(tmem + lane_base + tP + cc * 32, dv);
+          tmem_ld_wait();
+          const unsigned mk = (row1 ? s_m1[cc] : s_m0[cc]);
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            float e0, e1;
+            ffma2(e0, e1, sv[x], sv[x + 1], c, c, nl2, nl2);
+            const float p0 = (mk >> x) & 1u ? fast_exp2(e0) : 0.f;
+            const float p1 = (mk >> (x + 1)) & 1u ? fast_exp2(e1) : 0.f;
+            pp[x / 2] = pack_bf16x2(p0, p1);
+            dd[x / 2] = pack_bf16x2(p0 * (dv[x] - Dr), p1 * (dv[x + 1] - Dr));
+          }
+          // keys 32 cc .. in block cc / 2 (64 keys = one 128-byte row), chunks 4 (cc % 2) ..
+          const uint32_t o = (cc / 2) * (128 * 128);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            st_shared_v4(pb + o + sw128_off(m, (cc % 2) * 4 + q), pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+            st_shared_v4(db + o + sw128_off(m, (cc % 2) * 4 + q), dd[4 * q], dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      // ---- dQ += dS K_sel; dK_sel = dS^T Q, dV_sel = P^T dO (M = 128 keys, K = 128 rows)
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t IDESC_Q = idesc_bf16(128, D, 0, 1);
+        constexpr uint32_t IDESC_KV = idesc_bf16(128, D, 1, 1);
+        const uint64_t dsk = sdesc(smem_u32(smem + C::OFF_DS), 16, 1024);
+        const uint64_t kmn = sdesc(smem_u32(smem + C::OFF_K), 128 * 128, 1024);
+        const uint64_t dsm = sdesc(smem_u32(smem + C::OFF_DS), 128 * 128, 1024);
+        const uint64_t pm = sdesc(smem_u32(smem + C::OFF_P), 128 * 128, 1024);
+        const uint64_t qm = sdesc(smem_u32(smem + C::OFF_Q), 128 * 128, 1024);
+        const uint64_t dom = sdesc(smem_u32(smem + C::OFF_DO), 128 * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          umma_ss(tmem + tQ, sdesc_at(dsk, (kk / 4) * (128 * 128) + (kk % 4) * 32), sdesc_at(kmn, kk * 2048), IDESC_Q,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tmem + tK, sdesc_at(dsm, kk * 2048), sdesc_at(qm, kk * 2048), IDESC_KV, kk > 0);
+          umma_ss(tmem + tS, sdesc_at(pm, kk * 2048), sdesc_at(dom, kk * 2048), IDESC_KV, kk > 0);
+        }
+        umma_commit(&mma_bar);
+      }
+      if (!mma_wait(812)) { ok = false; break; }
+      // ---- scatter: thread tid owns key row tid of the tile; every lane runs the TMEM loads
+      {
+        float* dKr = p.dK + ((size_t)b * p.Lk + (j >= 0 ? j : 0)) * D;
+        float* dVr = p.dV + ((size_t)b * p.Lk + (j >= 0 ? j : 0)) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float a[32], v[32];
+          tmem_ld32(tmem + lane_base + tK + cc * 32, a);
+          tmem_ld32(tmem + lane_base + tS + cc * 32, v);
+          tmem_ld_wait();
+          if (j >= 0) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+              red_add_v4(dKr + cc * 32 + x, a[x] * p.scale, a[x + 1] * p.scale, a[x + 2] * p.scale, a[x + 3] * p.scale);
+              red_add_v4(dVr + cc * 32 + x, v[x], v[x + 1], v[x + 2], v[x + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();  // TMEM S / dK_sel and the shared tiles are reused by the next tile
+    }
+    if (!ok) break;
+    // ---- dQ rows: thread tid owns row tid (row tid / 64 of the pair, head tid % 64)
+    {
+      const int m = tid;
+      const bool have = m < H || two;
+      const size_t g = (size_t)(m < H ? r0 : r1) * H + (m & (H - 1));
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + tQ + cc * 32, o);
+        tmem_ld_wait();
+        if (have && ntiles > 0) {
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) w[x] = pack_bf16x2(o[2 * x] * p.scale, o[2 * x + 1] * p.scale);
+          uint4* dst = reinterpret_cast<uint4*>(p.dQ + g * D + cc * 32);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // the next pair's first dQ MMA overwrites the accumulator
+  }
+  cp_async_wait_all();
+  if (__syncthreads_or(bad) && tid == 0) report_status(p.st, kStatusBounds, 813);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+// =============================================================================================
 // launchers
 // =============================================================================================
 cudaError_t launch_prep(const __nv_bfloat16* dO, const __nv_bfloat16* out, const float* lse, float* Dv, float* lse2,
@@ -912,6 +1165,20 @@ static cudaError_t launch_sparse_t(const BwdParams& p, int sms, cudaStream_t str
 }
 
 cudaError_t launch_sparse_bwd(const BwdParams& p, int sms, cudaStream_t stream) {
+  if (p.H == 64 && p.D == 128 && p.Lq >= 2 && p.S <= PAIR_MAX / 2) {
+    // two adjacent rows per CTA over the union of their selections
+    static bool configured = false;
+    if (!configured) {
+      cudaFuncSetAttribute(sparse_bwd_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<128>::SMEM);
+      configured = true;
+    }
+    const int pairs = p.B * ((p.Lq + 1) / 2);
+    LaunchScope ls("sparse_bwd", stream);
+    const cudaError_t e = launch_k(sparse_bwd_pair_kernel<128>, dim3(pairs < sms ? pairs : sms), dim3(128),
+                                   PairCfg<128>::SMEM, stream, true, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (p.H == 64 && p.D == 128) return launch_sparse_t<64, 128>(p, sms, stream);
   if (p.H == 16 && p.D == 64) return launch_sparse_t<16, 64>(p, sms, stream);
   return cudaErrorInvalidValue;

@@ -130,6 +130,34 @@ def test_sparse_backward_random_indices(hs2, name, B, Lq, Lk, S):
     assert_grad_close(dv.double().cpu().numpy(), ref["dv"], "sparse dV")
 
 
+def test_sparse_backward_unsorted_indices_with_repeats(hs2):
+    """Index rows in no particular order, -1 slots anywhere and a key repeated within a row (each
+    slot counts once, as in the forward): the paired kernel then concatenates the two rows' lists
+    instead of merging them, and must still match the oracle."""
+    rng = np.random.default_rng(77)
+    B, Lq, Lk, S = 1, 9, 2000, 400
+    g = synth.SyntheticInputs(synth.small("prefill_32k", B=B, Lq=Lq, Lk=Lk))
+    wl = g.wl
+    idx = np.full((B, Lq, S), -1, np.int32)
+    for i in range(Lq):
+        n = int(rng.integers(50, S))
+        sel = rng.choice(Lk, size=n, replace=False).astype(np.int32)
+        sel[: n // 10] = sel[n // 10: 2 * (n // 10)]  # repeats
+        slots = rng.choice(S, size=n, replace=False)   # -1 slots scattered among the keys
+        idx[0, i, slots] = sel
+    qs = g.q_sparse(0)
+    q, k, v = to_torch_bf16(qs), to_torch_bf16(g.k), to_torch_bf16(g.v)
+    idx_t = torch.from_numpy(idx).cuda()
+    out, lse = hs2.sparse_attn(q, k, v, idx_t, scale=wl.scale, want_lse=True)
+    do_bits = g.grad_out(1)
+    dq, dk, dv = hs2.sparse_attn_bwd(q, k, v, idx_t, out, lse, to_torch_bf16(do_bits), scale=wl.scale)
+    torch.cuda.synchronize()
+    ref = oracle.attn_bwd(qs, g.k, g.v, do_bits, wl.scale, idx=idx)
+    assert_grad_close(bf16_to_f64(dq).reshape(ref["dq"].shape), ref["dq"], "sparse dQ (unsorted)")
+    assert_grad_close(dk.double().cpu().numpy(), ref["dk"], "sparse dK (unsorted)")
+    assert_grad_close(dv.double().cpu().numpy(), ref["dv"], "sparse dV (unsorted)")
+
+
 def test_block_backward_accumulates_kv_gradients(hs2):
     """A hybrid block: the full layer's selection, then a sparse layer with its own Q over the same
     K, V and indices. The two backward calls add into one pair of dK, dV buffers (KV Reuse), which
