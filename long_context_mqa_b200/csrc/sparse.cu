@@ -210,24 +210,15 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     phase ^= 1;
     if (!ok) break;
     tc_fence_after();
-    // ---- the row's 128 logits (warp-collective loads, one wait). Lanes 0..15 hold the head
-    // rows; lane l + 16 takes keys 64..127 of lane l's row (by shuffle), lane l keeps keys 0..63,
-    // so every lane exponentiates 64 keys. Both lanes of a pair keep the same running max.
+    // ---- the row's 128 logits (warp-collective loads, one wait). The head rows sit in the first
+    // 16 lanes of each quarter; lane l reads keys 0..63 of row l and lane l + 16 keys 64..127 of
+    // the same row, so every lane exponentiates 64 keys. Both lanes of a pair keep the same
+    // running max.
     const bool upper = lane >= 16;
     float sv[2][32];
-    {
-      float s4[4][32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + tS + cc * 32, s4[cc]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float hi = __shfl_xor_sync(0xffffffffu, s4[2 + h2][x], 16);
-          sv[h2][x] = upper ? hi : s4[h2][x];
-        }
-    }
+    tmem_ld16x2_32<64>(tmem + lane_base + tS, sv[0]);       // keys 0..31 | 64..95
+    tmem_ld16x2_32<64>(tmem + lane_base + tS + 32, sv[1]);  // keys 32..63 | 96..127
+    tmem_ld_wait();
     float rmax = -INFINITY;
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
@@ -311,19 +302,22 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   // ---- epilogue
   const bool have = ntiles > 0 && ok;  // block-uniform
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);  // the row's sum: both halves
+  // lane l < 16 holds columns 32 i .. 32 i + 31 of head row prow, lane l + 16 the same columns
+  // shifted by D / 2 (i < D / 64)
+  const int cbase = lane >= 16 ? D / 2 : 0;
   if (p.nsplit == 1) {
     if (have) {
+      const float inv = l_run > 0.f ? p.oscale / l_run : 0.f;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int i = 0; i < D / 64; ++i) {
         float o[32];
-        tmem_ld32(tmem + lane_base + tO + cc * 32, o);
+        tmem_ld16x2_32<D / 2>(tmem + lane_base + tO + i * 32, o);
         tmem_ld_wait();
-        if (owns) {
-          const float inv = l_run > 0.f ? p.oscale / l_run : 0.f;
+        if (prow < H) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(o[2 * x] * inv, o[2 * x + 1] * inv);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)r * H + head) * D + cc * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)r * H + prow) * D + cbase + i * 32);
 #pragma unroll
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
         }
@@ -345,27 +339,28 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   float* xm = xO + (size_t)n * HPR * D;
   float* xl = xm + n * MH;
   {
-    // this CTA's O rows (unnormalised), one TMEM wait, while the cluster barrier completes
-    float o[D / 32][32];
+    // this CTA's O rows (unnormalised; both lanes of a pair hold half a row), one TMEM wait,
+    // while the cluster barrier completes
+    float o[D / 64][32];
     if (have) {
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_base + tO + cc * 32, o[cc]);
+      for (int i = 0; i < D / 64; ++i) tmem_ld16x2_32<D / 2>(tmem + lane_base + tO + i * 32, o[i]);
       tmem_ld_wait();
     } else {
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc)
+      for (int i = 0; i < D / 64; ++i)
 #pragma unroll
-        for (int x = 0; x < 32; ++x) o[cc][x] = 0.f;
+        for (int x = 0; x < 32; ++x) o[i][x] = 0.f;
     }
     cluster_wait();  // every CTA of the cluster has started: its shared memory can be written
-    const int owner = head % n, k = head / n;
-    const uint32_t o_dst = dsmem_addr(smem_u32(xO + ((size_t)split * HPR + k) * D), owner);
-    if (owns) {
+    const int owner = prow % n, k = prow / n;
+    if (prow < H) {
+      const uint32_t o_dst = dsmem_addr(smem_u32(xO + ((size_t)split * HPR + k) * D + cbase), owner);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc)
+      for (int i = 0; i < D / 64; ++i)
 #pragma unroll
         for (int x = 0; x < 8; ++x)
-          st_dsmem_v4(o_dst + (cc * 32 + 4 * x) * 4, o[cc][4 * x], o[cc][4 * x + 1], o[cc][4 * x + 2], o[cc][4 * x + 3]);
+          st_dsmem_v4(o_dst + (i * 32 + 4 * x) * 4, o[i][4 * x], o[i][4 * x + 1], o[i][4 * x + 2], o[i][4 * x + 3]);
     }
     if (owns) {
       const float mv = l_run > 0.f && have ? m_run : -INFINITY, lv = have ? l_run : 0.f;
@@ -379,43 +374,53 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   __syncthreads();
   if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 256); }
   cluster_sync_all();  // all partials have landed; nothing reads another CTA's memory after this
-  // merge weights of this rank's heads (thread k < HPR: head rank + k*n)
-  if (tid < HPR && !p.gate) {
-    const int h = (int)rank + tid * n;
-    if (h < H) {
-      float M = -INFINITY, L = 0.f;
-      for (int s2 = 0; s2 < n; ++s2)
-        if (xl[s2 * MH + h] > 0.f) M = fmaxf(M, xm[s2 * MH + h]);
-      for (int s2 = 0; s2 < n; ++s2) {
-        const float l = xl[s2 * MH + h];
-        const float w = l > 0.f ? exp2f(xm[s2 * MH + h] - M) : 0.f;
-        wgt[s2 * MH + tid] = w;
-        L += l * w;
+  // merge weights of this rank's heads: a group of 16 lanes per head (lane s = split s), the
+  // max and the sum by shuffles within the group; every lane of a warp takes the same number
+  // of steps, so the shuffles are warp-uniform
+  {
+    const int s = tid & 15;
+    for (int k0 = 0; k0 < HPR; k0 += NT / 16) {
+      const int k = k0 + (tid >> 4);
+      const int h = (int)rank + k * n;
+      const bool hv = k < HPR && h < H;
+      const bool on = hv && s < n;
+      const float lx = on ? xl[s * MH + h] : 0.f;
+      const float mx = lx > 0.f ? xm[s * MH + h] : -INFINITY;
+      if (!p.gate) {
+        float M = mx;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = lx > 0.f ? exp2f(mx - M) : 0.f;
+        float L = lx * w;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (on) wgt[s * MH + k] = w;
+        if (hv && s == 0) {
+          wgt[16 * MH + k] = L > 0.f ? p.oscale / L : 0.f;
+          if (p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
+        }
+      } else {
+        // two branches, each its own softmax (splits below branch_split: the blocks; the rest:
+        // the window), mixed by the gate: the weights carry each branch's normalisation and share
+        const bool br = s >= p.branch_split;
+        float M0 = br ? -INFINITY : mx, M1 = br ? mx : -INFINITY;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          M0 = fmaxf(M0, __shfl_xor_sync(0xffffffffu, M0, o));
+          M1 = fmaxf(M1, __shfl_xor_sync(0xffffffffu, M1, o));
+        }
+        const float w = lx > 0.f ? exp2f(mx - (br ? M1 : M0)) : 0.f;
+        float L0 = br ? 0.f : lx * w, L1 = br ? lx * w : 0.f;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          L0 += __shfl_xor_sync(0xffffffffu, L0, o);
+          L1 += __shfl_xor_sync(0xffffffffu, L1, o);
+        }
+        const float g = hv ? p.gate[(size_t)r * H + h] : 0.f;
+        const float f0 = L0 > 0.f ? g / L0 : 0.f, f1 = L1 > 0.f ? (1.f - g) / L1 : 0.f;
+        if (on) wgt[s * MH + k] = w * (br ? f1 : f0);
+        if (hv && s == 0) wgt[16 * MH + k] = p.oscale;
       }
-      wgt[16 * MH + tid] = L > 0.f ? p.oscale / L : 0.f;
-      if (p.lse) p.lse[(size_t)r * H + h] = (M + log2f(L)) * 0.69314718055994531f;
-    }
-  } else if (tid < HPR) {
-    // two branches, each its own softmax (splits below branch_split: the blocks; the rest: the
-    // window), mixed by the gate: the weights carry each branch's normalisation and its share
-    const int h = (int)rank + tid * n;
-    if (h < H) {
-      const float g = p.gate[(size_t)r * H + h];
-      float M[2] = {-INFINITY, -INFINITY}, L[2] = {0.f, 0.f};
-      for (int s2 = 0; s2 < n; ++s2) {
-        const int br = s2 < p.branch_split ? 0 : 1;
-        if (xl[s2 * MH + h] > 0.f) M[br] = fmaxf(M[br], xm[s2 * MH + h]);
-      }
-      for (int s2 = 0; s2 < n; ++s2) {
-        const int br = s2 < p.branch_split ? 0 : 1;
-        const float l = xl[s2 * MH + h];
-        const float w = l > 0.f ? exp2f(xm[s2 * MH + h] - M[br]) : 0.f;
-        wgt[s2 * MH + tid] = w;
-        L[br] += l * w;
-      }
-      const float f0 = L[0] > 0.f ? g / L[0] : 0.f, f1 = L[1] > 0.f ? (1.f - g) / L[1] : 0.f;
-      for (int s2 = 0; s2 < n; ++s2) wgt[s2 * MH + tid] *= s2 < p.branch_split ? f0 : f1;
-      wgt[16 * MH + tid] = p.oscale;
     }
   }
   __syncthreads();
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     const int h = (int)rank + k * n;
     if (h >= H) continue;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int s2 = 0; s2 < n; ++s2) {
       const float w = wgt[s2 * MH + k];
       const float4 v4 = reinterpret_cast<const float4*>(xO + ((size_t)s2 * HPR + k) * D)[d4];
@@ -437,6 +443,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     reinterpret_cast<uint2*>(p.out + ((size_t)r * H + h) * D)[d4] = o2;
   }
 }
+
 
 size_t sparse_smem_bytes(int H, int D, int nsplit) {
   if (H == 64 && D == 128) return SpLayout<64, 128>::bytes(nsplit);
