@@ -34,6 +34,8 @@ namespace hs2 {
 namespace prefill {
 
 constexpr int NT = 320;
+constexpr int SC_WG = 4;                 // score pass: softmax warpgroups
+constexpr int NT_SC = 64 + 128 * SC_WG;  // score pass: + the producer and issuer warps
 constexpr float LOG2E = 1.4426950408889634f;
 // Of every 16 score-pass exponentials, how many exp2_fma2 computes on the FMA pipes instead of
 // the MUFU. Measured on B200 at L = 32k: 0 and 6 take the same time (the loop is not MUFU-bound),
@@ -376,7 +378,8 @@ __global__ void __launch_bounds__(NT, 1)
 template <int H, int D>
 struct ScCfg {
   static constexpr int NQ = 256 / H;        // queries per item
-  static constexpr int QW = NQ / 2;         // queries per warpgroup
+  static constexpr int QW = NQ / SC_WG;     // queries per warpgroup
+  static constexpr int CW = 256 / SC_WG;    // S columns per warpgroup (QW queries x H heads)
   static constexpr int CAP = H == 64 ? 1920 : 1152;  // candidate slots per query
   static constexpr int Q_BYTES = 256 * D * 2;
   static constexpr int KT_BYTES = 128 * D * 2;
@@ -407,8 +410,8 @@ template <int CAP>
 __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int keep, int wg, int wt, unsigned* hist,
                                          unsigned long long* s_prefix, int* s_need, int* s_cnt) {
   // bits on which all n keys agree need no radix pass: find the highest differing bit first
-  __shared__ unsigned long long s_and[2], s_or[2];
-  __shared__ int s_exact[2];
+  __shared__ unsigned long long s_and[SC_WG], s_or[SC_WG];
+  __shared__ int s_exact[SC_WG];
   if (wt == 0) { s_and[wg] = ~0ull; s_or[wg] = 0ull; *s_need = keep; *s_cnt = 0; s_exact[wg] = 0; }
   wg_bar(wg);
   {
@@ -492,7 +495,7 @@ __device__ unsigned long long wg_compact(unsigned long long* buf, int n, int kee
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT_SC, 1)
     score_select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, PfParams p) {
   using C = ScCfg<H, D>;
   extern __shared__ uint8_t smem_raw[];
@@ -504,10 +507,10 @@ __global__ void __launch_bounds__(NT, 1)
   __shared__ __align__(16) float slse2[256];
   __shared__ int cnt[C::NQ];
   __shared__ unsigned long long theta[C::NQ];
-  __shared__ unsigned hist[2][256];
-  __shared__ unsigned long long s_prefix[2];
-  __shared__ int s_need[2], s_cnt[2];
-  __shared__ unsigned s_wsum[2][4];  // per-warp totals of the final ordered write
+  __shared__ unsigned hist[SC_WG][256];
+  __shared__ unsigned long long s_prefix[SC_WG];
+  __shared__ int s_need[SC_WG], s_cnt[SC_WG];
+  __shared__ unsigned s_wsum[SC_WG][4];  // per-warp totals of the final ordered write
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const long long limit = p.wait_ns;
 
@@ -515,7 +518,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(&q_full, 1);
     mbar_init(&q_empty, 1);
     for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4 * SC_WG); }
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -615,18 +618,17 @@ __global__ void __launch_bounds__(NT, 1)
         if (ok) {
         tc_fence_after();
         const int key = j * 128 + row;
-        // this warpgroup's 128 columns (QW queries x H heads) in one go: the TMEM load latency
+        // this warpgroup's 64 columns (QW queries x H heads) in one go: the TMEM load latency
         // is paid once per tile, not once per 16 columns
-        float v0[32], v1[32], v2[32], v3[32];
-        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128, v0);
-        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 32, v1);
-        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 64, v2);
-        tmem_ld32(tmem + lane_base + buf * 256 + wg * 128 + 96, v3);
+        static_assert(C::CW == 64, "two 32-column loads per tile");
+        float v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * C::CW, v0);
+        tmem_ld32(tmem + lane_base + buf * 256 + wg * C::CW + 32, v1);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[buf]);  // the S buffer is free for the next tile
-        auto col = [&](int i) -> float { return i < 32 ? v0[i] : i < 64 ? v1[i - 32] : i < 96 ? v2[i - 64] : v3[i - 96]; };
+        auto col = [&](int i) -> float { return i < 32 ? v0[i] : v1[i - 32]; };
 #pragma unroll
         for (int qq = 0; qq < C::QW; ++qq) {
           const int q = wg * C::QW + qq;
@@ -821,7 +823,7 @@ static hs2_status run_t(const hs2_bf16* Q, const hs2_bf16* K, const hs2_bf16* V,
   }
   {
     LaunchScope ls("score_select", stream);
-    score_select_kernel<H, D><<<grid, NT, SC::SMEM, stream>>>(tmQ2, tmK, p);
+    score_select_kernel<H, D><<<grid, NT_SC, SC::SMEM, stream>>>(tmQ2, tmK, p);
   }
   return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
