@@ -879,7 +879,7 @@ __global__ void __launch_bounds__(128, 1) sparse_bwd_pair_kernel(BwdParams p) {
   __shared__ __align__(8) uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ float s_nl2[128], s_D[128];
-  __shared__ int s_warp[4], s_n[2];
+  __shared__ int s_warp[4], s_n[8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // TMEM: S (later dV_sel), dP, dQ of the two rows, dK_sel
   constexpr uint32_t tS = 0, tP = 128, tQ = 256, tK = 384;

@@ -184,11 +184,19 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
   tc_fence_after();
   const uint32_t tmem = tmem_base;
 
+  bool any_pv = false;  // a PV has written O (block-uniform)
   for (int t = 0; t < ntiles && ok; ++t) {
     cp_async_wait_all();
     fence_async_smem();
     __syncthreads();
     const bool all_valid = (vmask[0] & vmask[1] & vmask[2] & vmask[3]) == 0xFFFFFFFFu;
+    if ((vmask[0] | vmask[1] | vmask[2] | vmask[3]) == 0u) {
+      // no valid slot in the tile (a list's -1 tail): nothing to add. Every thread has read the
+      // masks before the next gather rewrites them.
+      __syncthreads();
+      if (t + 1 < ntiles) gather(t + 1);
+      continue;
+    }
     // ---- S = Q K^T
     if (tid == 0) {
       tc_fence_after();
@@ -235,7 +243,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     const float alpha = raise ? (m_run == -INFINITY ? 0.f : fast_exp2(m_run - mt)) : 1.f;
     if (raise) m_run = mt;
     l_run *= alpha;
-    if (t > 0 && __any_sync(0xffffffffu, raise)) {  // O row *= alpha (warp-collective)
+    if (any_pv && __any_sync(0xffffffffu, raise)) {  // O row *= alpha (warp-collective)
 #pragma unroll
       for (int cc = 0; cc < D / 16; ++cc) {
         float o[16];
@@ -284,7 +292,7 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
       for (int kk = 0; kk < TILE / 16; ++kk) {
         const uint64_t a = sdesc_at(pa, (kk / 4) * (MH * 128) + (kk % 4) * 32);
         const uint64_t bv = sdesc_at(va, kk * 2048);
-        umma_ss(tmem + tO, a, bv, IDESC, (t == 0 && kk == 0) ? 0u : 1u);
+        umma_ss(tmem + tO, a, bv, IDESC, (!any_pv && kk == 0) ? 0u : 1u);
       }
       umma_commit(&mma_bar);
     }
@@ -295,12 +303,13 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
     }
     phase ^= 1;
     tc_fence_after();
+    any_pv = true;
     if (ok && t + 1 < ntiles) gather(t + 1);  // the single K/V stage is free again
   }
   cp_async_wait_all();
   if (__syncthreads_or(bad) && tid == 0) report_status(p.st, kStatusBounds, 403);
   // ---- epilogue
-  const bool have = ntiles > 0 && ok;  // block-uniform
+  const bool have = any_pv && ok;  // block-uniform
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);  // the row's sum: both halves
   // lane l < 16 holds columns 32 i .. 32 i + 31 of head row prow, lane l + 16 the same columns
   // shifted by D / 2 (i < D / 64)
@@ -322,6 +331,10 @@ __global__ void __launch_bounds__(NT, 2) sparse_attn_kernel(SpParams p) {
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
         }
       }
+    } else if (ok && prow < H) {  // the row selected nothing: zeros
+      uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)r * H + prow) * D + cbase);
+#pragma unroll
+      for (int x = 0; x < D / 16; ++x) dst[x] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (owns && p.lse) p.lse[(size_t)r * H + head] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     tc_fence_before();
