@@ -120,6 +120,26 @@ lib = _load_library()
 LIBRARY_PATH = _LIB_PATH
 ABI_VERSION = lib.hs2_abi_version()
 
+
+def _load_marshalling():
+    """The C++ module that checks torch tensors and calls hs2_full_attn_select / hs2_sparse_attn
+    (bind/hs2_torch.cpp; a few microseconds of host time per call instead of the ctypes path's
+    tens). None when it is not built, and the ctypes path below serves every call."""
+    import importlib.util
+    import sysconfig
+    path = os.path.join(_PKG, "_hs2_torch" + sysconfig.get_config_var("EXT_SUFFIX"))
+    if not os.path.exists(path):
+        return None
+    spec = importlib.util.spec_from_file_location(__name__ + "._hs2_torch", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    addr = lambda f: ctypes.cast(f, ctypes.c_void_p).value
+    mod.set_entries(addr(lib.hs2_full_attn_select), addr(lib.hs2_sparse_attn))
+    return mod
+
+
+_fast = _load_marshalling()
+
 _ws_lock = threading.Lock()
 _ws_cache: dict = {}
 
@@ -183,6 +203,13 @@ def full_attn_select(q, k, v, *, scale=None, window=WINDOW, topk=TOPK, out=None,
 
     Returns (out [B,Lq,H,d] bf16, lse [B,Lq,H] fp32 natural log, idx [B,Lq,window+topk] int32).
     """
+    if _fast is not None and out is not None and lse is not None and idx is not None and workspace is not None:
+        # every buffer given (a decode loop): checks and call in C++
+        sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+        st = _stream_ptr(stream, q) if q.is_cuda else 0  # (a host tensor fails the checks in C++)
+        _check(_fast.full_attn_select(q, k, v, sc, window, topk, out, lse, idx, workspace, st),
+               "hs2_full_attn_select")
+        return out, lse, idx
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 3)
     _need(v, "v", torch.bfloat16, 3)
@@ -556,6 +583,12 @@ def sparse_attn(q, k, v, idx, *, scale=None, out=None, lse=None, want_lse=False,
 
     Returns out [B,Lq,H,d] bf16, or (out, lse) when want_lse or lse is given.
     """
+    if _fast is not None and out is not None and workspace is not None and (lse is not None or not want_lse):
+        # every buffer given (a decode loop): checks and call in C++
+        sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+        st = _stream_ptr(stream, q) if q.is_cuda else 0  # (a host tensor fails the checks in C++)
+        _check(_fast.sparse_attn(q, k, v, idx, sc, out, lse, workspace, st), "hs2_sparse_attn")
+        return (out, lse) if lse is not None else out
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 3)
     _need(v, "v", torch.bfloat16, 3)

@@ -1,5 +1,6 @@
 """Builds long_context_mqa_b200/libhs2.so (the C-ABI library) from csrc/*.cu with nvcc for
-sm_100a. Objects go to long_context_mqa_b200/_build/; the .so is written in-tree.
+sm_100a, and the torch argument-marshalling module _hs2_torch*.so from bind/hs2_torch.cpp. Objects
+go to long_context_mqa_b200/_build/; the .so files are written in-tree.
 
     python long_context_mqa_b200/_build.py [--force] [-v]
 """
@@ -78,6 +79,36 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+BIND_SRC = os.path.join(PKG, "bind", "hs2_torch.cpp")
+BIND_NAME = "_hs2_torch"
+
+
+def bind_path() -> str:
+    """The in-tree torch binding module (its file name carries the interpreter's extension suffix)."""
+    import sysconfig
+    return os.path.join(PKG, BIND_NAME + sysconfig.get_config_var("EXT_SUFFIX"))
+
+
+def build_binding(force: bool = False, verbose: bool = False) -> str:
+    """Compiles the torch marshalling module with torch's extension builder (host C++ only)."""
+    target = bind_path()
+    if not force and not _stale(target, [BIND_SRC]):
+        return target
+    from torch.utils import cpp_extension
+    bdir = os.path.join(OUT_DIR, "bind")
+    os.makedirs(bdir, exist_ok=True)
+    cpp_extension.load(name=BIND_NAME, sources=[BIND_SRC], build_directory=bdir, extra_cflags=["-O2"],
+                       verbose=verbose, is_python_module=True)
+    built = [f for f in os.listdir(bdir) if f.startswith(BIND_NAME) and f.endswith(".so")]
+    if not built:
+        raise RuntimeError("the torch binding module was not produced")
+    tmp = target + f".tmp{os.getpid()}"
+    shutil.copyfile(os.path.join(bdir, built[0]), tmp)
+    os.replace(tmp, target)
+    return target
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)
+    print(build_binding(force="--force" in sys.argv, verbose="-v" in sys.argv))

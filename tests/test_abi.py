@@ -116,3 +116,23 @@ def test_fp8_workspace_queries_and_argument_checks():
     assert L.hs2_sparse_attn_fp8kv(a, a, a, 1.0, 1.0, a, 1, 1, 1000, a, 4, 10, 64, 128, 1152, 0.1, a, None, a,
                                    1 << 20, None) == hs2.ERR_INVALID_ARG
     assert L.hs2_selftest_e4m3(a, a, a, 3, None) == hs2.ERR_INVALID_ARG  # odd count
+
+
+def test_marshalling_module_checks_arguments_before_any_call():
+    """The C++ marshalling module of the binding (its fast path, taken when every buffer is given)
+    loads, and rejects host tensors, wrong dtypes and shapes with ValueError without calling the
+    library."""
+    import torch
+    import long_context_mqa_b200 as hs2
+    assert hs2._fast is not None, "the marshalling module was not built"
+    q = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 10, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 64)
+    idx = torch.zeros(1, 1, 1152, dtype=torch.int32)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        hs2.full_attn_select(q, kv, kv, out=q, lse=lse, idx=idx, workspace=ws)
+    with pytest.raises(ValueError):
+        hs2.sparse_attn(q, kv, kv, idx, out=q, workspace=ws)
+    with pytest.raises(ValueError):  # a wrong dtype is reported the same way by the C++ checks
+        hs2._fast.full_attn_select(q.float(), kv, kv, 0.1, 128, 1024, q, lse, idx, ws, 0)
