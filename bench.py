@@ -19,6 +19,7 @@ this host's cores, on a bounded sample of the same workload, extrapolated to a s
 from __future__ import annotations
 
 import argparse
+import ctypes
 import csv
 import io
 import json
@@ -556,15 +557,33 @@ def run_gpu(args):
     outs_e = [torch.empty_like(out) for _ in range(wl.n_sparse)]
     h_outs = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(wl.n_sparse)]
     h2d = (h_in0.numel() + h_in1.numel()) * 2
+    # the new token's K/V rows go from the upload buffer into row Lk - 1 of every sequence (pitch
+    # Lk * d elements) by one 2-D device copy each, through the runtime torch already loaded
+    cudart = ctypes.CDLL("libcudart.so.12")
+    cudart.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_size_t, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+    cudart.cudaMemcpyAsync.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+    up0 = (d_in0.data_ptr(), h_in0.data_ptr(), h_in0.numel() * 2, 1)  # cudaMemcpyHostToDevice
+    last = wl.n_sparse - 1
+    down_last = (h_outs[last].data_ptr(), outs_e[last].data_ptr(), outs_e[last].numel() * 2, 2)  # DeviceToHost
+    copies_done = torch.cuda.Event()
+    row_bytes, pitch = wl.d * 2, wl.Lk * wl.d * 2
+    appends = ((k.data_ptr() + (wl.Lk - 1) * row_bytes, krow_e.data_ptr()),
+               (v.data_ptr() + (wl.Lk - 1) * row_bytes, vrow_e.data_ptr()))
+    d2d = 3  # cudaMemcpyDeviceToDevice
+    step_done = torch.cuda.Event()
     d2h = n_out0 + wl.n_sparse * on * 2
     copy_stream = torch.cuda.Stream(device=dev)
     ev_in1 = torch.cuda.Event()
     ev_layer = [torch.cuda.Event() for _ in range(1 + wl.n_sparse)]
 
     def e2e_step():
-        d_in0.copy_(h_in0, non_blocking=True)
-        k[:, -1:, :].copy_(krow_e)                       # the new token's K/V rows join the cache
-        v[:, -1:, :].copy_(vrow_e)
+        sp = stream.cuda_stream
+        if cudart.cudaMemcpyAsync(*up0, sp):
+            raise RuntimeError("cudaMemcpyAsync failed")
+        for dst, src in appends:                         # the new token's K/V rows join the cache
+            if cudart.cudaMemcpy2DAsync(dst, pitch, src, row_bytes, row_bytes, wl.B, d2d, sp):
+                raise RuntimeError("cudaMemcpy2DAsync failed")
         hs2.full_attn_select(q_e, k, v, scale=wl.scale, out=out_e, lse=lse, idx=idx_e, workspace=ws_full)
         ev_layer[0].record(stream)
         with torch.cuda.stream(copy_stream):
@@ -575,11 +594,18 @@ def run_gpu(args):
         stream.wait_event(ev_in1)
         for i in range(wl.n_sparse):
             hs2.sparse_attn(qs_e[i], k, v, idx_e, scale=wl.scale, out=outs_e[i], workspace=ws_sp[i])
+            if i == last:  # the last layer's output comes back on its own stream, right after it
+                if cudart.cudaMemcpyAsync(*down_last, sp):
+                    raise RuntimeError("cudaMemcpyAsync failed")
+                break
             ev_layer[i + 1].record(stream)
             with torch.cuda.stream(copy_stream):
                 copy_stream.wait_event(ev_layer[i + 1])
                 h_outs[i].copy_(outs_e[i], non_blocking=True)
-        copy_stream.synchronize()                       # the caller reads the step's results
+        copies_done.record(copy_stream)
+        step_done.record(stream)
+        while not (step_done.query() and copies_done.query()):  # the caller waits for the results
+            pass
 
     e2e_steps = max(10, min(args.steps, 200))
     for _ in range(3):
@@ -650,7 +676,7 @@ def run_gpu(args):
             "roofline": roofline, "step_roofline": step_roof, "kernel_ms_per_step": breakdown,
             "sparse_gather": sparse_gather,
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps, "note": "public Python API; per step from pinned memory: the full layer's query and the new token's K/V rows (one copy, then written into the cache), the sparse layers' queries (one copy on a second stream, overlapping the full layer); each layer's results copied back on that stream once the layer is done; the step ends when the last copy has landed"},
+                    "steps": e2e_steps, "note": "public Python API; per step from pinned memory: the full layer's query and the new token's K/V rows (one copy; the rows then written into the cache by a 2-D device copy each), the sparse layers' queries (one copy on a second stream, overlapping the full layer); each layer's results copied back on that stream once the layer is done; the step ends when the last copy has landed (polled)"},
             "gpu_launches": launches_total, "clocks": clocks.summary(),
             "device_status": [status, status_sp], "cpu_baseline": cpu, "selection_check": sel,
             "ragged": ragged, "fp8_kv": fp8, "v1": v1, "prefill": prefill, "backward": backward, "configs": configs,

@@ -33,9 +33,54 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
+// The encoded maps of the last few distinct argument sets, per host thread: a decode loop calls
+// with the same buffers every step, and an encoding is a pure function of its arguments.
+namespace {
+struct TmapEntry {
+  uint64_t key[12];
+  CUtensorMap map;
+  bool used;
+};
+constexpr int kTmapCache = 8;
+thread_local TmapEntry t_tmaps[kTmapCache];
+thread_local int t_tmap_next = 0;
+TmapEntry* tmap_find(const uint64_t (&key)[12]) {
+  for (auto& e : t_tmaps)
+    if (e.used && memcmp(e.key, key, sizeof(key)) == 0) return &e;
+  return nullptr;
+}
+void tmap_store(const uint64_t (&key)[12], const CUtensorMap& m) {
+  TmapEntry& e = t_tmaps[t_tmap_next];
+  t_tmap_next = (t_tmap_next + 1) % kTmapCache;
+  memcpy(e.key, key, sizeof(key));
+  e.map = m;
+  e.used = true;
+}
+}  // namespace
+
+static bool make_tmap_3d_uncached(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                                  uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner,
+                                  uint32_t box_rows, bool swizzle128, int elem_bytes);
+
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                   uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner, uint32_t box_rows,
                   bool swizzle128, int elem_bytes) {
+  const uint64_t key[12] = {3, (uint64_t)(uintptr_t)base, inner, rows, batch, row_stride_el, batch_stride_el,
+                            box_inner, box_rows, (uint64_t)swizzle128, (uint64_t)elem_bytes, 0};
+  if (const TmapEntry* e = tmap_find(key)) {
+    *m = e->map;
+    return true;
+  }
+  if (!make_tmap_3d_uncached(m, base, inner, rows, batch, row_stride_el, batch_stride_el, box_inner, box_rows,
+                             swizzle128, elem_bytes))
+    return false;
+  tmap_store(key, *m);
+  return true;
+}
+
+static bool make_tmap_3d_uncached(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                                  uint64_t row_stride_el, uint64_t batch_stride_el, uint32_t box_inner,
+                                  uint32_t box_rows, bool swizzle128, int elem_bytes) {
   auto enc = get_encoder();
   if (!enc || (elem_bytes != 1 && elem_bytes != 2)) return false;
   cuuint64_t dims[3] = {inner, rows, batch};
@@ -50,6 +95,11 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t row
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_el,
                   uint32_t box_inner, uint32_t box_rows) {
+  const uint64_t key[12] = {2, (uint64_t)(uintptr_t)base, inner, rows, row_stride_el, box_inner, box_rows, 0, 0, 0, 0, 0};
+  if (const TmapEntry* e = tmap_find(key)) {
+    *m = e->map;
+    return true;
+  }
   auto enc = get_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -58,7 +108,7 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t row
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS ? (tmap_store(key, *m), true) : false;
 }
 
 static long long g_wait_ns = -1;
