@@ -129,9 +129,13 @@ struct PageRun {
 
 // the first phase-1 (sampled) tile at or after local tile lt
 __device__ __forceinline__ int first_sample(int lt, int st) { return (lt + st - 1) / st * st; }
-// phase 1 of sequence b takes every st-th tile: about `target` tiles (every tile when target is 0)
+// phase 1 of sequence b takes every st-th tile: about `target` tiles (every tile when target is
+// 0), and at most an eighth of the sequence's tiles (at least 4): a short sequence of a ragged
+// batch sampled in full would give the CTAs covering it most of the first pass while every other
+// CTA waits at the grid barrier
 __device__ __forceinline__ int sample_stride(const Sched& S, int b, int target) {
   const int tiles = (int)(S.seq_start[b + 1] - S.seq_start[b]);
+  if (target > 0 && target > tiles / 8) target = tiles / 8 > 4 ? tiles / 8 : 4;
   return target > 0 && tiles / target > 1 ? tiles / target : 1;
 }
 
