@@ -138,9 +138,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int local = 0;
     for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++local) {
       const int ab = local & 1;
-      int okw = 1;
-      if (lane == 0) okw = wait_abortable(&acc_full[ab], (local >> 1) & 1, limit, &abort_flag, p.st, 521) ? 1 : 0;
-      okw = __shfl_sync(0xffffffffu, okw, 0);
+      int okw = __all_sync(0xffffffffu, mbar_try_wait(smem_u32(&acc_full[ab]), (local >> 1) & 1));
+      if (!okw) {  // not complete yet: lane 0 waits (bounded) and passes the answer on
+        if (lane == 0) okw = wait_abortable(&acc_full[ab], (local >> 1) & 1, limit, &abort_flag, p.st, 521) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+      }
       if (!okw) break;
       tc_fence_after();
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;

@@ -74,6 +74,7 @@ __device__ __forceinline__ bool wait_abortable(uint64_t* bar, uint32_t parity, l
 }
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit, volatile int* abort_flag,
                                           DevStatus* st, unsigned where) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(smem_u32(bar), parity))) return true;  // completed: no divergent wait
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = wait_abortable(bar, parity, limit, abort_flag, st, where) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
