@@ -18,13 +18,16 @@
 //   candidate buffer in shared memory of unique 64-bit keys (score bits << 32 | ~index: larger key
 //   == higher score, then lower index). A key enters only if it beats the query's current
 //   threshold; when the buffer nears capacity an exact MSB radix select keeps the top-k and
-//   raises the threshold. Keys are visited newest first. At the end the kept indices plus the
-//   forced window are sorted ascending into idx.
+//   raises the threshold. Keys are visited newest first. At the end the kept indices are
+//   written ascending (a bitmap over the candidate range and one prefix count; a sort only past
+//   the bitmap's capacity), then the forced window.
 //
 // Both kernels are persistent: CTAs take work items in order of decreasing causal work, round
-// robin. Warp roles (320 threads): warp 0 TMA producer, warp 1 tcgen05 issuer + TMEM owner,
-// warps 2..5 warpgroup A, warps 6..9 warpgroup B (warp w reads TMEM lanes 32*(w%4)..+31).
-// Every wait is bounded and reports a timeout through the status word.
+// robin. Warp roles: warp 0 TMA producer, warp 1 tcgen05 issuer + TMEM owner, then the softmax
+// warpgroups (warp w reads TMEM lanes 32*(w%4)..+31): fa_fwd (320 threads) warps 2..5 and 6..9
+// for tiles A and B; score_select (576 threads) four warpgroups, each owning a quarter of the 256
+// (query, head) columns, i.e. a quarter of the item's queries. Every wait is bounded and reports
+// a timeout through the status word.
 #include "decode.h"
 #include "host_util.h"
 #include "prefill.h"
