@@ -445,19 +445,22 @@ __global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
       if (lane == 0) { mbar_arrive(&ka_full[kb]); mbar_arrive(&r_empty[slot]); }
       return true;
     };
-    auto widen_v = [&](uint32_t item, bool valid_row) -> bool {
+    // a V tile in two steps: the row's 8 chunks into registers (the e4m3 slot is then free), and
+    // later, once the previous PV has read the f16 buffer, widened into it
+    auto load_v = [&](uint32_t item, bool valid_row, uint4 (&x)[D / 16]) -> bool {
       const int slot = (int)(item % NR);
       if (!warp_wait_bar(&r_full[slot], (item / NR) & 1, limit, &abort_flag, p.st, 229)) return false;
-      // the row's 8 chunks in registers first (the e4m3 slot is then free), then the f16 buffer
-      // once the previous PV has read it
-      const uint32_t src = smem_u32(sR + slot * SLOT_BYTES), dst = smem_u32(sV);
-      uint4 x[D / 16];
+      const uint32_t src = smem_u32(sR + slot * SLOT_BYTES);
 #pragma unroll
       for (int c = 0; c < D / 16; ++c)
         x[c] = valid_row ? ld_shared_v4(src + sw128_off(row, c)) : make_uint4(0u, 0u, 0u, 0u);
       __syncwarp();
       if (lane == 0) mbar_arrive(&r_empty[slot]);
+      return true;
+    };
+    auto store_v = [&](const uint4 (&x)[D / 16]) -> bool {
       if (!warp_wait_bar(&v16_empty, (nv & 1) ^ 1, limit, &abort_flag, p.st, 232)) return false;
+      const uint32_t dst = smem_u32(sV);
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
         uint32_t h[8];
@@ -500,11 +503,16 @@ __global__ void __launch_bounds__(F8 ? NTHREADS_F8 : NTHREADS, 1)
         auto v_valid = [&](uint32_t x) {  // row of tile x (descending from t) inside the sequence
           return (t - (long long)x - (long long)S.seq_start[b]) * TILE + row < (long long)n_b;
         };
+        // ring items K(0) K(1) V(0) K(2) V(1) ... K(n-1) V(n-2) V(n-1), taken in that order; V(x)
+        // is widened after K(x + 2), so that the wait for PV(x - 1) overlaps a K tile's work
+        if (ok && !widen_k(base, js)) ok = false;
+        if (ok && n > 1 && !widen_k(base + 1, js + 1)) ok = false;
         for (uint32_t x = 0; x < n && ok; ++x) {
-          if (!widen_k(base + (x == 0 ? 0u : 2 * x - 1), js + x)) { ok = false; break; }
-          if (x > 0 && !widen_v(base + 2 * x, v_valid(x - 1))) { ok = false; break; }
+          uint4 vr[D / 16];
+          if (!load_v(x == n - 1 ? base + 2 * n - 1 : base + 2 * x + 2, v_valid(x), vr)) { ok = false; break; }
+          if (x + 2 < n && !widen_k(base + 2 * x + 3, js + x + 2)) { ok = false; break; }
+          if (!store_v(vr)) { ok = false; break; }
         }
-        if (ok && !widen_v(base + 2 * n - 1, v_valid(n - 1))) ok = false;
         ri = base + 2 * n;
         js += n;
         jp += n;
