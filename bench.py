@@ -607,8 +607,9 @@ def run_gpu(args):
         while not (step_done.query() and copies_done.query()):  # the caller waits for the results
             pass
 
-    e2e_steps = max(10, min(args.steps, 200))
-    for _ in range(3):
+    # enough steps that a single host hiccup (a page fault, a scheduler tick) does not set the number
+    e2e_steps = max(200, min(args.steps, 1000))
+    for _ in range(10):
         e2e_step()
     _barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
